@@ -1,0 +1,445 @@
+"""Benchmark of Echo's compensated 4-bit all-reduce on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload large|llama|depth|tiny] [--fixup exit|side|deferred]
+                    [--uncompensated] [--mode step|sweep|overlap|depth-chain]
+
+Default (mode "step"): one step = one echo_allreduce call (entry + reduce +
+exit kernels) of P=8 virtual ranks x 2^29 bf16 elements (1 GiB) per rank,
+G=128, compensator on, inputs resident in HBM.  Prints ONE JSON line with
+the input GB/s per call (all ranks' input bytes / call time), the whole-call
+fraction of the HBM roofline (minimal bytes of a call / measured copy
+bandwidth / call time), the roofline of the dominant kernel (echo_entry)
+from CUDA events on its launch stream, the end-to-end figure through the
+host-buffer C call (host<->device copies inside the timed region), the
+oracle timed on host cores as the CPU baseline, and the SM clocks sampled
+during the timed region.
+
+With --gpus N under torchrun every rank runs its own independent call on
+its own GPU (the path is emulated on one GPU; there is no cross-GPU data
+exchange), timed between barriers and reported as the max over ranks.
+
+--impl reference times the CPU oracle on bounded samples of the same
+workload (rank 0 only) and prints the same JSON line with "impl":
+"reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_error_compensated_echo_b200 import workloads as W  # noqa: E402
+
+METRIC = "compensated 4-bit reduce input GB/s & % HBM roofline, P=8 virtual ranks, 1 GB/rank"
+UNIT = "GB/s"
+# fix-up placement timed by default (bit-identical to the others; fewest bytes)
+BENCH_FIXUP = "deferred"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_FILES = ("bit_error_compensated_echo_b200/csrc/echo_kernels.cuh",
+                "bit_error_compensated_echo_b200/csrc/echo.cu")
+
+WORKLOADS = {"large": W.LARGE, "llama": W.LLAMA, "depth": W.DEPTH, "tiny": W.TINY}
+
+
+# ------------------------------------------------------------ byte counts
+
+def transport_bytes_per_elem(G: int) -> float:
+    """q: packed codes (1/2 byte) + fp32 scale per G elements."""
+    return 0.5 + 4.0 / G
+
+
+def call_min_bytes(P: int, N: int, G: int, comp: bool) -> float:
+    """Minimal HBM bytes of one call when each stage boundary is an HBM
+    wire: read x, (read+write both states), write the P outputs, write and
+    read the entry transport, write and read the reduced transport once,
+    (write e_req and read it once)."""
+    q = transport_bytes_per_elem(G)
+    if comp:
+        return P * N * (2 + 16 + 2 + 2 * q) + N * (2 * q + 8)
+    return P * N * (2 + 2 + 2 * q) + N * 2 * q
+
+
+def entry_bytes(P: int, N: int, G: int, comp: bool, fixup: str) -> float:
+    """Algorithmic bytes of one echo_entry launch: read x (2 B), read and
+    write both states (16 B), write codes + scales (q B) per rank-element;
+    in deferred mode also read e_req of each rank's own chunk (4 B per
+    element of N)."""
+    q = transport_bytes_per_elem(G)
+    b = P * N * (2 + q)
+    if comp:
+        b += P * N * 16
+        if fixup == "deferred":
+            b += N * 4
+    return b
+
+
+def reduce_bytes(P: int, N: int, G: int, comp: bool) -> float:
+    q = transport_bytes_per_elem(G)
+    return P * N * q + N * q + (N * 4 if comp else 0)
+
+
+def exit_bytes(P: int, N: int, G: int, comp: bool, fixup: str) -> float:
+    q = transport_bytes_per_elem(G)
+    b = N * q + P * N * 2
+    if comp and fixup == "exit":
+        b += N * (4 + 16)
+    return b
+
+
+# ------------------------------------------------------------ environment
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_FILES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, comp: bool, fixup: str):
+    """DRAM bytes per echo_entry launch from the committed ncu summary, if
+    it was captured from the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "echo_entry_traffic.md")
+    if not os.path.exists(path):
+        return None
+    want = "%s comp=%d fixup=%s" % (workload, int(comp), fixup)
+    src = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            if line.startswith("traffic:"):
+                # traffic: <workload> comp=<0|1> fixup=<mode> src=<hash> bytes=<int>
+                parts = line.split()
+                key = " ".join(parts[1:4])
+                kv = dict(p.split("=", 1) for p in parts[4:] if "=" in p)
+                if key == want and kv.get("src") == src:
+                    return float(kv["bytes"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi SM clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="echo_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [s.strip() for s in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, ws: int, device) -> float:
+    if ws == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, ws: int, device) -> float:
+    if ws == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate(per_rank_ms, per_rank_bytes):
+    """Whole-job throughput: bytes of all ranks / slowest rank's time."""
+    t = max(per_rank_ms)
+    return sum(per_rank_bytes) / (t / 1e3) / 1e9, t
+
+
+# ------------------------------------------------------------ CPU baseline
+
+def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: int = 7):
+    """Time the oracle (as it stands, one host thread) on ``ncols`` group
+    columns of workload ``w``; inputs are the device inputs at those columns
+    when given, else a host draw of the same distribution."""
+    import oracle
+    cols = W.column_sample(w, ncols, seed=seed)
+    idx = W.column_elements(cols, w.G)
+    if x_dev is not None:
+        ti = torch.from_numpy(idx).to(x_dev.device)
+        xb = W.bf16_bits(x_dev.index_select(1, ti))
+    else:
+        small = W.with_size(w, rows=1, hidden=idx.size)
+        xb = W.bf16_bits(W.generate(small, 0, "cpu"))
+    prm = oracle.Params(P=w.P, N=w.N, G=w.G, compensate=comp)
+    mf = np.zeros((w.P, idx.size), np.float32)
+    ms = np.zeros_like(mf)
+    t0 = time.perf_counter()
+    oracle.allreduce(prm, xb, mf, ms, cols)
+    dt = time.perf_counter() - t0
+    nbytes = 2 * w.P * idx.size
+    return nbytes / dt / 1e9, dt, cols.size
+
+
+# ------------------------------------------------------------ modes
+
+def run_step_mode(args, ws, rank, local):
+    from bit_error_compensated_echo_b200.api import EchoPlan
+
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    comp = not args.uncompensated
+    fixup = args.fixup
+    P, N, G = w.P, w.N, w.G
+    peak, peak_kind = load_peaks()
+
+    x = torch.empty((P, N), dtype=torch.bfloat16, device=dev)
+    W.generate(w, rank, dev, out=x)
+    out = torch.empty_like(x)
+    plan = EchoPlan(P, N, G, compensate=comp, fixup=fixup, device=local)
+    side = torch.cuda.Stream(device=dev) if fixup == "side" else None
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        plan.allreduce(x, out=out, side_stream=side)
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    plan.profile_enable(True)
+    plan.profile_read(reset=True)
+    barrier(ws)
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        plan.allreduce(x, out=out, side_stream=side)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(ws)
+    prof = plan.profile_read(reset=True)
+    plan.profile_enable(False)
+    clk = clocks.stop() if rank == 0 else None
+    ms_local = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms_local, ws, dev)
+    total_in = sum_over_ranks(2.0 * P * N, ws, dev)
+    value = total_in / (ms / 1e3) / 1e9
+
+    # end to end: host buffers through echo_allreduce_host
+    e2e = None
+    if not args.no_e2e:
+        xh = torch.empty((P, N), dtype=torch.bfloat16, pin_memory=True)
+        xh.copy_(x)
+        yh = torch.empty((P, N), dtype=torch.bfloat16, pin_memory=True)
+        with EchoPlan(P, N, G, compensate=comp, fixup=fixup, device=local) as hp:
+            for _ in range(args.warmup):
+                hp.allreduce_host(xh, yh)
+            torch.cuda.synchronize(dev)
+            barrier(ws)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.e2e_steps):
+                hp.allreduce_host(xh, yh)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier(ws)
+            e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, ws, dev)
+        e2e = {"value": round(total_in / (e_ms / 1e3) / 1e9, 3), "unit": UNIT,
+               "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": 2 * P * N,
+               "d2h_bytes_per_step": 2 * P * N}
+        del xh, yh
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        gbs, dt, ncols = oracle_sample_run(w, comp, args.cpu_cols, x_dev=x)
+        cpu = {"value": round(gbs, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": "%d of %d group columns (x %d ranks x G=%d) of the same inputs, one "
+                         "call from zero state, %.1f s on one host thread" %
+                         (ncols, N // G, P, G, dt)}
+
+    if rank == 0:
+        calls = prof["calls"]
+        entry_ms = prof["entry_ms"] / max(calls, 1)
+        eb = entry_bytes(P, N, G, comp, fixup)
+        achieved = eb / (entry_ms / 1e3) / 1e9
+        bmin = call_min_bytes(P, N, G, comp)
+        traffic = ncu_traffic(w.name, comp, fixup)
+        line = {
+            "metric": METRIC if comp else METRIC.replace("compensated", "uncompensated"),
+            "value": round(value, 3), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, int4 transport, f32 sum+state",
+            "data": "synthetic (seeded N(0,0.5^2) bf16 draws, no dataset)",
+            "config": {"workload": w.name, "P": P, "N_per_rank": N, "G": G,
+                       "compensate": comp, "fixup": fixup, "alpha": 0.5, "beta_fast": 0.5,
+                       "beta_slow": 0.95, "l2": "inputs larger than L2 (%.1f GiB of x per step)"
+                       % (2 * P * N / 2**30), "parallelism": "replicas" if ws > 1 else "1 GPU"},
+            "call_roofline": {"min_bytes": bmin, "achieved_gbs": round(bmin / (ms / 1e3) / 1e9, 1),
+                              "peak": peak, "frac": round(bmin / (ms / 1e3) / 1e9 / peak, 4),
+                              "time_at_peak_ms": round(bmin / peak / 1e6, 3)},
+            "roofline": {"kernel": "echo_entry", "bound": "hbm", "achieved": round(achieved, 1),
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "algorithmic_bytes": eb, "avg_launch_ms": round(entry_ms, 4)},
+            "kernels_ms": {k: round(prof[k] / max(calls, 1), 4)
+                           for k in ("entry_ms", "reduce_ms", "exit_ms", "fixup_ms")},
+            "gpu_launches": int(prof["launches"]),
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    plan.close()
+
+
+def run_reference(args, ws, rank):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    comp = not args.uncompensated
+    for i in range(args.warmup):
+        oracle_sample_run(w, comp, args.ref_cols, seed=100 + i)
+    times, nbytes = [], 0
+    for i in range(args.steps):
+        gbs, dt, ncols = oracle_sample_run(w, comp, args.ref_cols, seed=1000 + i)
+        times.append(dt)
+        nbytes = 2 * w.P * ncols * w.G
+    ms = 1e3 * sum(times) / len(times)
+    value = nbytes / (ms / 1e3) / 1e9
+    sample = ("%d of %d group columns (x %d ranks x G=%d) per step, host draw of the same "
+              "distribution, one call from zero state" % (args.ref_cols + 2, w.N // w.G, w.P, w.G))
+    line = {
+        "metric": METRIC if comp else METRIC.replace("compensated", "uncompensated"),
+        "value": round(value, 6), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, int4 transport, f32 sum+state",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "P": w.P, "N_per_rank": w.N, "G": w.G,
+                   "compensate": comp},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="large")
+    ap.add_argument("--fixup", choices=("exit", "side", "deferred"), default=BENCH_FIXUP)
+    ap.add_argument("--uncompensated", action="store_true")
+    ap.add_argument("--mode", choices=("step",), default="step")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-cols", type=int, default=65536,
+                    help="group columns of the CPU-baseline sample")
+    ap.add_argument("--ref-cols", type=int, default=16384,
+                    help="group columns per step of the reference arm")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+
+    ws, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank)
+        else:
+            run_step_mode(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

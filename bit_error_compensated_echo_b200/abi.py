@@ -1,0 +1,179 @@
+"""ctypes binding of the C ABI in include/echo.h -- same names, argument
+marshalling only.
+
+Every function here forwards to the function of the same name in
+libecho_b200.so and raises ``EchoError`` (carrying the status code) when it
+returns anything but ECHO_OK.  Pointers are passed as Python ints (device
+or host addresses), streams as cudaStream_t handles (ints; 0 is the legacy
+default stream).  Importing this module loads the library and fails loudly
+if it has not been built: there is no other implementation to fall back on.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libecho_b200.so")
+
+ECHO_MAX_RANKS = 8
+
+STATUS = {
+    0: "ECHO_OK", 1: "ECHO_ERR_INVALID_ARG", 2: "ECHO_ERR_SHAPE",
+    3: "ECHO_ERR_ALIGNMENT", 4: "ECHO_ERR_UNSUPPORTED", 5: "ECHO_ERR_OOM",
+    6: "ECHO_ERR_CUDA", 7: "ECHO_ERR_TIMEOUT",
+}
+ECHO_OK, ECHO_ERR_INVALID_ARG, ECHO_ERR_SHAPE, ECHO_ERR_ALIGNMENT = 0, 1, 2, 3
+ECHO_ERR_UNSUPPORTED, ECHO_ERR_OOM, ECHO_ERR_CUDA, ECHO_ERR_TIMEOUT = 4, 5, 6, 7
+
+ECHO_FIXUP_EXIT, ECHO_FIXUP_SIDE, ECHO_FIXUP_DEFERRED = 0, 1, 2
+FIXUP_MODES = {"exit": ECHO_FIXUP_EXIT, "side": ECHO_FIXUP_SIDE,
+               "deferred": ECHO_FIXUP_DEFERRED}
+
+
+class EchoError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s" % (where, STATUS.get(status, "status %d" % status)))
+
+
+class echo_config(ctypes.Structure):
+    _fields_ = [("P", ctypes.c_int32), ("G", ctypes.c_int32), ("N", ctypes.c_int64),
+                ("compensate", ctypes.c_int32), ("alpha", ctypes.c_float),
+                ("beta_fast", ctypes.c_float), ("beta_slow", ctypes.c_float),
+                ("device", ctypes.c_int32), ("fixup", ctypes.c_int32)]
+
+
+class echo_debug_view(ctypes.Structure):
+    _fields_ = [("m_fast", ctypes.c_void_p), ("m_slow", ctypes.c_void_p),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("rcodes", ctypes.c_void_p), ("rscales", ctypes.c_void_p),
+                ("e_req", ctypes.c_void_p), ("fixup_pending", ctypes.c_int32)]
+
+
+class echo_profile(ctypes.Structure):
+    _fields_ = [("calls", ctypes.c_int64), ("entry_ms", ctypes.c_double),
+                ("reduce_ms", ctypes.c_double), ("exit_ms", ctypes.c_double),
+                ("fixup_ms", ctypes.c_double), ("launches", ctypes.c_int64)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            "libecho_b200.so is not built (%s); run "
+            "`python -m bit_error_compensated_echo_b200.build` -- the CUDA "
+            "library is the only implementation of this path" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    vp, st = ctypes.c_void_p, ctypes.c_int
+    sig = {
+        "echo_config_default": (None, [ctypes.POINTER(echo_config)]),
+        "echo_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(echo_config)]),
+        "echo_plan_create": (st, [ctypes.POINTER(vp), ctypes.POINTER(echo_config)]),
+        "echo_plan_destroy": (st, [vp]),
+        "echo_allreduce": (st, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, vp]),
+        "echo_allreduce_host": (st, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp]),
+        "echo_reset_state": (st, [vp, vp]),
+        "echo_get_state": (st, [vp, vp, vp, vp]),
+        "echo_set_state": (st, [vp, vp, vp, vp]),
+        "echo_debug_view_get": (st, [vp, ctypes.POINTER(echo_debug_view)]),
+        "echo_profile_enable": (st, [vp, ctypes.c_int32]),
+        "echo_profile_read": (st, [vp, ctypes.POINTER(echo_profile), ctypes.c_int32]),
+        "echo_launches_per_call": (ctypes.c_int32, [vp]),
+        "echo_status_string": (ctypes.c_char_p, [st]),
+        "echo_abi_version": (ctypes.c_int32, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+def _check(status: int, where: str):
+    if status != ECHO_OK:
+        raise EchoError(status, where)
+
+
+def _ptr_array(ptrs: Sequence[int]):
+    arr = (ctypes.c_void_p * max(1, len(ptrs)))()
+    for i, p in enumerate(ptrs):
+        arr[i] = p
+    return arr
+
+
+def echo_config_default() -> echo_config:
+    cfg = echo_config()
+    lib.echo_config_default(ctypes.byref(cfg))
+    return cfg
+
+
+def echo_workspace_bytes(cfg: echo_config) -> int:
+    return int(lib.echo_workspace_bytes(ctypes.byref(cfg)))
+
+
+def echo_plan_create(cfg: echo_config) -> int:
+    h = ctypes.c_void_p()
+    _check(lib.echo_plan_create(ctypes.byref(h), ctypes.byref(cfg)), "echo_plan_create")
+    return h.value
+
+
+def echo_plan_destroy(plan: int) -> None:
+    _check(lib.echo_plan_destroy(plan), "echo_plan_destroy")
+
+
+def echo_allreduce(plan: int, in_device: Sequence[int], out_device: Sequence[int],
+                   stream: int = 0, side_stream: int = 0) -> None:
+    _check(lib.echo_allreduce(plan, _ptr_array(in_device), _ptr_array(out_device),
+                              stream or None, side_stream or None), "echo_allreduce")
+
+
+def echo_allreduce_host(plan: int, in_host: Sequence[int], out_host: Sequence[int],
+                        stream: int = 0) -> None:
+    _check(lib.echo_allreduce_host(plan, _ptr_array(in_host), _ptr_array(out_host),
+                                   stream or None), "echo_allreduce_host")
+
+
+def echo_reset_state(plan: int, stream: int = 0) -> None:
+    _check(lib.echo_reset_state(plan, stream or None), "echo_reset_state")
+
+
+def echo_get_state(plan: int, m_fast_device: int, m_slow_device: int, stream: int = 0) -> None:
+    _check(lib.echo_get_state(plan, m_fast_device, m_slow_device, stream or None),
+           "echo_get_state")
+
+
+def echo_set_state(plan: int, m_fast_device: int, m_slow_device: int, stream: int = 0) -> None:
+    _check(lib.echo_set_state(plan, m_fast_device, m_slow_device, stream or None),
+           "echo_set_state")
+
+
+def echo_debug_view_get(plan: int) -> echo_debug_view:
+    v = echo_debug_view()
+    _check(lib.echo_debug_view_get(plan, ctypes.byref(v)), "echo_debug_view_get")
+    return v
+
+
+def echo_profile_enable(plan: int, on: bool) -> None:
+    _check(lib.echo_profile_enable(plan, int(bool(on))), "echo_profile_enable")
+
+
+def echo_profile_read(plan: int, reset: bool = False) -> echo_profile:
+    p = echo_profile()
+    _check(lib.echo_profile_read(plan, ctypes.byref(p), int(bool(reset))), "echo_profile_read")
+    return p
+
+
+def echo_launches_per_call(plan: int) -> int:
+    return int(lib.echo_launches_per_call(plan))
+
+
+def echo_status_string(status: int) -> str:
+    return lib.echo_status_string(status).decode()
+
+
+def echo_abi_version() -> int:
+    return int(lib.echo_abi_version())

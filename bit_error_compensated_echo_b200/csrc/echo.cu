@@ -1,0 +1,535 @@
+// echo.cu -- the plan and the C ABI declared in include/echo.h.
+//
+// A plan owns one device allocation carved into the EMA states, the entry
+// transport (packed codes + scales of all P ranks: the 4-bit "wire" of the
+// reduce-scatter), the reduced transport (the wire of the all-gather) and
+// e_req.  A call launches three kernels on the caller's stream -- entry,
+// reduce, exit -- plus, in side-stream mode, the owner fix-up on the side
+// stream.  Host code here only validates, carves memory, orders streams and
+// launches: every step of the arithmetic runs in echo_kernels.cuh.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "echo.h"
+#include "echo_kernels.cuh"
+
+using namespace echo;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+    size_t m_fast, m_slow, codes, scales, rcodes, rscales, e_req, total;
+};
+
+Layout layout_of(const echo_config &c) {
+    Layout L{};
+    const size_t N = (size_t)c.N, P = (size_t)c.P, G = (size_t)c.G;
+    const bool comp = c.compensate != 0;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = off;
+        off += align_up(bytes);
+        return at;
+    };
+    L.m_fast = comp ? take(P * N * 4) : 0;
+    L.m_slow = comp ? take(P * N * 4) : 0;
+    L.codes = take(P * N / 2);
+    L.scales = take(P * (N / G) * 4);
+    L.rcodes = take(N / 2);
+    L.rscales = take((N / G) * 4);
+    L.e_req = comp ? take(N * 4) : 0;
+    L.total = off;
+    return L;
+}
+
+echo_status validate(const echo_config *c) {
+    if (!c) return ECHO_ERR_INVALID_ARG;
+    if (c->P < 1 || c->P > ECHO_MAX_RANKS) return ECHO_ERR_UNSUPPORTED;
+    if (c->G != 32 && c->G != 64 && c->G != 128) return ECHO_ERR_UNSUPPORTED;
+    if (c->N <= 0 || c->N % ((int64_t)c->P * c->G) != 0) return ECHO_ERR_SHAPE;
+    auto unit = [](float v) { return std::isfinite(v) && v >= 0.0f && v <= 1.0f; };
+    if (!unit(c->alpha) || !unit(c->beta_fast) || !unit(c->beta_slow))
+        return ECHO_ERR_INVALID_ARG;
+    if (c->compensate != 0 && c->compensate != 1) return ECHO_ERR_INVALID_ARG;
+    if (c->fixup < ECHO_FIXUP_EXIT || c->fixup > ECHO_FIXUP_DEFERRED)
+        return ECHO_ERR_INVALID_ARG;
+    if (c->device < 0) return ECHO_ERR_INVALID_ARG;
+    return ECHO_OK;
+}
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+    int prev = -1;
+    cudaError_t err = cudaSuccess;
+    explicit DeviceGuard(int dev) {
+        err = cudaGetDevice(&prev);
+        if (err == cudaSuccess && prev != dev) err = cudaSetDevice(dev);
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+struct ProfRecord {
+    cudaEvent_t ev[6];   // entry start, entry end, reduce end, exit end, fixup start, fixup end
+    bool side;
+};
+
+}  // namespace
+
+struct echo_plan {
+    echo_config cfg;
+    Layout L;
+    int64_t n_vec = 0, chunk_vec = 0;
+    Consts k{};
+    char *ws = nullptr;
+    float *m_fast = nullptr, *m_slow = nullptr, *scales = nullptr, *rscales = nullptr,
+          *e_req = nullptr;
+    uint32_t *codes = nullptr, *rcodes = nullptr;
+    bool pending = false;            // deferred fix-up not yet applied
+    bool side_inflight = false;      // a side-stream fix-up may still run
+    cudaEvent_t ev_reduced = nullptr, ev_side_done = nullptr;
+    void *stage = nullptr;           // host-call staging: [P][N] in, [P][N] out
+    bool profiling = false;
+    std::vector<ProfRecord> records;
+    std::vector<cudaEvent_t> pool;
+    echo_profile totals{};
+};
+
+namespace {
+
+echo_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return ECHO_OK;
+    if (e == cudaErrorMemoryAllocation) return ECHO_ERR_OOM;
+    return ECHO_ERR_CUDA;
+}
+
+#define ECHO_TRY(expr)                                   \
+    do {                                                 \
+        cudaError_t e_ = (expr);                         \
+        if (e_ != cudaSuccess) return from_cuda(e_);     \
+    } while (0)
+
+cudaEvent_t take_event(echo_plan *p) {
+    if (!p->pool.empty()) {
+        cudaEvent_t e = p->pool.back();
+        p->pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+template <int G, bool COMP, bool DEFER>
+void launch_entry_t(echo_plan *p, const InPtrs &x, cudaStream_t st) {
+    dim3 grid((unsigned)((p->n_vec + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
+    echo_entry_kernel<G, COMP, DEFER><<<grid, kThreads, 0, st>>>(
+        x, p->m_fast, p->m_slow, p->codes, p->scales, p->e_req, p->n_vec, p->chunk_vec, p->k);
+}
+
+template <int G>
+void launch_entry_g(echo_plan *p, const InPtrs &x, cudaStream_t st, bool defer) {
+    if (!p->cfg.compensate) launch_entry_t<G, false, false>(p, x, st);
+    else if (defer) launch_entry_t<G, true, true>(p, x, st);
+    else launch_entry_t<G, true, false>(p, x, st);
+}
+
+void launch_entry(echo_plan *p, const InPtrs &x, cudaStream_t st, bool defer) {
+    switch (p->cfg.G) {
+        case 32: launch_entry_g<32>(p, x, st, defer); break;
+        case 64: launch_entry_g<64>(p, x, st, defer); break;
+        default: launch_entry_g<128>(p, x, st, defer); break;
+    }
+}
+
+template <int G, int P>
+void launch_reduce_t(echo_plan *p, cudaStream_t st) {
+    dim3 grid((unsigned)((p->chunk_vec + kThreads - 1) / kThreads), (unsigned)P);
+    if (p->cfg.compensate)
+        echo_reduce_kernel<G, P, true><<<grid, kThreads, 0, st>>>(
+            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec);
+    else
+        echo_reduce_kernel<G, P, false><<<grid, kThreads, 0, st>>>(
+            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec);
+}
+
+template <int G>
+void launch_reduce_g(echo_plan *p, cudaStream_t st) {
+    switch (p->cfg.P) {
+        case 1: launch_reduce_t<G, 1>(p, st); break;
+        case 2: launch_reduce_t<G, 2>(p, st); break;
+        case 3: launch_reduce_t<G, 3>(p, st); break;
+        case 4: launch_reduce_t<G, 4>(p, st); break;
+        case 5: launch_reduce_t<G, 5>(p, st); break;
+        case 6: launch_reduce_t<G, 6>(p, st); break;
+        case 7: launch_reduce_t<G, 7>(p, st); break;
+        default: launch_reduce_t<G, 8>(p, st); break;
+    }
+}
+
+void launch_reduce(echo_plan *p, cudaStream_t st) {
+    switch (p->cfg.G) {
+        case 32: launch_reduce_g<32>(p, st); break;
+        case 64: launch_reduce_g<64>(p, st); break;
+        default: launch_reduce_g<128>(p, st); break;
+    }
+}
+
+template <int G>
+void launch_exit_g(echo_plan *p, const OutPtrs &out, cudaStream_t st, bool fix) {
+    dim3 grid((unsigned)((p->chunk_vec + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
+    if (fix)
+        echo_exit_kernel<G, true><<<grid, kThreads, 0, st>>>(
+            p->rcodes, p->rscales, out, p->cfg.P, p->m_fast, p->m_slow, p->e_req, p->n_vec,
+            p->chunk_vec, p->k);
+    else
+        echo_exit_kernel<G, false><<<grid, kThreads, 0, st>>>(
+            p->rcodes, p->rscales, out, p->cfg.P, p->m_fast, p->m_slow, p->e_req, p->n_vec,
+            p->chunk_vec, p->k);
+}
+
+void launch_exit(echo_plan *p, const OutPtrs &out, cudaStream_t st, bool fix) {
+    switch (p->cfg.G) {
+        case 32: launch_exit_g<32>(p, out, st, fix); break;
+        case 64: launch_exit_g<64>(p, out, st, fix); break;
+        default: launch_exit_g<128>(p, out, st, fix); break;
+    }
+}
+
+void launch_fixup(echo_plan *p, const float *sf, const float *ss, float *df, float *ds, bool apply,
+                  bool only_owner, cudaStream_t st) {
+    dim3 grid((unsigned)((p->chunk_vec + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
+    echo_fixup_kernel<<<grid, kThreads, 0, st>>>(sf, ss, df, ds, p->e_req, p->n_vec, p->chunk_vec,
+                                                 p->cfg.P, apply ? 1 : 0, only_owner ? 1 : 0, p->k);
+}
+
+bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+// Wait (on st) for a side-stream fix-up that may still be writing the state.
+cudaError_t order_after_side(echo_plan *p, cudaStream_t st) {
+    if (!p->side_inflight) return cudaSuccess;
+    return cudaStreamWaitEvent(st, p->ev_side_done, 0);
+}
+
+}  // namespace
+
+extern "C" {
+
+void echo_config_default(echo_config *cfg) {
+    if (!cfg) return;
+    std::memset(cfg, 0, sizeof *cfg);
+    cfg->compensate = 1;
+    cfg->alpha = 0.5f;
+    cfg->beta_fast = 0.5f;
+    cfg->beta_slow = 0.95f;
+    cfg->device = 0;
+    cfg->fixup = ECHO_FIXUP_EXIT;
+}
+
+size_t echo_workspace_bytes(const echo_config *cfg) {
+    if (validate(cfg) != ECHO_OK) return 0;
+    return layout_of(*cfg).total;
+}
+
+echo_status echo_plan_create(echo_plan **out, const echo_config *cfg) {
+    if (!out) return ECHO_ERR_INVALID_ARG;
+    *out = nullptr;
+    echo_status v = validate(cfg);
+    if (v != ECHO_OK) return v;
+
+    DeviceGuard guard(cfg->device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+
+    echo_plan *p = new (std::nothrow) echo_plan();
+    if (!p) return ECHO_ERR_OOM;
+    p->cfg = *cfg;
+    p->L = layout_of(*cfg);
+    p->n_vec = cfg->N / kVec;
+    p->chunk_vec = p->n_vec / cfg->P;
+    p->k.alpha = cfg->alpha;
+    p->k.one_m_alpha = 1.0f - cfg->alpha;
+    p->k.beta_fast = cfg->beta_fast;
+    p->k.one_m_beta_fast = 1.0f - cfg->beta_fast;
+    p->k.beta_slow = cfg->beta_slow;
+    p->k.one_m_beta_slow = 1.0f - cfg->beta_slow;
+
+    cudaError_t e = cudaMalloc((void **)&p->ws, p->L.total);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        delete p;
+        return from_cuda(e);
+    }
+    const bool comp = cfg->compensate != 0;
+    p->m_fast = comp ? (float *)(p->ws + p->L.m_fast) : nullptr;
+    p->m_slow = comp ? (float *)(p->ws + p->L.m_slow) : nullptr;
+    p->codes = (uint32_t *)(p->ws + p->L.codes);
+    p->scales = (float *)(p->ws + p->L.scales);
+    p->rcodes = (uint32_t *)(p->ws + p->L.rcodes);
+    p->rscales = (float *)(p->ws + p->L.rscales);
+    p->e_req = comp ? (float *)(p->ws + p->L.e_req) : nullptr;
+
+    e = cudaEventCreateWithFlags(&p->ev_reduced, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_side_done, cudaEventDisableTiming);
+    if (e == cudaSuccess && comp) {
+        e = cudaMemset(p->m_fast, 0, (size_t)cfg->P * cfg->N * 4);
+        if (e == cudaSuccess) e = cudaMemset(p->m_slow, 0, (size_t)cfg->P * cfg->N * 4);
+        if (e == cudaSuccess) e = cudaMemset(p->e_req, 0, (size_t)cfg->N * 4);
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        echo_plan_destroy(p);
+        return from_cuda(e);
+    }
+    *out = p;
+    return ECHO_OK;
+}
+
+echo_status echo_plan_destroy(echo_plan *p) {
+    if (!p) return ECHO_OK;
+    DeviceGuard guard(p->cfg.device);
+    cudaError_t e = cudaDeviceSynchronize();
+    for (auto &r : p->records)
+        for (auto ev : r.ev)
+            if (ev) cudaEventDestroy(ev);
+    for (auto ev : p->pool) cudaEventDestroy(ev);
+    if (p->ev_reduced) cudaEventDestroy(p->ev_reduced);
+    if (p->ev_side_done) cudaEventDestroy(p->ev_side_done);
+    if (p->stage) cudaFree(p->stage);
+    if (p->ws) cudaFree(p->ws);
+    delete p;
+    return from_cuda(e);
+}
+
+int32_t echo_launches_per_call(const echo_plan *p) {
+    if (!p) return 0;
+    return (p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_SIDE) ? 4 : 3;
+}
+
+echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out, void *stream,
+                           void *side_stream) {
+    if (!p || !in || !out) return ECHO_ERR_INVALID_ARG;
+    const int P = p->cfg.P;
+    const size_t bytes = (size_t)p->cfg.N * 2;
+    InPtrs xi{};
+    OutPtrs yo{};
+    for (int r = 0; r < P; ++r) {
+        if (!in[r] || !out[r]) return ECHO_ERR_INVALID_ARG;
+        if (!aligned16(in[r]) || !aligned16(out[r])) return ECHO_ERR_ALIGNMENT;
+        xi.p[r] = (const uint4 *)in[r];
+        yo.p[r] = (uint4 *)out[r];
+    }
+    // outputs receive the same values at the same offsets: they must not
+    // overlap one another (inputs are only read, before any output write)
+    for (int r = 0; r < P; ++r)
+        for (int s = r + 1; s < P; ++s) {
+            const char *a = (const char *)out[r], *b = (const char *)out[s];
+            if (a < b + bytes && b < a + bytes) return ECHO_ERR_INVALID_ARG;
+        }
+
+    DeviceGuard guard(p->cfg.device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaStream_t side = (cudaStream_t)side_stream;
+    const bool comp = p->cfg.compensate != 0;
+    const int mode = p->cfg.fixup;
+
+    ProfRecord rec{};
+    if (p->profiling) {
+        for (int i = 0; i < 6; ++i) rec.ev[i] = nullptr;
+        for (int i = 0; i < 4; ++i) {
+            rec.ev[i] = take_event(p);
+            if (!rec.ev[i]) return ECHO_ERR_CUDA;
+        }
+    }
+
+    ECHO_TRY(order_after_side(p, st));
+    const bool defer = comp && mode == ECHO_FIXUP_DEFERRED && p->pending;
+
+    if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[0], st));
+    launch_entry(p, xi, st, defer);
+    ECHO_TRY(cudaGetLastError());
+    if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[1], st));
+    launch_reduce(p, st);
+    ECHO_TRY(cudaGetLastError());
+    if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[2], st));
+
+    const bool fix_in_exit = comp && mode == ECHO_FIXUP_EXIT;
+    const bool fix_on_side = comp && mode == ECHO_FIXUP_SIDE;
+    if (fix_on_side && side) ECHO_TRY(cudaEventRecord(p->ev_reduced, st));
+    launch_exit(p, yo, st, fix_in_exit);
+    ECHO_TRY(cudaGetLastError());
+    if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[3], st));
+
+    if (fix_on_side) {
+        cudaStream_t fs = side ? side : st;
+        if (side) ECHO_TRY(cudaStreamWaitEvent(side, p->ev_reduced, 0));
+        if (p->profiling) {
+            rec.ev[4] = take_event(p);
+            rec.ev[5] = take_event(p);
+            if (!rec.ev[4] || !rec.ev[5]) return ECHO_ERR_CUDA;
+            rec.side = true;
+            ECHO_TRY(cudaEventRecord(rec.ev[4], fs));
+        }
+        launch_fixup(p, p->m_fast, p->m_slow, p->m_fast, p->m_slow, true, true, fs);
+        ECHO_TRY(cudaGetLastError());
+        if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[5], fs));
+        if (side) {
+            ECHO_TRY(cudaEventRecord(p->ev_side_done, side));
+            p->side_inflight = true;
+        } else {
+            p->side_inflight = false;
+        }
+    }
+    if (comp && mode == ECHO_FIXUP_DEFERRED) p->pending = true;
+    if (p->profiling) p->records.push_back(rec);
+    return ECHO_OK;
+}
+
+echo_status echo_allreduce_host(echo_plan *p, const void *const *in_host, void *const *out_host,
+                                void *stream) {
+    if (!p || !in_host || !out_host) return ECHO_ERR_INVALID_ARG;
+    const int P = p->cfg.P;
+    for (int r = 0; r < P; ++r)
+        if (!in_host[r] || !out_host[r]) return ECHO_ERR_INVALID_ARG;
+    DeviceGuard guard(p->cfg.device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    const size_t bytes = (size_t)p->cfg.N * 2;
+    if (!p->stage) {
+        cudaError_t e = cudaMalloc(&p->stage, 2 * (size_t)P * bytes);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            p->stage = nullptr;
+            return from_cuda(e);
+        }
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    const void *din[ECHO_MAX_RANKS];
+    void *dout[ECHO_MAX_RANKS];
+    for (int r = 0; r < P; ++r) {
+        din[r] = (char *)p->stage + (size_t)r * bytes;
+        dout[r] = (char *)p->stage + (size_t)(P + r) * bytes;
+        ECHO_TRY(cudaMemcpyAsync((void *)din[r], in_host[r], bytes, cudaMemcpyHostToDevice, st));
+    }
+    echo_status s = echo_allreduce(p, din, dout, stream, nullptr);
+    if (s != ECHO_OK) return s;
+    for (int r = 0; r < P; ++r)
+        ECHO_TRY(cudaMemcpyAsync(out_host[r], dout[r], bytes, cudaMemcpyDeviceToHost, st));
+    return ECHO_OK;
+}
+
+echo_status echo_reset_state(echo_plan *p, void *stream) {
+    if (!p) return ECHO_ERR_INVALID_ARG;
+    if (!p->cfg.compensate) return ECHO_OK;
+    DeviceGuard guard(p->cfg.device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    ECHO_TRY(order_after_side(p, st));
+    const size_t bytes = (size_t)p->cfg.P * p->cfg.N * 4;
+    ECHO_TRY(cudaMemsetAsync(p->m_fast, 0, bytes, st));
+    ECHO_TRY(cudaMemsetAsync(p->m_slow, 0, bytes, st));
+    p->pending = false;
+    return ECHO_OK;
+}
+
+echo_status echo_get_state(echo_plan *p, float *m_fast, float *m_slow, void *stream) {
+    if (!p || !m_fast || !m_slow || !p->cfg.compensate) return ECHO_ERR_INVALID_ARG;
+    if (!aligned16(m_fast) || !aligned16(m_slow)) return ECHO_ERR_ALIGNMENT;
+    DeviceGuard guard(p->cfg.device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    ECHO_TRY(order_after_side(p, st));
+    launch_fixup(p, p->m_fast, p->m_slow, m_fast, m_slow, p->pending, false, st);
+    ECHO_TRY(cudaGetLastError());
+    return ECHO_OK;
+}
+
+echo_status echo_set_state(echo_plan *p, const float *m_fast, const float *m_slow, void *stream) {
+    if (!p || !m_fast || !m_slow || !p->cfg.compensate) return ECHO_ERR_INVALID_ARG;
+    DeviceGuard guard(p->cfg.device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    ECHO_TRY(order_after_side(p, st));
+    const size_t bytes = (size_t)p->cfg.P * p->cfg.N * 4;
+    ECHO_TRY(cudaMemcpyAsync(p->m_fast, m_fast, bytes, cudaMemcpyDeviceToDevice, st));
+    ECHO_TRY(cudaMemcpyAsync(p->m_slow, m_slow, bytes, cudaMemcpyDeviceToDevice, st));
+    p->pending = false;
+    return ECHO_OK;
+}
+
+echo_status echo_debug_view_get(echo_plan *p, echo_debug_view *v) {
+    if (!p || !v) return ECHO_ERR_INVALID_ARG;
+    v->m_fast = p->m_fast;
+    v->m_slow = p->m_slow;
+    v->codes = (uint8_t *)p->codes;
+    v->scales = p->scales;
+    v->rcodes = (uint8_t *)p->rcodes;
+    v->rscales = p->rscales;
+    v->e_req = p->e_req;
+    v->fixup_pending = p->pending ? 1 : 0;
+    return ECHO_OK;
+}
+
+echo_status echo_profile_enable(echo_plan *p, int32_t on) {
+    if (!p) return ECHO_ERR_INVALID_ARG;
+    p->profiling = on != 0;
+    return ECHO_OK;
+}
+
+echo_status echo_profile_read(echo_plan *p, echo_profile *out, int32_t reset) {
+    if (!p) return ECHO_ERR_INVALID_ARG;
+    DeviceGuard guard(p->cfg.device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    for (auto &r : p->records) {
+        float ms = 0.0f;
+        ECHO_TRY(cudaEventSynchronize(r.ev[3]));
+        ECHO_TRY(cudaEventElapsedTime(&ms, r.ev[0], r.ev[1]));
+        p->totals.entry_ms += ms;
+        ECHO_TRY(cudaEventElapsedTime(&ms, r.ev[1], r.ev[2]));
+        p->totals.reduce_ms += ms;
+        ECHO_TRY(cudaEventElapsedTime(&ms, r.ev[2], r.ev[3]));
+        p->totals.exit_ms += ms;
+        p->totals.launches += 3;
+        if (r.side) {
+            ECHO_TRY(cudaEventSynchronize(r.ev[5]));
+            ECHO_TRY(cudaEventElapsedTime(&ms, r.ev[4], r.ev[5]));
+            p->totals.fixup_ms += ms;
+            p->totals.launches += 1;
+        }
+        p->totals.calls += 1;
+        for (auto ev : r.ev)
+            if (ev) p->pool.push_back(ev);
+    }
+    p->records.clear();
+    if (out) *out = p->totals;
+    if (reset) p->totals = echo_profile{};
+    return ECHO_OK;
+}
+
+const char *echo_status_string(echo_status s) {
+    switch (s) {
+        case ECHO_OK: return "ECHO_OK";
+        case ECHO_ERR_INVALID_ARG: return "ECHO_ERR_INVALID_ARG";
+        case ECHO_ERR_SHAPE: return "ECHO_ERR_SHAPE";
+        case ECHO_ERR_ALIGNMENT: return "ECHO_ERR_ALIGNMENT";
+        case ECHO_ERR_UNSUPPORTED: return "ECHO_ERR_UNSUPPORTED";
+        case ECHO_ERR_OOM: return "ECHO_ERR_OOM";
+        case ECHO_ERR_CUDA: return "ECHO_ERR_CUDA";
+        case ECHO_ERR_TIMEOUT: return "ECHO_ERR_TIMEOUT";
+    }
+    return "ECHO_ERR_UNKNOWN";
+}
+
+int32_t echo_abi_version(void) { return ECHO_ABI_VERSION; }
+
+}  // extern "C"

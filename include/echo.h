@@ -1,0 +1,213 @@
+/*
+ * echo.h -- C ABI of the B200 implementation of Echo, the error-compensated
+ * 4-bit tensor-parallel all-reduce ("Echo: Error-Compensated 4-Bit
+ * Tensor-Parallel Communication for LLM Training and Inference",
+ * arXiv 2610.14277).
+ *
+ * What one call computes (sources, by page and section):
+ *  - ai4snews news summary, "Interpretation", paragraph 1: the all-reduce
+ *    moves 4-bit integer values and sums them in high precision.
+ *  - arXiv abstract (fugumt mirror), "Abstract": each value is quantized at
+ *    most twice per call for any number of ranks; the sum reveals the error
+ *    it injects and the error is fed back into later calls.
+ *  - ai4snews news summary, "Interpretation", paragraph 2: the compensator
+ *    is two moving averages with different decay rates; a correction is
+ *    added to the input before each all-reduce and the averages are
+ *    refreshed from the output residual.
+ *
+ * Per call, for P ranks of N elements each, group size G:
+ *   1. c_r  = alpha*m_fast_r + (1-alpha)*m_slow_r;  xt_r = float(x_r) + c_r
+ *   2. per group of G: a = max|xt|, scale = a/7,
+ *      k = clamp(rint_half_even(xt/scale), -7, 7); codes packed two per
+ *      byte (element 2j in the low nibble), scales fp32
+ *   3. e_in_r = xt_r - k*scale;  m <- beta*m + (1-beta)*e_in_r (both EMAs)
+ *   4. reduce-scatter: the owner o of chunk [o*N/P, (o+1)*N/P) sums
+ *      s = sum over r = 0..P-1 (ascending) of k_r*scale_r in fp32
+ *   5. requantize s with step 2 -> (k2, scale2); y = bf16_rne(k2*scale2);
+ *      e_req = s - float(y)
+ *   6. all-gather: every rank receives y
+ *   7. the owner's states only: m <- m + (1-beta)*e_req (both EMAs)
+ * With the compensator off, c = 0 and no state is read or written.
+ * The constants alpha, beta_fast, beta_slow are parameters: the pages do not
+ * fix them (defaults 0.5, 0.5, 0.95).
+ *
+ * All P ranks live on one GPU; the 4-bit "wire" between the stages is the
+ * packed codes and scales in HBM.  Every quantity at element i depends only
+ * on the G-element group column of i across the P ranks.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *device* are CUDA device pointers on the plan's device;
+ *    pointers named *host* are host pointers (pinned for asynchronous
+ *    copies).  Streams are cudaStream_t handles passed as void*; NULL is the
+ *    legacy default stream.
+ *  - Calls are stream-ordered and asynchronous: nothing synchronizes the
+ *    host except echo_plan_create, echo_plan_destroy and echo_profile_read.
+ *  - All argument checks happen on the host before any launch and return a
+ *    status; a CUDA error returns ECHO_ERR_CUDA.  Nothing aborts.
+ *  - A plan is not thread-safe; calls on one plan must not overlap.
+ */
+#ifndef ECHO_H
+#define ECHO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ECHO_ABI_VERSION 1
+#define ECHO_MAX_RANKS 8
+
+typedef enum echo_status {
+    ECHO_OK = 0,
+    ECHO_ERR_INVALID_ARG = 1, /* null pointer, value out of range */
+    ECHO_ERR_SHAPE = 2,       /* N <= 0 or N % (P*G) != 0 */
+    ECHO_ERR_ALIGNMENT = 3,   /* a buffer not 16-byte aligned */
+    ECHO_ERR_UNSUPPORTED = 4, /* P or G outside the supported set */
+    ECHO_ERR_OOM = 5,         /* device allocation failed */
+    ECHO_ERR_CUDA = 6,        /* a CUDA runtime call failed */
+    ECHO_ERR_TIMEOUT = 7      /* reserved: no kernel here waits on a flag */
+} echo_status;
+
+/* Where the owner's requantization error enters its EMA states (step 7).
+ * All three give bit-identical states, outputs and codes. */
+typedef enum echo_fixup_mode {
+    /* inside the exit kernel that writes the outputs */
+    ECHO_FIXUP_EXIT = 0,
+    /* in its own kernel on the side stream given to echo_allreduce, so it
+     * can run beside the caller's next matrix multiplication (the pages'
+     * "update running beside the next matmul"); the next call on the plan
+     * waits for it */
+    ECHO_FIXUP_SIDE = 1,
+    /* kept pending in the plan and folded into the next call's entry pass,
+     * which reads the state anyway (fewest HBM bytes) */
+    ECHO_FIXUP_DEFERRED = 2
+} echo_fixup_mode;
+
+typedef struct echo_config {
+    int32_t P;          /* ranks, 1..ECHO_MAX_RANKS */
+    int32_t G;          /* group size: 32, 64 or 128 */
+    int64_t N;          /* elements per rank, N > 0, N % (P*G) == 0 */
+    int32_t compensate; /* 1: dual-EMA compensator on, 0: off */
+    float alpha;        /* weight of the fast EMA in the correction, [0,1] */
+    float beta_fast;    /* decay of the fast EMA, [0,1] */
+    float beta_slow;    /* decay of the slow EMA, [0,1] */
+    int32_t device;     /* CUDA device ordinal the plan lives on */
+    int32_t fixup;      /* echo_fixup_mode */
+} echo_config;
+
+typedef struct echo_plan echo_plan;
+
+/* Fill *cfg with the defaults: compensate = 1, alpha = 0.5,
+ * beta_fast = 0.5, beta_slow = 0.95, device = 0, fixup = ECHO_FIXUP_EXIT;
+ * P, G, N are set to 0 and must be filled in. */
+void echo_config_default(echo_config *cfg);
+
+/* Bytes of device memory a plan for *cfg allocates: the EMA states
+ * (2*P*N fp32 when compensating), the entry transport (P*N/2 code bytes +
+ * P*N/G fp32 scales), the reduced transport (N/2 + 4*N/G bytes) and e_req
+ * (N fp32 when compensating), each sub-buffer 256-byte aligned.
+ * Returns 0 for an invalid config. */
+size_t echo_workspace_bytes(const echo_config *cfg);
+
+/* Validate *cfg, allocate the plan's device workspace on cfg->device and
+ * zero the compensator state (m_0 = 0).  Synchronizes the device.
+ * The plan owns its workspace; release it with echo_plan_destroy.
+ * Errors: INVALID_ARG (null, constants outside [0,1], bad fixup mode),
+ * UNSUPPORTED (P, G), SHAPE (N), OOM, CUDA.  *out is NULL on error. */
+echo_status echo_plan_create(echo_plan **out, const echo_config *cfg);
+
+/* Free everything the plan allocated (after synchronizing its device).
+ * NULL is accepted and ignored. */
+echo_status echo_plan_destroy(echo_plan *plan);
+
+/* One compensated 4-bit all-reduce over the P ranks (steps 1-7 above).
+ *   in_device[r]  : bf16, N contiguous elements of rank r (read)
+ *   out_device[r] : bf16, N contiguous elements (written with y); may equal
+ *                   in_device[r] (in-place)
+ *   stream        : stream the entry, reduce and exit kernels run on
+ *   side_stream   : used with ECHO_FIXUP_SIDE only (the owner fix-up runs
+ *                   there after an event on stream); NULL runs the fix-up
+ *                   on stream.  Ignored by the other modes.
+ * Both pointer arrays are host arrays of P device pointers, each 16-byte
+ * aligned.  Buffers are owned by the caller and must stay valid until the
+ * call completes on the stream.  Output buffers must not overlap each other
+ * or another rank's input.
+ * Errors: INVALID_ARG (null plan/arrays/pointers), ALIGNMENT, CUDA. */
+echo_status echo_allreduce(echo_plan *plan, const void *const *in_device,
+                           void *const *out_device, void *stream,
+                           void *side_stream);
+
+/* The same call on host buffers: copies the P inputs host -> device into a
+ * staging area the plan allocates on first use (2*P*N*2 bytes, kept until
+ * echo_plan_destroy), runs echo_allreduce on stream, and copies the P
+ * outputs device -> host.  in_host[r], out_host[r]: N bf16 elements each;
+ * pinned host memory makes the copies asynchronous, pageable memory makes
+ * them synchronous.  The caller synchronizes stream before reading out_host.
+ * Errors: INVALID_ARG, OOM (staging), CUDA. */
+echo_status echo_allreduce_host(echo_plan *plan, const void *const *in_host,
+                                void *const *out_host, void *stream);
+
+/* Zero the compensator state (m_fast = m_slow = 0) and drop any pending
+ * deferred fix-up, on stream.  A no-op (ECHO_OK) when compensate == 0. */
+echo_status echo_reset_state(echo_plan *plan, void *stream);
+
+/* Copy the current states, with any pending deferred fix-up applied, into
+ * caller device buffers m_fast_device, m_slow_device ([P][N] fp32, rank
+ * major), on stream.  The plan's state is not changed.
+ * Errors: INVALID_ARG (null, or compensate == 0), CUDA. */
+echo_status echo_get_state(echo_plan *plan, float *m_fast_device,
+                           float *m_slow_device, void *stream);
+
+/* Overwrite the states from caller device buffers ([P][N] fp32) and drop
+ * any pending fix-up, on stream (checkpoint restore, tests).
+ * Errors: INVALID_ARG (null, or compensate == 0), CUDA. */
+echo_status echo_set_state(echo_plan *plan, const float *m_fast_device,
+                           const float *m_slow_device, void *stream);
+
+/* Device pointers into the plan's workspace, for inspection by tests.  The
+ * contents are those left by the last call; with ECHO_FIXUP_DEFERRED the
+ * states lack the pending fix-up (echo_get_state applies it). */
+typedef struct echo_debug_view {
+    float *m_fast;      /* [P][N] fp32, or NULL when not compensating */
+    float *m_slow;      /* [P][N] fp32, or NULL */
+    uint8_t *codes;     /* [P][N/2] entry codes */
+    float *scales;      /* [P][N/G] entry scales */
+    uint8_t *rcodes;    /* [N/2] requantized sum codes */
+    float *rscales;     /* [N/G] requantization scales */
+    float *e_req;       /* [N] requantization error, or NULL */
+    int32_t fixup_pending; /* 1 if a deferred fix-up is pending */
+} echo_debug_view;
+
+echo_status echo_debug_view_get(echo_plan *plan, echo_debug_view *view);
+
+/* Per-kernel timing with CUDA events recorded on the stream each kernel is
+ * launched on.  While enabled, every call records events around its
+ * kernels; echo_profile_read synchronizes on them, adds the elapsed times
+ * to the totals below and returns them; reset clears the totals. */
+typedef struct echo_profile {
+    int64_t calls;          /* calls recorded */
+    double entry_ms;        /* total time of echo_entry launches */
+    double reduce_ms;       /* total time of echo_reduce launches */
+    double exit_ms;         /* total time of echo_exit launches */
+    double fixup_ms;        /* total time of side-stream fix-up launches */
+    int64_t launches;       /* kernels launched by the recorded calls */
+} echo_profile;
+
+echo_status echo_profile_enable(echo_plan *plan, int32_t on);
+echo_status echo_profile_read(echo_plan *plan, echo_profile *out, int32_t reset);
+
+/* Kernels launched by one echo_allreduce call with this plan. */
+int32_t echo_launches_per_call(const echo_plan *plan);
+
+/* Static name of a status code. */
+const char *echo_status_string(echo_status s);
+
+int32_t echo_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ECHO_H */
