@@ -82,6 +82,8 @@ def _load():
         "echo_launches_per_call": (ctypes.c_int32, [vp]),
         "echo_status_string": (ctypes.c_char_p, [st]),
         "echo_abi_version": (ctypes.c_int32, []),
+        "echo_allreduce_noalloc": (st, [ctypes.POINTER(echo_config), ctypes.POINTER(vp),
+                                        ctypes.POINTER(vp), vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -177,3 +179,17 @@ def echo_status_string(status: int) -> str:
 
 def echo_abi_version() -> int:
     return int(lib.echo_abi_version())
+
+
+ECHO_NOALLOC_MAX_SCRATCH_BYTES = 80 << 20
+
+
+def echo_allreduce_noalloc(cfg: echo_config, in_device: Sequence[int],
+                           out_device: Sequence[int], m_fast_device: int, m_slow_device: int,
+                           stream: int = 0) -> None:
+    """The allocation-free call: no plan, caller-owned state, scratch in the
+    library's fixed device array (see include/echo.h)."""
+    _check(lib.echo_allreduce_noalloc(ctypes.byref(cfg), _ptr_array(in_device),
+                                      _ptr_array(out_device), m_fast_device or None,
+                                      m_slow_device or None, stream or None),
+           "echo_allreduce_noalloc")

@@ -201,6 +201,49 @@ echo_status echo_profile_read(echo_plan *plan, echo_profile *out, int32_t reset)
 /* Kernels launched by one echo_allreduce call with this plan. */
 int32_t echo_launches_per_call(const echo_plan *plan);
 
+/* ------------------------------------------------------------------------
+ * Allocation-free call.  The paper has no counterpart: this entry point
+ * exists for callers that cannot allocate device memory on their call path,
+ * for example a serving process whose memory manager reserves the whole GPU
+ * up front and accounts for every byte (a library cudaMalloc would fail or
+ * break that accounting), code that cannot afford the device-wide
+ * synchronization that cudaMalloc and cudaFree imply, or a plugin host that
+ * hands a library only its buffers and a stream.
+ *
+ * It computes exactly what echo_allreduce computes for a plan made from
+ * *cfg with ECHO_FIXUP_EXIT (cfg->fixup is ignored), but without a plan:
+ *   in_device[r], out_device[r] : as for echo_allreduce (P bf16 buffers of
+ *                                 N elements, 16-byte aligned)
+ *   m_fast_device, m_slow_device: the compensator state, owned by the
+ *                                 caller: [P][N] fp32, rank major, zero
+ *                                 before the first call, updated in place
+ *                                 (ignored, may be NULL, when
+ *                                 cfg->compensate == 0)
+ *   stream                      : where the three kernels run
+ * The scratch the kernels hand each other (entry codes and scales, the
+ * requantized codes and scales and, compensating, e_req) lives in one
+ * file-scope device array of ECHO_NOALLOC_MAX_SCRATCH_BYTES, which every
+ * GPU that loads this code holds until the process exits.  A call needs
+ *   P*N/2 + 4*P*N/G + N/2 + 4*N/G (+ 4*N when compensating)
+ * bytes, each part rounded up to 256; a call that needs more returns
+ * ECHO_ERR_UNSUPPORTED before launching anything (80 MiB holds, e.g., 8
+ * ranks of 2048 x 4096 bf16 activations with the compensator on).
+ * The first call on a device looks up the array's address with
+ * cudaGetSymbolAddress while that device is current; make that first call
+ * before any stream capture.  All calls on a device share the one array and
+ * it keeps the last call's contents: nothing in it needs to start at zero
+ * (every byte a call reads was written earlier in the same call), but calls
+ * that overlap on the GPU -- on streams not ordered with each other, or
+ * from several host threads at once -- race on it and corrupt each other's
+ * results.  Order them on one stream.
+ * Calls no cudaMalloc, cudaFree or host allocator.  Errors as for
+ * echo_allreduce, plus UNSUPPORTED for the size limit. */
+#define ECHO_NOALLOC_MAX_SCRATCH_BYTES ((size_t)80 << 20)
+
+echo_status echo_allreduce_noalloc(const echo_config *cfg, const void *const *in_device,
+                                   void *const *out_device, float *m_fast_device,
+                                   float *m_slow_device, void *stream);
+
 /* Static name of a status code. */
 const char *echo_status_string(echo_status s);
 
