@@ -49,8 +49,10 @@ UNIT = "GB/s"
 # fix-up placement timed by default (bit-identical to the others; fewest bytes)
 BENCH_FIXUP = "deferred"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_FILES = ("bit_error_compensated_echo_b200/csrc/echo_kernels.cuh",
-                "bit_error_compensated_echo_b200/csrc/echo.cu")
+# sources of the dominant kernel (echo_entry): an ncu traffic figure is
+# reported only if it was captured from exactly these files
+KERNEL_FILES = ("bit_error_compensated_echo_b200/csrc/echo_common.cuh",
+                "bit_error_compensated_echo_b200/csrc/echo_entry.cuh")
 
 WORKLOADS = {"large": W.LARGE, "llama": W.LLAMA, "depth": W.DEPTH, "tiny": W.TINY}
 
@@ -421,9 +423,9 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-cols", type=int, default=65536,
+    ap.add_argument("--cpu-cols", type=int, default=655360,
                     help="group columns of the CPU-baseline sample")
-    ap.add_argument("--ref-cols", type=int, default=16384,
+    ap.add_argument("--ref-cols", type=int, default=131072,
                     help="group columns per step of the reference arm")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":

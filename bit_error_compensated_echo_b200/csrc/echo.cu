@@ -6,7 +6,7 @@
 // e_req.  A call launches three kernels on the caller's stream -- entry,
 // reduce, exit -- plus, in side-stream mode, the owner fix-up on the side
 // stream.  Host code here only validates, carves memory, orders streams and
-// launches: every step of the arithmetic runs in echo_kernels.cuh.
+// launches: every step of the arithmetic runs in the kernels of echo_*.cuh.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -16,7 +16,10 @@
 #include <vector>
 
 #include "echo.h"
-#include "echo_kernels.cuh"
+#include "echo_entry.cuh"
+#include "echo_exit.cuh"
+#include "echo_fixup.cuh"
+#include "echo_reduce.cuh"
 
 using namespace echo;
 
@@ -155,7 +158,7 @@ void launch_entry(echo_plan *p, const InPtrs &x, cudaStream_t st, bool defer) {
 
 template <int G, int P>
 void launch_reduce_t(echo_plan *p, cudaStream_t st) {
-    dim3 grid((unsigned)((p->chunk_vec + kThreads - 1) / kThreads), (unsigned)P);
+    dim3 grid(reduce_blocks(p->chunk_vec), (unsigned)P);
     if (p->cfg.compensate)
         echo_reduce_kernel<G, P, true><<<grid, kThreads, 0, st>>>(
             p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec);

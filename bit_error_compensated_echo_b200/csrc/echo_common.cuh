@@ -1,0 +1,239 @@
+// echo_common.cuh -- shared definitions of the sm_100a kernels of Echo's error-compensated 4-bit
+// all-reduce ("Echo: Error-Compensated 4-Bit Tensor-Parallel Communication",
+// ai4snews news summary "Interpretation" and the arXiv abstract on the
+// fugumt mirror).  The operation each kernel computes is written out in
+// include/echo.h; here is how it maps onto the B200.
+//
+// The path is elementwise codec work bound by HBM bandwidth, not a
+// contraction, so there are no tensor cores.  A thread owns a run of
+// consecutive elements of one rank (8 in the entry and exit passes: one
+// 16-byte bf16 vector, two float4 of each EMA state, one 32-bit word of
+// packed codes; 16 in the reduce pass).  A group of G elements is G/8 (or
+// G/16) adjacent lanes of one warp; its absmax is a butterfly of
+// __shfl_xor_sync (max is order-free, so it is exact).  All fp32 arithmetic
+// uses the explicitly rounded intrinsics (__fadd_rn, __fmul_rn, __fdiv_rn),
+// which the compiler never contracts into FMA, so every value is the same
+// IEEE-754 single-precision result as a plain scalar evaluation of the
+// definition.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace echo {
+
+constexpr int kVec = 8;          // elements per thread (entry, exit)
+constexpr int kThreads = 256;    // threads per block of every kernel
+constexpr int kMaxRanks = 8;
+
+struct InPtrs {
+    const uint4 *p[kMaxRanks];   // rank r's bf16 input, 8 elements per uint4
+};
+struct OutPtrs {
+    uint4 *p[kMaxRanks];
+};
+
+struct Consts {
+    float alpha, one_m_alpha;
+    float beta_fast, one_m_beta_fast;
+    float beta_slow, one_m_beta_slow;
+};
+
+// ------------------------------------------------------------ helpers
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float f[8]) {
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xffff0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xffff0000u);
+    f[4] = __uint_as_float(v.z << 16);
+    f[5] = __uint_as_float(v.z & 0xffff0000u);
+    f[6] = __uint_as_float(v.w << 16);
+    f[7] = __uint_as_float(v.w & 0xffff0000u);
+}
+
+// max over the LANES adjacent lanes that hold one group
+template <int LANES>
+__device__ __forceinline__ float group_absmax(float a) {
+#pragma unroll
+    for (int off = 1; off < LANES; off <<= 1)
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+    return a;
+}
+
+// ---- packed fp32 pairs (sm_100 add/sub/mul .rn.f32x2)
+//
+// Each lane of a pair is an ordinary IEEE-754 fp32 operation rounded to
+// nearest even (subnormals kept), so a pair op gives exactly the two scalar
+// results; it issues once for both.  ptxas contracts a packed multiply whose
+// result feeds a packed add or subtract into one fused multiply-add (single
+// rounding) even with explicit .rn, so a pair multiply is only ever used
+// where its result goes through a min/max or a conversion first; every
+// multiply-then-add of the definition uses the scalar __fmul_rn/__fadd_rn,
+// which are never contracted.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+// ---- exact integer <-> float steps without conversion instructions
+//
+// In [2^23, 2^24) consecutive floats are consecutive integers, so adding
+// 1.5*2^23 to a float q with |q| <= 7 rounds q to an integer under the
+// current rounding (nearest, ties to even -- the same result as rint(q)),
+// and the low nibble of the sum's bit pattern is that integer in 4-bit two's
+// complement (the bits of 1.5*2^23 end in 0x0).  Going back, 2^23 + u with
+// u = (k + 8) in 0..15 has bit pattern 0x4B000000 | u, and subtracting
+// 2^23 + 8 gives k exactly.  Both replace the int<->float conversion
+// instructions, which issue at a fraction of the fp32 add rate.
+constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
+constexpr float kCodeMagic = 8388616.0f;     // 2^23 + 8
+
+// Codes 2j and 2j+1 of a packed word, as a float pair.  lo_nibs/hi_nibs
+// are (w ^ 0x88888888) & 0x0F0F0F0F and ((w ^ 0x88888888) >> 4) & 0x0F0F0F0F:
+// byte j of each holds k + 8 of element 2j / 2j+1.  One byte permute per
+// element builds the bit pattern 0x4B0000uu = 2^23 + u, and one packed
+// subtract of 2^23 + 8 leaves k exactly.
+__device__ __forceinline__ float2 code_pair(uint32_t lo_nibs, uint32_t hi_nibs, int j) {
+    const float2 m = make_float2(__uint_as_float(__byte_perm(lo_nibs, 0x4B000000u, 0x7540 + j)),
+                                 __uint_as_float(__byte_perm(hi_nibs, 0x4B000000u, 0x7540 + j)));
+    return sub2(m, splat2(kCodeMagic));
+}
+__device__ __forceinline__ uint32_t low_nibbles(uint32_t w) {
+    return (w ^ 0x88888888u) & 0x0F0F0F0Fu;
+}
+__device__ __forceinline__ uint32_t high_nibbles(uint32_t w) {
+    return ((w ^ 0x88888888u) >> 4) & 0x0F0F0F0Fu;
+}
+
+// bf16 round-to-nearest-even of a pair, returned as one word (first value in
+// the low half), and the pair's exact fp32 values
+__device__ __forceinline__ uint32_t bf16x2_bits_rn(float2 v) {
+    const __nv_bfloat162 b = __float22bfloat162_rn(v);
+    return *reinterpret_cast<const uint32_t *>(&b);
+}
+__device__ __forceinline__ float2 bf16x2_to_f32(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// scale = a / 7, or 0 for an all-zero group
+__device__ __forceinline__ float group_scale(float a) {
+    return a != 0.0f ? __fdiv_rn(a, 7.0f) : 0.0f;
+}
+
+// Quantize 8 values of a group with one IEEE division per element:
+// k = clamp(rint(v / scale), -7, 7), ties to even, all 0 when scale == 0;
+// packed as quantize8 below, k as floats in kf.  Preferred where the values
+// are short bf16 numbers: their quotients land on or near half-integers
+// often, which would send quantize8 to its exact path most of the time.
+__device__ __forceinline__ uint32_t quantize8_div(const float v[8], float scale, float kf[8]) {
+    if (scale == 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) kf[i] = 0.0f;
+        return 0u;
+    }
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float q = fminf(fmaxf(__fdiv_rn(v[i], scale), -7.0f), 7.0f);
+        const float t = __fadd_rn(q, kRoundMagic);
+        kf[i] = __fsub_rn(t, kRoundMagic);
+        w |= (__float_as_uint(t) & 0xfu) << (4 * i);
+    }
+    return w;
+}
+
+// Quantize 8 values of a group: k = clamp(rint(v / scale), -7, 7), ties to
+// even, all 0 when scale == 0.  Returns the packed word (element i in bits
+// 4i..4i+3, so byte j holds element 2j in its low nibble and 2j+1 in its
+// high nibble) and k as floats in kf.
+//
+// inv is 1/scale rounded (0 when scale == 0, which makes every code 0).
+// For a normal scale, q~ = v*inv differs from the rounded quotient
+// fl(v/scale) by less than 2^-20 (both lie within a few units in the last
+// place of |v/scale| <= 7), so the two round to the same integer unless the
+// exact quotient lies within 2^-19 of a half-integer.  The fast path rounds
+// q~ and flags any element whose q~ lies within 2^-18 of a half-integer;
+// then (rarely), and for every group whose scale is subnormal, all 8 codes
+// are taken from the IEEE division itself.  Either way the codes are
+// exactly those of rint(v/scale).
+struct GroupScale {
+    float scale;  // a / 7 (0 for an all-zero group)
+    float inv;    // 1 / scale rounded, 0 when scale == 0
+    bool exact;   // subnormal scale: always use the division
+};
+
+__device__ __forceinline__ GroupScale make_group_scale(float a) {
+    GroupScale g;
+    g.scale = a != 0.0f ? __fdiv_rn(a, 7.0f) : 0.0f;
+    g.exact = g.scale != 0.0f && g.scale < 1.17549435e-38f;  // below FLT_MIN
+    g.inv = (g.scale != 0.0f && !g.exact) ? __frcp_rn(g.scale) : 0.0f;
+    return g;
+}
+
+__device__ __forceinline__ uint32_t quantize8_exact(const float v[8], float scale, float kf[8]) {
+    uint32_t w = 0;
+    for (int i = 0; i < 8; ++i) {
+        float t = kRoundMagic;
+        if (scale != 0.0f)
+            t = __fadd_rn(fminf(fmaxf(__fdiv_rn(v[i], scale), -7.0f), 7.0f), kRoundMagic);
+        kf[i] = __fsub_rn(t, kRoundMagic);
+        w |= (__float_as_uint(t) & 0xfu) << (4 * i);
+    }
+    return w;
+}
+
+__device__ __forceinline__ uint32_t quantize8(const float v[8], const GroupScale &g, float kf[8]) {
+    uint32_t w = 0;
+    bool near_tie = g.exact;
+    const float2 inv2 = splat2(g.inv), magic2 = splat2(kRoundMagic);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        float2 q = mul2(make_float2(v[i], v[i + 1]), inv2);
+        q.x = fminf(fmaxf(q.x, -7.0f), 7.0f);
+        q.y = fminf(fmaxf(q.y, -7.0f), 7.0f);
+        const float2 t = add2(q, magic2);
+        const float2 k = sub2(t, magic2);
+        const float2 d = sub2(q, k);
+        kf[i] = k.x;
+        kf[i + 1] = k.y;
+        near_tie |= fmaxf(fabsf(d.x), fabsf(d.y)) > 0.5f - 0x1p-18f;
+        w |= (__float_as_uint(t.x) & 0xfu) << (4 * i);
+        w |= (__float_as_uint(t.y) & 0xfu) << (4 * i + 4);
+    }
+    if (near_tie) w = quantize8_exact(v, g.scale, kf);
+    return w;
+}
+
+__device__ __forceinline__ void ld8(const float *p, float v[8]) {
+    const float4 a = reinterpret_cast<const float4 *>(p)[0];
+    const float4 b = reinterpret_cast<const float4 *>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void st8(float *p, const float v[8]) {
+    reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+}  // namespace echo

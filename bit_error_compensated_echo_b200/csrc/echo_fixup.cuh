@@ -1,0 +1,45 @@
+// echo_fixup.cuh -- the owner fix-up as its own launch, and state reads
+// (operation: include/echo.h; conventions: echo_common.cuh)
+#pragma once
+
+#include "echo_common.cuh"
+
+namespace echo {
+
+// ------------------------------------------------------------ owner fix-up
+//
+// The owner fix-up alone, as its own launch (side-stream mode), or, with
+// dst != src, a copy of the states that applies a pending fix-up on the way
+// (reading the state of a plan in deferred mode).  Grid: x over the vectors
+// of one owner chunk, y = rank; only rank == owner adds the fix-up.
+__global__ void __launch_bounds__(kThreads)
+echo_fixup_kernel(const float *__restrict__ src_fast, const float *__restrict__ src_slow,
+                  float *__restrict__ dst_fast, float *__restrict__ dst_slow,
+                  const float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec,
+                  int P, int apply, int only_owner, Consts k) {
+    const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (local >= chunk_vec) return;
+    const int o = blockIdx.y;
+    for (int r = 0; r < P; ++r) {
+        const bool own = (r == o);
+        if (only_owner && !own) continue;
+        const int64_t j = (int64_t)o * chunk_vec + local;
+        const int64_t e0 = ((int64_t)r * n_vec + j) * kVec;
+        float mf[8], ms[8];
+        ld8(src_fast + e0, mf);
+        ld8(src_slow + e0, ms);
+        if (own && apply) {
+            float er[8];
+            ld8(e_req + j * kVec, er);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                mf[i] = __fadd_rn(mf[i], __fmul_rn(k.one_m_beta_fast, er[i]));
+                ms[i] = __fadd_rn(ms[i], __fmul_rn(k.one_m_beta_slow, er[i]));
+            }
+        }
+        st8(dst_fast + e0, mf);
+        st8(dst_slow + e0, ms);
+    }
+}
+
+}  // namespace echo

@@ -12,12 +12,9 @@
 #include <mutex>
 
 #include "echo.h"
-// This file launches only the entry, reduce and exit kernel templates.  The
-// header also defines the (non-template) fix-up kernel, whose one external
-// definition belongs to echo.cu; it gets a file-local name here.
-#define echo_fixup_kernel echo_fixup_kernel_unused_in_noalloc
-#include "echo_kernels.cuh"
-#undef echo_fixup_kernel
+#include "echo_entry.cuh"
+#include "echo_exit.cuh"
+#include "echo_reduce.cuh"
 
 using namespace echo;
 
@@ -80,17 +77,18 @@ void launch_all(const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigne
     float *e_req = comp ? (float *)(s + L.e_req) : nullptr;
     dim3 g_entry((unsigned)((n_vec + kThreads - 1) / kThreads), (unsigned)P);
     dim3 g_chunk((unsigned)((chunk_vec + kThreads - 1) / kThreads), (unsigned)P);
+    dim3 g_red(reduce_blocks(chunk_vec), (unsigned)P);
     if (comp) {
         echo_entry_kernel<G, true, false><<<g_entry, kThreads, 0, st>>>(
             x, mf, ms, codes, scales, e_req, n_vec, chunk_vec, k);
-        echo_reduce_kernel<G, P, true><<<g_chunk, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, true><<<g_red, kThreads, 0, st>>>(
             codes, scales, rcodes, rscales, e_req, n_vec, chunk_vec);
         echo_exit_kernel<G, true><<<g_chunk, kThreads, 0, st>>>(
             rcodes, rscales, y, P, mf, ms, e_req, n_vec, chunk_vec, k);
     } else {
         echo_entry_kernel<G, false, false><<<g_entry, kThreads, 0, st>>>(
             x, nullptr, nullptr, codes, scales, nullptr, n_vec, chunk_vec, k);
-        echo_reduce_kernel<G, P, false><<<g_chunk, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, false><<<g_red, kThreads, 0, st>>>(
             codes, scales, rcodes, rscales, nullptr, n_vec, chunk_vec);
         echo_exit_kernel<G, false><<<g_chunk, kThreads, 0, st>>>(
             rcodes, rscales, y, P, nullptr, nullptr, nullptr, n_vec, chunk_vec, k);

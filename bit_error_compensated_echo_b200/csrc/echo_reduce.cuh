@@ -1,0 +1,92 @@
+// echo_reduce.cuh -- the reduce-scatter half: dequantize, fp32 sum, requantize
+// (operation: include/echo.h; conventions: echo_common.cuh)
+#pragma once
+
+#include "echo_common.cuh"
+
+namespace echo {
+
+// ------------------------------------------------------------ echo_reduce
+//
+// Reduce-scatter half: for every element, dequantize the P ranks' codes,
+// sum them in fp32 in ascending rank order from +0, requantize the sum,
+// pack it, and (compensating) write e_req = s - float(bf16(k2*scale2)).
+// Each thread owns 16 consecutive elements: one 8-byte word pair of codes
+// per rank, all P loads issued before any arithmetic so that every thread
+// keeps P*8 bytes of the transport in flight.
+// Grid: x over the N/(16P) runs of one owner chunk, y = owner.
+constexpr int kRedVec = 16;
+
+// blocks along x for an owner chunk of chunk_vec 8-element vectors
+inline unsigned reduce_blocks(int64_t chunk_vec) {
+    return (unsigned)((chunk_vec / 2 + kThreads - 1) / kThreads);
+}
+
+template <int G, int P, bool COMP>
+__global__ void __launch_bounds__(kThreads)
+echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
+                   uint32_t *__restrict__ rcodes, float *__restrict__ rscales,
+                   float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec) {
+    constexpr int LANES = G / kRedVec;              // lanes per group
+    const int o = blockIdx.y;
+    const int64_t n_run = n_vec / 2;                // 16-element runs per rank
+    const int64_t chunk_run = chunk_vec / 2;        // runs per owner chunk
+    const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    const bool valid = local < chunk_run;
+    const int64_t j = (int64_t)o * chunk_run + local;  // run index in a rank
+    const int64_t n_groups = n_run / LANES;
+    const uint2 *codes2 = reinterpret_cast<const uint2 *>(codes);
+
+    uint2 w[P];
+    float sc[P];
+#pragma unroll
+    for (int r = 0; r < P; ++r) {
+        w[r] = valid ? __ldcs(codes2 + (int64_t)r * n_run + j) : make_uint2(0u, 0u);
+        sc[r] = valid ? __ldg(scales + (int64_t)r * n_groups + j / LANES) : 0.0f;
+    }
+    float s[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s[i] = 0.0f;
+#pragma unroll
+    for (int r = 0; r < P; ++r) {
+        const uint32_t lx = low_nibbles(w[r].x), hx = high_nibbles(w[r].x);
+        const uint32_t ly = low_nibbles(w[r].y), hy = high_nibbles(w[r].y);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 kx = code_pair(lx, hx, p), ky = code_pair(ly, hy, p);
+            s[2 * p] = __fadd_rn(s[2 * p], __fmul_rn(kx.x, sc[r]));
+            s[2 * p + 1] = __fadd_rn(s[2 * p + 1], __fmul_rn(kx.y, sc[r]));
+            s[8 + 2 * p] = __fadd_rn(s[8 + 2 * p], __fmul_rn(ky.x, sc[r]));
+            s[9 + 2 * p] = __fadd_rn(s[9 + 2 * p], __fmul_rn(ky.y, sc[r]));
+        }
+    }
+
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(s[i]));
+    a = group_absmax<LANES>(a);
+    const GroupScale gs = make_group_scale(a);
+    const float scale2 = gs.scale;
+    float k2[16];
+    const uint32_t w0 = quantize8(s, gs, k2);
+    const uint32_t w1 = quantize8(s + 8, gs, k2 + 8);
+    if (!valid) return;
+
+    reinterpret_cast<uint2 *>(rcodes)[j] = make_uint2(w0, w1);
+    if ((threadIdx.x & (LANES - 1)) == 0) rscales[j / LANES] = scale2;
+    if (COMP) {
+        float e[16];
+        const float2 sc2 = splat2(scale2);
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            const float2 y = bf16x2_to_f32(bf16x2_bits_rn(mul2(make_float2(k2[i], k2[i + 1]), sc2)));
+            const float2 d = sub2(make_float2(s[i], s[i + 1]), y);
+            e[i] = d.x;
+            e[i + 1] = d.y;
+        }
+        st8(e_req + j * kRedVec, e);
+        st8(e_req + j * kRedVec + 8, e + 8);
+    }
+}
+
+}  // namespace echo

@@ -67,7 +67,7 @@ typedef enum echo_status {
     ECHO_ERR_UNSUPPORTED = 4, /* P or G outside the supported set */
     ECHO_ERR_OOM = 5,         /* device allocation failed */
     ECHO_ERR_CUDA = 6,        /* a CUDA runtime call failed */
-    ECHO_ERR_TIMEOUT = 7      /* reserved: no kernel here waits on a flag */
+    ECHO_ERR_TIMEOUT = 7      /* reserved: no kernel here waits on a flag or barrier */
 } echo_status;
 
 /* Where the owner's requantization error enters its EMA states (step 7).
@@ -106,7 +106,7 @@ void echo_config_default(echo_config *cfg);
 
 /* Bytes of device memory a plan for *cfg allocates: the EMA states
  * (2*P*N fp32 when compensating), the entry transport (P*N/2 code bytes +
- * P*N/G fp32 scales), the reduced transport (N/2 + 4*N/G bytes) and e_req
+ * P*N/G fp32 scales), the reduced transport (N/2 + 4*N/G bytes), e_req
  * (N fp32 when compensating), each sub-buffer 256-byte aligned.
  * Returns 0 for an invalid config. */
 size_t echo_workspace_bytes(const echo_config *cfg);

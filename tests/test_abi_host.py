@@ -88,6 +88,7 @@ def test_workspace_bytes_closed_form(abi):
     for P, G, k, comp in ((8, 128, 64, 1), (2, 32, 3, 0), (5, 64, 7, 1)):
         N = P * G * k
         c = _cfg(abi, P=P, G=G, N=N, compensate=comp)
+        # codes, scales, reduced codes and scales
         want = al(P * N // 2) + al(P * (N // G) * 4) + al(N // 2) + al((N // G) * 4)
         if comp:
             want += 2 * al(P * N * 4) + al(N * 4)
