@@ -410,6 +410,164 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def _time_calls(fn, steps, flush, stream):
+    """Median device time of fn() over steps launches, L2 flushed between."""
+    times = []
+    for k in range(steps):
+        flush.fill_(float(k))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def run_sweep_mode(args, ws, rank, local):
+    """Sizes 1 MiB..1 GiB per rank x P in {2,4,8} x G in {32,64,128} x
+    compensated / off: GB/s, fraction of the call roofline, packed ratio;
+    eager and CUDA-graph-captured times, L2 flushed between timed calls."""
+    from bit_error_compensated_echo_b200.api import EchoPlan
+    if rank != 0:
+        return
+    dev = torch.device("cuda", local)
+    peak, peak_kind = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    points = W.sweep()
+    if args.sweep_max_mib:
+        points = [w for w in points if w.N * 2 <= args.sweep_max_mib << 20]
+    for w in points:
+        x = W.generate(w, 0, dev)
+        out = torch.empty_like(x)
+        plan = EchoPlan(w.P, w.N, w.G, compensate=w.compensate, fixup=BENCH_FIXUP, device=local)
+        for _ in range(max(args.warmup, 3)):
+            plan.allreduce(x, out=out)
+        torch.cuda.synchronize()
+        t_eager = _time_calls(lambda: plan.allreduce(x, out=out), args.steps, flush, stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            plan.allreduce(x, out=out)
+        g.replay()
+        torch.cuda.synchronize()
+        t_graph = _time_calls(g.replay, args.steps, flush, stream)
+        del g
+        bmin = call_min_bytes(w.P, w.N, w.G, w.compensate)
+        q = transport_bytes_per_elem(w.G)
+        row = {"mode": "sweep", "point": w.name, "MiB_per_rank": w.N * 2 // (1 << 20), "P": w.P,
+               "G": w.G, "compensate": w.compensate, "ms_eager": round(t_eager, 4),
+               "ms_graph": round(t_graph, 4),
+               "input_gbs": round(2 * w.P * w.N / (min(t_eager, t_graph) / 1e3) / 1e9, 2),
+               "roofline_frac": round(bmin / peak / (min(t_eager, t_graph) / 1e3) / 1e9, 4),
+               "min_bytes": bmin, "packed_ratio": q / 2}
+        dv = plan.debug_view()
+        row["packed_ratio_allocated"] = (dv["codes"].numel() + 4 * dv["scales"].numel()) / (2.0 * w.P * w.N)
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+        plan.close()
+        del x, out, plan
+        torch.cuda.empty_cache()
+    if args.sweep_table:
+        with open(args.sweep_table, "w") as f:
+            f.write("| MiB/rank | P | G | mode | ms eager | ms graph | input GB/s | % of call roofline | packed/bf16 |\n")
+            f.write("|---|---|---|---|---|---|---|---|---|\n")
+            for r in rows:
+                f.write("| %d | %d | %d | %s | %.4f | %.4f | %.1f | %.1f | %.6f |\n" % (
+                    r["MiB_per_rank"], r["P"], r["G"], "comp" if r["compensate"] else "off",
+                    r["ms_eager"], r["ms_graph"], r["input_gbs"], 100 * r["roofline_frac"],
+                    r["packed_ratio"]))
+
+
+def run_overlap_mode(args, ws, rank, local):
+    """1 GiB per rank, P=8: the stand-in next matmul (bf16 8192^3) after each
+    call, with the owner fix-up in the exit kernel, on a side stream beside
+    the matmul, or deferred; plus the fused compensation cost (compensated
+    minus uncompensated call) and the compensator written as separate torch
+    operations, for context."""
+    from bit_error_compensated_echo_b200.api import EchoPlan
+    if rank != 0:
+        return
+    dev = torch.device("cuda", local)
+    w = W.LARGE
+    x = torch.empty((w.P, w.N), dtype=torch.bfloat16, device=dev)
+    W.generate(w, 0, dev, out=x)
+    out = torch.empty_like(x)
+    ga = torch.randn((8192, 8192), device=dev).to(torch.bfloat16)
+    gb = torch.randn((8192, 8192), device=dev).to(torch.bfloat16)
+    gc = torch.empty((8192, 8192), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(device=dev)
+
+    def timed(fn, steps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    res = {"mode": "overlap", "workload": w.name, "gemm": "bf16 8192x8192x8192 torch.matmul"}
+    res["gemm_ms"] = round(timed(lambda: torch.matmul(ga, gb, out=gc), args.steps), 4)
+    for comp, fixup in ((False, "exit"), (True, "exit"), (True, "side"), (True, "deferred")):
+        plan = EchoPlan(w.P, w.N, w.G, compensate=comp, fixup=fixup, device=local)
+        key = ("comp_" + fixup) if comp else "off"
+        res["call_ms_" + key] = round(timed(lambda: plan.allreduce(x, out=out, side_stream=side),
+                                            args.steps), 4)
+
+        def step():
+            plan.allreduce(x, out=out, side_stream=side)
+            torch.matmul(ga, gb, out=gc)
+        res["call_plus_gemm_ms_" + key] = round(timed(step, args.steps), 4)
+        plan.close()
+    res["fused_compensation_ms"] = round(res["call_ms_comp_deferred"] - res["call_ms_off"], 4)
+
+    # the compensator as separate torch ops (correction, quantize-dequantize
+    # for the entry error, both EMA updates), rank by rank
+    mf = torch.zeros((w.N,), dtype=torch.float32, device=dev)
+    ms = torch.zeros_like(mf)
+
+    def torch_compensator():
+        for r in range(w.P):
+            c = 0.5 * mf + 0.5 * ms
+            xt = x[r].float() + c
+            g = xt.view(-1, w.G)
+            scale = g.abs().amax(dim=1, keepdim=True) / 7.0
+            k = torch.where(scale > 0, torch.round(g / scale), torch.zeros_like(g)).clamp_(-7, 7)
+            e = (g - k * scale).view(-1)
+            mf.mul_(0.5).add_(0.5 * e)
+            ms.mul_(0.95).add_(0.05 * e)
+    res["torch_ops_compensator_ms"] = round(timed(torch_compensator, max(2, args.steps // 3)), 3)
+    res["note"] = ("call_plus_gemm = one all-reduce followed by the matmul on the same stream; "
+                   "side = owner fix-up on a second stream beside the matmul")
+    print(json.dumps(res), flush=True)
+
+
+def run_depth_chain_mode(args, ws, rank, local):
+    """Deviation from the exact fp32 chain per site, forward and backward."""
+    from bit_error_compensated_echo_b200 import depth_chain
+    if rank != 0:
+        return
+    t0 = time.perf_counter()
+    res = depth_chain.run(P=8, tokens=W.DEPTH.rows, hidden=W.DEPTH.hidden, sites=W.DEPTH.calls,
+                          G=W.DEPTH.G, seed=W.DEPTH.seed, device="cuda:%d" % local)
+    line = {"mode": "depth-chain", "workload": W.DEPTH.name,
+            "seconds": round(time.perf_counter() - t0, 1),
+            "note": "RMS deviation from the exact fp32 chain after each site (and relative "
+                    "Frobenius deviation), compensated / uncompensated 4-bit / bf16 all-reduce"}
+    for k, v in res.items():
+        line[k] = {c: [float("%.4g" % x) for x in arr] for c, arr in v.items()}
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -419,7 +577,10 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="large")
     ap.add_argument("--fixup", choices=("exit", "side", "deferred"), default=BENCH_FIXUP)
     ap.add_argument("--uncompensated", action="store_true")
-    ap.add_argument("--mode", choices=("step",), default="step")
+    ap.add_argument("--mode", choices=("step", "depth-chain", "sweep", "overlap"), default="step")
+    ap.add_argument("--sweep-max-mib", type=int, default=0,
+                    help="sweep only points up to this many MiB per rank (0: all)")
+    ap.add_argument("--sweep-table", default="", help="also write the sweep as a markdown table")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -435,6 +596,12 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             run_reference(args, ws, rank)
+        elif args.mode == "depth-chain":
+            run_depth_chain_mode(args, ws, rank, local)
+        elif args.mode == "sweep":
+            run_sweep_mode(args, ws, rank, local)
+        elif args.mode == "overlap":
+            run_overlap_mode(args, ws, rank, local)
         else:
             run_step_mode(args, ws, rank, local)
     finally:

@@ -1,0 +1,148 @@
+"""Synthetic depth chain: how the all-reduce's error accumulates over sites.
+
+The pages claim the accumulated error stays bounded independently of depth
+when each injected rounding error is fed back into later calls, under the
+assumption that the network does not keep amplifying a perturbation along
+one direction (arXiv abstract on the fugumt mirror; ai4snews news summary,
+"Interpretation" and "Perspective").  This harness measures that on a
+synthetic pre-norm residual chain of tensor-parallel sites, each followed
+by the all-reduce of the P ranks' partial products:
+
+    forward  h_{l+1} = h_l + AR( partial_r = RMSNorm(h_l)[:, B_r] @ W_l[B_r, :] )
+    backward g <- g + J_RMSNorm(h_l)^T AR( partial_r = g[:, B_r] @ W_l^T[B_r, :] )
+
+with W_l Haar-orthogonal (QR of a Gaussian, signs fixed, seeded 1000 + l),
+B_r the r-th block of hidden/P features, RMSNorm with unit weight and
+eps = 1e-6, everything else in fp32.  Orthogonal maps and RMSNorm do not
+amplify perturbations, which is the bound's assumption.  Four chains run
+side by side: the exact chain (fp32 partials summed in fp32), the
+compensated 4-bit all-reduce, the uncompensated one, and a bf16 all-reduce
+(bf16 partials summed in fp32, rounded to bf16).  Per site it reports the
+absolute RMS deviation from the exact chain and the relative Frobenius
+deviation.
+
+The matrix products, RMSNorm and the residual adds are torch (they stand
+in for the model around the all-reduce); the all-reduce is the library's.
+The compensated and uncompensated chains each use their own plan (their own
+state), separate for the forward and the backward pass.
+"""
+from __future__ import annotations
+
+from typing import Dict, List
+
+import torch
+
+from . import workloads as W
+from .api import EchoPlan
+
+EPS = 1e-6
+
+
+def haar_orthogonal(n: int, seed: int, device) -> torch.Tensor:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    a = torch.randn((n, n), generator=g, dtype=torch.float64)
+    q, r = torch.linalg.qr(a)
+    q = q * torch.sign(torch.diagonal(r)).unsqueeze(0)
+    return q.to(torch.float32).to(device)
+
+
+def rmsnorm(h: torch.Tensor) -> torch.Tensor:
+    return h * torch.rsqrt((h * h).mean(dim=-1, keepdim=True) + EPS)
+
+
+def rmsnorm_jt(h: torch.Tensor, u: torch.Tensor) -> torch.Tensor:
+    """J_RMSNorm(h)^T u, row by row (the Jacobian is symmetric):
+    (u - n * <n, u> / d) / rms with n = RMSNorm(h)."""
+    d = h.shape[-1]
+    inv = torch.rsqrt((h * h).mean(dim=-1, keepdim=True) + EPS)
+    n = h * inv
+    return (u - n * (n * u).sum(dim=-1, keepdim=True) / d) * inv
+
+
+def partials(a: torch.Tensor, w: torch.Tensor, P: int, out: torch.Tensor) -> torch.Tensor:
+    """out[r] = a[:, B_r] @ w[B_r, :] for the P feature blocks B_r (fp32)."""
+    d = a.shape[-1]
+    blk = d // P
+    for r in range(P):
+        torch.matmul(a[:, r * blk:(r + 1) * blk], w[r * blk:(r + 1) * blk, :], out=out[r])
+    return out
+
+
+class _Chain:
+    def __init__(self, name, h0, plan=None):
+        self.name, self.h, self.plan = name, h0.clone(), plan
+
+
+def _ar(kind: str, parts32: torch.Tensor, plan, buf_bf16, out_bf16) -> torch.Tensor:
+    """The site's all-reduce of the P partials ([P, T, D] fp32) -> [T, D] fp32."""
+    if kind == "exact":
+        return parts32.sum(dim=0)
+    buf_bf16.copy_(parts32)
+    if kind == "bf16":
+        return buf_bf16.float().sum(dim=0).to(torch.bfloat16).float()
+    P = parts32.shape[0]
+    plan.allreduce(buf_bf16.view(P, -1), out=out_bf16.view(P, -1))
+    return out_bf16[0].float()
+
+
+def _dev(h, ref):
+    diff = (h - ref).double()
+    return (float(diff.pow(2).mean().sqrt()),
+            float(diff.norm() / ref.double().norm().clamp_min(1e-30)))
+
+
+def run(P: int = 8, tokens: int = 32768, hidden: int = 1024, sites: int = 56, G: int = 128,
+        seed: int = 3, device: str = "cuda", backward: bool = True) -> Dict[str, Dict[str, List[float]]]:
+    """Run the four chains; returns {pass: {chain: [rms per site]}, ...}."""
+    dev = torch.device(device)
+    wl = W.Workload("depth", P=1, rows=tokens, hidden=hidden, G=G, seed=seed, dist="student_t")
+    h0 = W.generate(wl, 0, dev)[0].view(tokens, hidden).float()
+    N = tokens * hidden
+    parts = torch.empty((P, tokens, hidden), dtype=torch.float32, device=dev)
+    buf = torch.empty((P, tokens, hidden), dtype=torch.bfloat16, device=dev)
+    out = torch.empty_like(buf)
+    res: Dict[str, Dict[str, List[float]]] = {}
+
+    def one_pass(direction: str, start: torch.Tensor, ws, h_exact_fwd=None):
+        plans = {"comp": EchoPlan(P, N, G, compensate=True, device=dev.index or 0, fixup="deferred"),
+                 "off": EchoPlan(P, N, G, compensate=False, device=dev.index or 0)}
+        chains = [_Chain("exact", start), _Chain("comp", start, plans["comp"]),
+                  _Chain("off", start, plans["off"]), _Chain("bf16", start)]
+        rms = {c.name: [] for c in chains if c.name != "exact"}
+        rel = {c.name: [] for c in chains if c.name != "exact"}
+        try:
+            for step, wmat in enumerate(ws):
+                for c in chains:
+                    if direction == "forward":
+                        partials(rmsnorm(c.h), wmat, P, parts)
+                        c.h = c.h + _ar(c.name, parts, c.plan, buf, out)
+                    else:
+                        partials(c.h, wmat.t().contiguous(), P, parts)
+                        u = _ar(c.name, parts, c.plan, buf, out)
+                        c.h = c.h + rmsnorm_jt(h_exact_fwd[len(ws) - 1 - step], u)
+                ref = chains[0].h
+                for c in chains[1:]:
+                    a, b = _dev(c.h, ref)
+                    rms[c.name].append(a)
+                    rel[c.name].append(b)
+        finally:
+            for p in plans.values():
+                p.close()
+        return chains[0].h, rms, rel
+
+    ws = [haar_orthogonal(hidden, 1000 + l, dev) for l in range(1, sites + 1)]
+    # exact forward activations per site, for the backward Jacobians
+    h_ex = [h0.clone()]
+    for wmat in ws[:-1]:
+        partials(rmsnorm(h_ex[-1]), wmat, P, parts)
+        h_ex.append(h_ex[-1] + parts.sum(dim=0))
+    _, rms_f, rel_f = one_pass("forward", h0, ws)
+    res["forward_rms"], res["forward_rel"] = rms_f, rel_f
+    if backward:
+        wg = W.Workload("depth_grad", P=1, rows=tokens, hidden=hidden, G=G, seed=seed + 100,
+                        dist="student_t")
+        g0 = W.generate(wg, 0, dev)[0].view(tokens, hidden).float()
+        _, rms_b, rel_b = one_pass("backward", g0, list(reversed(ws)), h_exact_fwd=h_ex)
+        res["backward_rms"], res["backward_rel"] = rms_b, rel_b
+    return res
