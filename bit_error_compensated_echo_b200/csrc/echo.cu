@@ -103,6 +103,8 @@ struct echo_plan {
     bool side_inflight = false;      // a side-stream fix-up may still run
     cudaEvent_t ev_reduced = nullptr, ev_side_done = nullptr;
     void *stage = nullptr;           // host-call staging: [P][N] in, [P][N] out
+    cudaStream_t hstream[3] = {nullptr, nullptr, nullptr};  // host call: copy in, compute, copy out
+    cudaEvent_t hev[2 * 16 + 2] = {};                       // host call: per-slab and boundary events
     bool profiling = false;
     std::vector<ProfRecord> records;
     std::vector<cudaEvent_t> pool;
@@ -135,87 +137,91 @@ cudaEvent_t take_event(echo_plan *p) {
 }
 
 template <int G, bool COMP, bool DEFER>
-void launch_entry_t(echo_plan *p, const InPtrs &x, cudaStream_t st) {
-    dim3 grid((unsigned)((p->n_vec + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
+void launch_entry_t(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st) {
+    dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)(p->cfg.P * p->cfg.P));
     echo_entry_kernel<G, COMP, DEFER><<<grid, kThreads, 0, st>>>(
-        x, p->m_fast, p->m_slow, p->codes, p->scales, p->e_req, p->n_vec, p->chunk_vec, p->k);
+        x, p->m_fast, p->m_slow, p->codes, p->scales, p->e_req, p->n_vec, p->chunk_vec, sl,
+        p->cfg.P, p->k);
 }
 
 template <int G>
-void launch_entry_g(echo_plan *p, const InPtrs &x, cudaStream_t st, bool defer) {
-    if (!p->cfg.compensate) launch_entry_t<G, false, false>(p, x, st);
-    else if (defer) launch_entry_t<G, true, true>(p, x, st);
-    else launch_entry_t<G, true, false>(p, x, st);
+void launch_entry_g(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
+    if (!p->cfg.compensate) launch_entry_t<G, false, false>(p, x, sl, st);
+    else if (defer) launch_entry_t<G, true, true>(p, x, sl, st);
+    else launch_entry_t<G, true, false>(p, x, sl, st);
 }
 
-void launch_entry(echo_plan *p, const InPtrs &x, cudaStream_t st, bool defer) {
+void launch_entry(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
     switch (p->cfg.G) {
-        case 32: launch_entry_g<32>(p, x, st, defer); break;
-        case 64: launch_entry_g<64>(p, x, st, defer); break;
-        default: launch_entry_g<128>(p, x, st, defer); break;
+        case 32: launch_entry_g<32>(p, x, sl, st, defer); break;
+        case 64: launch_entry_g<64>(p, x, sl, st, defer); break;
+        default: launch_entry_g<128>(p, x, sl, st, defer); break;
     }
 }
 
 template <int G, int P>
-void launch_reduce_t(echo_plan *p, cudaStream_t st) {
-    dim3 grid(reduce_blocks(p->chunk_vec), (unsigned)P);
+void launch_reduce_t(echo_plan *p, Slab sl, cudaStream_t st) {
+    dim3 grid(reduce_blocks(sl.v_count), (unsigned)P);
     if (p->cfg.compensate)
         echo_reduce_kernel<G, P, true><<<grid, kThreads, 0, st>>>(
-            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec);
+            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl);
     else
         echo_reduce_kernel<G, P, false><<<grid, kThreads, 0, st>>>(
-            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec);
+            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl);
 }
 
 template <int G>
-void launch_reduce_g(echo_plan *p, cudaStream_t st) {
+void launch_reduce_g(echo_plan *p, Slab sl, cudaStream_t st) {
     switch (p->cfg.P) {
-        case 1: launch_reduce_t<G, 1>(p, st); break;
-        case 2: launch_reduce_t<G, 2>(p, st); break;
-        case 3: launch_reduce_t<G, 3>(p, st); break;
-        case 4: launch_reduce_t<G, 4>(p, st); break;
-        case 5: launch_reduce_t<G, 5>(p, st); break;
-        case 6: launch_reduce_t<G, 6>(p, st); break;
-        case 7: launch_reduce_t<G, 7>(p, st); break;
-        default: launch_reduce_t<G, 8>(p, st); break;
+        case 1: launch_reduce_t<G, 1>(p, sl, st); break;
+        case 2: launch_reduce_t<G, 2>(p, sl, st); break;
+        case 3: launch_reduce_t<G, 3>(p, sl, st); break;
+        case 4: launch_reduce_t<G, 4>(p, sl, st); break;
+        case 5: launch_reduce_t<G, 5>(p, sl, st); break;
+        case 6: launch_reduce_t<G, 6>(p, sl, st); break;
+        case 7: launch_reduce_t<G, 7>(p, sl, st); break;
+        default: launch_reduce_t<G, 8>(p, sl, st); break;
     }
 }
 
-void launch_reduce(echo_plan *p, cudaStream_t st) {
+void launch_reduce(echo_plan *p, Slab sl, cudaStream_t st) {
     switch (p->cfg.G) {
-        case 32: launch_reduce_g<32>(p, st); break;
-        case 64: launch_reduce_g<64>(p, st); break;
-        default: launch_reduce_g<128>(p, st); break;
+        case 32: launch_reduce_g<32>(p, sl, st); break;
+        case 64: launch_reduce_g<64>(p, sl, st); break;
+        default: launch_reduce_g<128>(p, sl, st); break;
     }
 }
 
 template <int G>
-void launch_exit_g(echo_plan *p, const OutPtrs &out, cudaStream_t st, bool fix) {
-    dim3 grid((unsigned)((p->chunk_vec + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
+void launch_exit_g(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+    dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
     if (fix)
         echo_exit_kernel<G, true><<<grid, kThreads, 0, st>>>(
             p->rcodes, p->rscales, out, p->cfg.P, p->m_fast, p->m_slow, p->e_req, p->n_vec,
-            p->chunk_vec, p->k);
+            p->chunk_vec, sl, p->k);
     else
         echo_exit_kernel<G, false><<<grid, kThreads, 0, st>>>(
             p->rcodes, p->rscales, out, p->cfg.P, p->m_fast, p->m_slow, p->e_req, p->n_vec,
-            p->chunk_vec, p->k);
+            p->chunk_vec, sl, p->k);
 }
 
-void launch_exit(echo_plan *p, const OutPtrs &out, cudaStream_t st, bool fix) {
+void launch_exit(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
     switch (p->cfg.G) {
-        case 32: launch_exit_g<32>(p, out, st, fix); break;
-        case 64: launch_exit_g<64>(p, out, st, fix); break;
-        default: launch_exit_g<128>(p, out, st, fix); break;
+        case 32: launch_exit_g<32>(p, out, sl, st, fix); break;
+        case 64: launch_exit_g<64>(p, out, sl, st, fix); break;
+        default: launch_exit_g<128>(p, out, sl, st, fix); break;
     }
 }
 
 void launch_fixup(echo_plan *p, const float *sf, const float *ss, float *df, float *ds, bool apply,
-                  bool only_owner, cudaStream_t st) {
-    dim3 grid((unsigned)((p->chunk_vec + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
+                  bool only_owner, Slab sl, cudaStream_t st) {
+    dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
     echo_fixup_kernel<<<grid, kThreads, 0, st>>>(sf, ss, df, ds, p->e_req, p->n_vec, p->chunk_vec,
-                                                 p->cfg.P, apply ? 1 : 0, only_owner ? 1 : 0, p->k);
+                                                 sl, p->cfg.P, apply ? 1 : 0, only_owner ? 1 : 0,
+                                                 p->k);
 }
+
+Slab whole(const echo_plan *p) { return Slab{0, p->chunk_vec}; }
 
 bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 
@@ -306,6 +312,10 @@ echo_status echo_plan_destroy(echo_plan *p) {
         for (auto ev : r.ev)
             if (ev) cudaEventDestroy(ev);
     for (auto ev : p->pool) cudaEventDestroy(ev);
+    for (auto ev : p->hev)
+        if (ev) cudaEventDestroy(ev);
+    for (auto hs : p->hstream)
+        if (hs) cudaStreamDestroy(hs);
     if (p->ev_reduced) cudaEventDestroy(p->ev_reduced);
     if (p->ev_side_done) cudaEventDestroy(p->ev_side_done);
     if (p->stage) cudaFree(p->stage);
@@ -360,17 +370,17 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
     const bool defer = comp && mode == ECHO_FIXUP_DEFERRED && p->pending;
 
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[0], st));
-    launch_entry(p, xi, st, defer);
+    launch_entry(p, xi, whole(p), st, defer);
     ECHO_TRY(cudaGetLastError());
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[1], st));
-    launch_reduce(p, st);
+    launch_reduce(p, whole(p), st);
     ECHO_TRY(cudaGetLastError());
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[2], st));
 
     const bool fix_in_exit = comp && mode == ECHO_FIXUP_EXIT;
     const bool fix_on_side = comp && mode == ECHO_FIXUP_SIDE;
     if (fix_on_side && side) ECHO_TRY(cudaEventRecord(p->ev_reduced, st));
-    launch_exit(p, yo, st, fix_in_exit);
+    launch_exit(p, yo, whole(p), st, fix_in_exit);
     ECHO_TRY(cudaGetLastError());
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[3], st));
 
@@ -384,7 +394,7 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
             rec.side = true;
             ECHO_TRY(cudaEventRecord(rec.ev[4], fs));
         }
-        launch_fixup(p, p->m_fast, p->m_slow, p->m_fast, p->m_slow, true, true, fs);
+        launch_fixup(p, p->m_fast, p->m_slow, p->m_fast, p->m_slow, true, true, whole(p), fs);
         ECHO_TRY(cudaGetLastError());
         if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[5], fs));
         if (side) {
@@ -416,18 +426,65 @@ echo_status echo_allreduce_host(echo_plan *p, const void *const *in_host, void *
             return from_cuda(e);
         }
     }
+    if (!p->hstream[0]) {
+        for (auto &hs : p->hstream) ECHO_TRY(cudaStreamCreateWithFlags(&hs, cudaStreamNonBlocking));
+        for (auto &ev : p->hev) ECHO_TRY(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    }
     cudaStream_t st = (cudaStream_t)stream;
-    const void *din[ECHO_MAX_RANKS];
-    void *dout[ECHO_MAX_RANKS];
+    cudaStream_t s_in = p->hstream[0], s_comp = p->hstream[1], s_out = p->hstream[2];
+    cudaEvent_t ev_start = p->hev[32], ev_done = p->hev[33];
+
+    InPtrs xi{};
+    OutPtrs yo{};
+    char *din[ECHO_MAX_RANKS];
+    char *dout[ECHO_MAX_RANKS];
     for (int r = 0; r < P; ++r) {
         din[r] = (char *)p->stage + (size_t)r * bytes;
         dout[r] = (char *)p->stage + (size_t)(P + r) * bytes;
-        ECHO_TRY(cudaMemcpyAsync((void *)din[r], in_host[r], bytes, cudaMemcpyHostToDevice, st));
+        xi.p[r] = (const uint4 *)din[r];
+        yo.p[r] = (uint4 *)dout[r];
     }
-    echo_status s = echo_allreduce(p, din, dout, stream, nullptr);
-    if (s != ECHO_OK) return s;
-    for (int r = 0; r < P; ++r)
-        ECHO_TRY(cudaMemcpyAsync(out_host[r], dout[r], bytes, cudaMemcpyDeviceToHost, st));
+
+    // Slab k is vectors [k*sv, (k+1)*sv) of every owner chunk: one strided
+    // copy per rank moves it (P rows of sv*16 bytes, pitch chunk_vec*16).
+    const int64_t align = p->cfg.G / kVec;  // slab edges on group edges (and even)
+    int64_t nslab = 16;
+    if (p->chunk_vec / align < nslab) nslab = p->chunk_vec / align;
+    int64_t sv = (p->chunk_vec + nslab - 1) / nslab;
+    sv = (sv + align - 1) / align * align;
+    const size_t pitch = (size_t)p->chunk_vec * 16;
+
+    ECHO_TRY(cudaEventRecord(ev_start, st));
+    for (auto hs : p->hstream) ECHO_TRY(cudaStreamWaitEvent(hs, ev_start, 0));
+    ECHO_TRY(order_after_side(p, s_comp));
+    p->side_inflight = false;
+    const bool comp = p->cfg.compensate != 0;
+    const bool deferred = comp && p->cfg.fixup == ECHO_FIXUP_DEFERRED;
+    const bool defer = deferred && p->pending;
+    for (int64_t k = 0; k < nslab; ++k) {
+        const int64_t vb = k * sv;
+        if (vb >= p->chunk_vec) break;
+        const int64_t vc = vb + sv <= p->chunk_vec ? sv : p->chunk_vec - vb;
+        const Slab sl{vb, vc};
+        const size_t off = (size_t)vb * 16, width = (size_t)vc * 16;
+        for (int r = 0; r < P; ++r)
+            ECHO_TRY(cudaMemcpy2DAsync(din[r] + off, pitch, (const char *)in_host[r] + off, pitch,
+                                       width, (size_t)P, cudaMemcpyHostToDevice, s_in));
+        ECHO_TRY(cudaEventRecord(p->hev[2 * k], s_in));
+        ECHO_TRY(cudaStreamWaitEvent(s_comp, p->hev[2 * k], 0));
+        launch_entry(p, xi, sl, s_comp, defer);
+        launch_reduce(p, sl, s_comp);
+        launch_exit(p, yo, sl, s_comp, comp && !deferred);
+        ECHO_TRY(cudaGetLastError());
+        ECHO_TRY(cudaEventRecord(p->hev[2 * k + 1], s_comp));
+        ECHO_TRY(cudaStreamWaitEvent(s_out, p->hev[2 * k + 1], 0));
+        for (int r = 0; r < P; ++r)
+            ECHO_TRY(cudaMemcpy2DAsync((char *)out_host[r] + off, pitch, dout[r] + off, pitch,
+                                       width, (size_t)P, cudaMemcpyDeviceToHost, s_out));
+    }
+    ECHO_TRY(cudaEventRecord(ev_done, s_out));
+    ECHO_TRY(cudaStreamWaitEvent(st, ev_done, 0));
+    if (deferred) p->pending = true;
     return ECHO_OK;
 }
 
@@ -452,7 +509,7 @@ echo_status echo_get_state(echo_plan *p, float *m_fast, float *m_slow, void *str
     if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     ECHO_TRY(order_after_side(p, st));
-    launch_fixup(p, p->m_fast, p->m_slow, m_fast, m_slow, p->pending, false, st);
+    launch_fixup(p, p->m_fast, p->m_slow, m_fast, m_slow, p->pending, false, whole(p), st);
     ECHO_TRY(cudaGetLastError());
     return ECHO_OK;
 }

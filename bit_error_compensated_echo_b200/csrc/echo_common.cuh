@@ -34,6 +34,16 @@ struct OutPtrs {
     uint4 *p[kMaxRanks];
 };
 
+// A slab: the vectors [v_begin, v_begin + v_count) of every owner chunk
+// (a vector is 8 elements; owner chunk o is vectors [o*chunk_vec,
+// (o+1)*chunk_vec) of every rank).  A whole call is the slab (0, chunk_vec);
+// the host-buffer call pipelines copies and kernels slab by slab.  Both
+// bounds are multiples of G/8 and even, so groups and 16-element runs never
+// straddle a slab edge.
+struct Slab {
+    int64_t v_begin, v_count;
+};
+
 struct Consts {
     float alpha, one_m_alpha;
     float beta_fast, one_m_beta_fast;

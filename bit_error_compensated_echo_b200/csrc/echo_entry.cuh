@@ -9,7 +9,7 @@ namespace echo {
 // ------------------------------------------------------------ echo_entry
 //
 // Correction add + group quantize + pack + partial EMA update, for every
-// rank.  Grid: x over the N/8 vectors of a rank, y = rank.
+// rank.  Grid: x over the slab's vectors, y = rank * P + owner chunk.
 //   COMP  : compensator on (read/write the states)
 //   DEFER : apply the previous call's pending owner fix-up first
 //           (state += (1-beta)*e_req on this rank's own chunk), which is the
@@ -19,11 +19,12 @@ __global__ void __launch_bounds__(kThreads, COMP ? 5 : 8)
 echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_slow,
                   uint32_t *__restrict__ codes, float *__restrict__ scales,
                   const float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec,
-                  Consts k) {
+                  Slab sl, int P, Consts k) {
     constexpr int LANES = G / kVec;
-    const int r = blockIdx.y;
-    const int64_t j = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    const bool valid = j < n_vec;
+    const int r = blockIdx.y / P, o = blockIdx.y % P;  // rank, owner chunk
+    const int64_t l = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    const bool valid = l < sl.v_count;
+    const int64_t j = (int64_t)o * chunk_vec + sl.v_begin + l;  // vector in rank r
 
     float xt[8], mf[8], ms[8];
     if (valid) {
@@ -32,7 +33,7 @@ echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_sl
             const int64_t e0 = ((int64_t)r * n_vec + j) * kVec;
             ld8(m_fast + e0, mf);
             ld8(m_slow + e0, ms);
-            if (DEFER && j >= r * chunk_vec && j < (r + 1) * chunk_vec) {
+            if (DEFER && o == r) {
                 float er[8];
                 ld8(e_req + j * kVec, er);
 #pragma unroll

@@ -11,17 +11,18 @@ namespace echo {
 // All-gather half: dequantize the reduced codes once to bf16 and write them
 // to all P outputs.  FIX: also apply the owner's fix-up of both EMAs
 // (state += (1-beta)*e_req) for the owner's chunk.
-// Grid: x over the vectors of one owner chunk, y = owner.
+// Grid: x over the vectors of the slab, y = owner.
 template <int G, bool FIX>
 __global__ void __launch_bounds__(kThreads)
 echo_exit_kernel(const uint32_t *__restrict__ rcodes, const float *__restrict__ rscales,
                  OutPtrs out, int P, float *__restrict__ m_fast, float *__restrict__ m_slow,
-                 const float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec, Consts k) {
+                 const float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec, Slab sl,
+                 Consts k) {
     constexpr int LANES = G / kVec;
     const int o = blockIdx.y;
     const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (local >= chunk_vec) return;
-    const int64_t j = (int64_t)o * chunk_vec + local;
+    if (local >= sl.v_count) return;
+    const int64_t j = (int64_t)o * chunk_vec + sl.v_begin + local;
 
     const uint32_t w = __ldg(rcodes + j);
     const float2 sc2 = splat2(__ldg(rscales + j / LANES));

@@ -11,19 +11,19 @@ namespace echo {
 // The owner fix-up alone, as its own launch (side-stream mode), or, with
 // dst != src, a copy of the states that applies a pending fix-up on the way
 // (reading the state of a plan in deferred mode).  Grid: x over the vectors
-// of one owner chunk, y = rank; only rank == owner adds the fix-up.
+// of the slab, y = owner chunk; only rank == owner adds the fix-up.
 __global__ void __launch_bounds__(kThreads)
 echo_fixup_kernel(const float *__restrict__ src_fast, const float *__restrict__ src_slow,
                   float *__restrict__ dst_fast, float *__restrict__ dst_slow,
                   const float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec,
-                  int P, int apply, int only_owner, Consts k) {
+                  Slab sl, int P, int apply, int only_owner, Consts k) {
     const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (local >= chunk_vec) return;
+    if (local >= sl.v_count) return;
     const int o = blockIdx.y;
     for (int r = 0; r < P; ++r) {
         const bool own = (r == o);
         if (only_owner && !own) continue;
-        const int64_t j = (int64_t)o * chunk_vec + local;
+        const int64_t j = (int64_t)o * chunk_vec + sl.v_begin + local;
         const int64_t e0 = ((int64_t)r * n_vec + j) * kVec;
         float mf[8], ms[8];
         ld8(src_fast + e0, mf);

@@ -14,26 +14,26 @@ namespace echo {
 // Each thread owns 16 consecutive elements: one 8-byte word pair of codes
 // per rank, all P loads issued before any arithmetic so that every thread
 // keeps P*8 bytes of the transport in flight.
-// Grid: x over the N/(16P) runs of one owner chunk, y = owner.
+// Grid: x over the 16-element runs of the slab, y = owner.
 constexpr int kRedVec = 16;
 
-// blocks along x for an owner chunk of chunk_vec 8-element vectors
-inline unsigned reduce_blocks(int64_t chunk_vec) {
-    return (unsigned)((chunk_vec / 2 + kThreads - 1) / kThreads);
+// blocks along x for a slab of v_count 8-element vectors
+inline unsigned reduce_blocks(int64_t v_count) {
+    return (unsigned)((v_count / 2 + kThreads - 1) / kThreads);
 }
 
 template <int G, int P, bool COMP>
 __global__ void __launch_bounds__(kThreads)
 echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
                    uint32_t *__restrict__ rcodes, float *__restrict__ rscales,
-                   float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec) {
+                   float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec, Slab sl) {
     constexpr int LANES = G / kRedVec;              // lanes per group
     const int o = blockIdx.y;
     const int64_t n_run = n_vec / 2;                // 16-element runs per rank
     const int64_t chunk_run = chunk_vec / 2;        // runs per owner chunk
     const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    const bool valid = local < chunk_run;
-    const int64_t j = (int64_t)o * chunk_run + local;  // run index in a rank
+    const bool valid = local < sl.v_count / 2;
+    const int64_t j = (int64_t)o * chunk_run + sl.v_begin / 2 + local;  // run index in a rank
     const int64_t n_groups = n_run / LANES;
     const uint2 *codes2 = reinterpret_cast<const uint2 *>(codes);
 

@@ -139,12 +139,18 @@ echo_status echo_allreduce(echo_plan *plan, const void *const *in_device,
                            void *const *out_device, void *stream,
                            void *side_stream);
 
-/* The same call on host buffers: copies the P inputs host -> device into a
- * staging area the plan allocates on first use (2*P*N*2 bytes, kept until
- * echo_plan_destroy), runs echo_allreduce on stream, and copies the P
- * outputs device -> host.  in_host[r], out_host[r]: N bf16 elements each;
- * pinned host memory makes the copies asynchronous, pageable memory makes
- * them synchronous.  The caller synchronizes stream before reading out_host.
+/* The same call on host buffers, pipelined: the call is cut into up to 16
+ * slabs (the same sub-range of every owner chunk); each slab's inputs are
+ * copied host -> device, its three kernels run, and its outputs are copied
+ * device -> host, on three internal streams, so copies in both directions
+ * overlap each other and the kernels.  The staging area (2*P*N*2 bytes) and
+ * the internal streams and events are created on first use and kept until
+ * echo_plan_destroy.  The work starts after everything already queued on
+ * stream, and stream waits for its end: synchronize stream before reading
+ * out_host.  in_host[r], out_host[r]: N bf16 elements each; pinned host
+ * memory makes the copies asynchronous, pageable memory makes them
+ * synchronous.  Results, codes and states equal echo_allreduce's; with
+ * ECHO_FIXUP_SIDE the fix-up runs in the exit kernel here.
  * Errors: INVALID_ARG, OOM (staging), CUDA. */
 echo_status echo_allreduce_host(echo_plan *plan, const void *const *in_host,
                                 void *const *out_host, void *stream);

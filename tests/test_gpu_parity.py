@@ -199,16 +199,38 @@ def test_state_roundtrip_and_reset():
         assert not plan.debug_view()["fixup_pending"]
 
 
-def test_host_call_matches_device_call():
-    w = W.with_size(W.TINY, P=4, rows=1, hidden=4 * 128 * 20, G=128)
-    with _plan(w.P, w.N, w.G) as a, _plan(w.P, w.N, w.G) as b:
-        for t in range(3):
+@pytest.mark.parametrize("fixup", ["exit", "side", "deferred"])
+@pytest.mark.parametrize("P,G,k", [(4, 128, 20), (3, 32, 37), (8, 64, 5), (2, 128, 1)],
+                         ids=lambda v: str(v))
+def test_host_call_matches_device_call(fixup, P, G, k):
+    """The pipelined host-buffer call (slabs of every owner chunk, copies
+    and kernels overlapped on three streams) gives the device call's bytes
+    and states, call after call, including ragged last slabs."""
+    N = P * G * k
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    side = torch.cuda.Stream()
+    with _plan(P, N, G, True, fixup) as a, _plan(P, N, G, True, fixup) as b:
+        yh = torch.empty((P, N), dtype=torch.bfloat16, pin_memory=True)
+        for t in range(4):
             x = W.generate(w, t, DEV)
-            yd = a.allreduce(x)
+            yd = a.allreduce(x, side_stream=side)
             xh = x.cpu().pin_memory()
-            yh = b.allreduce_host(xh)
+            b.allreduce_host(xh, yh)
             torch.cuda.synchronize()
-            assert torch.equal(yd.cpu(), yh)
+            assert torch.equal(yd.cpu(), yh), t
+            ma, mb = a.get_state(), b.get_state()
+            torch.cuda.synchronize()
+            assert torch.equal(ma[0], mb[0]) and torch.equal(ma[1], mb[1]), t
+
+
+def test_host_call_uncompensated_large_slabs():
+    w = W.with_size(W.TINY, P=8, rows=1, hidden=8 * 128 * 1000, G=128)
+    with _plan(w.P, w.N, w.G, False) as a, _plan(w.P, w.N, w.G, False) as b:
+        x = W.generate(w, 0, DEV)
+        yd = a.allreduce(x)
+        yh = b.allreduce_host(x.cpu().pin_memory())
+        torch.cuda.synchronize()
+        assert torch.equal(yd.cpu(), yh)
 
 
 def test_profile_counts_launches():
