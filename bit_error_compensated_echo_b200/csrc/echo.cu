@@ -164,10 +164,12 @@ void launch_reduce_t(echo_plan *p, Slab sl, cudaStream_t st) {
     dim3 grid(reduce_blocks(sl.v_count), (unsigned)P);
     if (p->cfg.compensate)
         echo_reduce_kernel<G, P, true><<<grid, kThreads, 0, st>>>(
-            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl);
+            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl,
+            p->k.neg_zero);
     else
         echo_reduce_kernel<G, P, false><<<grid, kThreads, 0, st>>>(
-            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl);
+            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl,
+            p->k.neg_zero);
 }
 
 template <int G>
@@ -272,6 +274,7 @@ echo_status echo_plan_create(echo_plan **out, const echo_config *cfg) {
     p->k.one_m_beta_fast = 1.0f - cfg->beta_fast;
     p->k.beta_slow = cfg->beta_slow;
     p->k.one_m_beta_slow = 1.0f - cfg->beta_slow;
+    p->k.neg_zero = -0.0f;
 
     cudaError_t e = cudaMalloc((void **)&p->ws, p->L.total);
     if (e != cudaSuccess) {

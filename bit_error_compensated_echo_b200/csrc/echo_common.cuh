@@ -48,6 +48,7 @@ struct Consts {
     float alpha, one_m_alpha;
     float beta_fast, one_m_beta_fast;
     float beta_slow, one_m_beta_slow;
+    float neg_zero;   // -0.0f, passed at run time (see prod2)
 };
 
 // ------------------------------------------------------------ helpers
@@ -78,10 +79,11 @@ __device__ __forceinline__ float group_absmax(float a) {
 // nearest even (subnormals kept), so a pair op gives exactly the two scalar
 // results; it issues once for both.  ptxas contracts a packed multiply whose
 // result feeds a packed add or subtract into one fused multiply-add (single
-// rounding) even with explicit .rn, so a pair multiply is only ever used
-// where its result goes through a min/max or a conversion first; every
-// multiply-then-add of the definition uses the scalar __fmul_rn/__fadd_rn,
-// which are never contracted.
+// rounding) even with explicit .rn, so a product that feeds an add is
+// written as prod2: a packed fma whose addend is -0 held in a register that
+// is only known at run time.  a*b + (-0) rounds exactly like a*b (also for
+// signed zeros), and ptxas cannot fold an addend it does not know, so the
+// product stays separately rounded.
 __device__ __forceinline__ float2 add2(float2 a, float2 b) {
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -104,6 +106,17 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     return d;
 }
 __device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+// the separately rounded products a.x*b.x, a.y*b.y; z must hold the run-time
+// value (-0.0f, -0.0f)
+__device__ __forceinline__ float2 prod2(float2 a, float2 b, float2 z) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rz, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rz, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rz;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(z.x), "f"(z.y));
+    return d;
+}
 
 // ---- exact integer <-> float steps without conversion instructions
 //
@@ -212,25 +225,26 @@ __device__ __forceinline__ uint32_t quantize8_exact(const float v[8], float scal
     return w;
 }
 
-__device__ __forceinline__ uint32_t quantize8(const float v[8], const GroupScale &g, float kf[8]) {
+// For a normal scale, |v*inv| <= 7*(1 + 2^-22) < 7.5, so no clamp is needed
+// on the fast path (the exact path keeps it).
+__device__ __forceinline__ uint32_t quantize8(const float v[8], const GroupScale &g, float kf[8],
+                                              float2 z) {
     uint32_t w = 0;
-    bool near_tie = g.exact;
     const float2 inv2 = splat2(g.inv), magic2 = splat2(kRoundMagic);
+    float dmax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-        float2 q = mul2(make_float2(v[i], v[i + 1]), inv2);
-        q.x = fminf(fmaxf(q.x, -7.0f), 7.0f);
-        q.y = fminf(fmaxf(q.y, -7.0f), 7.0f);
+        const float2 q = prod2(make_float2(v[i], v[i + 1]), inv2, z);
         const float2 t = add2(q, magic2);
         const float2 k = sub2(t, magic2);
         const float2 d = sub2(q, k);
         kf[i] = k.x;
         kf[i + 1] = k.y;
-        near_tie |= fmaxf(fabsf(d.x), fabsf(d.y)) > 0.5f - 0x1p-18f;
+        dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
         w |= (__float_as_uint(t.x) & 0xfu) << (4 * i);
         w |= (__float_as_uint(t.y) & 0xfu) << (4 * i + 4);
     }
-    if (near_tie) w = quantize8_exact(v, g.scale, kf);
+    if (g.exact || dmax > 0.5f - 0x1p-18f) w = quantize8_exact(v, g.scale, kf);
     return w;
 }
 

@@ -83,14 +83,14 @@ void launch_all(const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigne
         echo_entry_kernel<G, true, false><<<g_entry, kThreads, 0, st>>>(
             x, mf, ms, codes, scales, e_req, n_vec, chunk_vec, sl, P, k);
         echo_reduce_kernel<G, P, true><<<g_red, kThreads, 0, st>>>(
-            codes, scales, rcodes, rscales, e_req, n_vec, chunk_vec, sl);
+            codes, scales, rcodes, rscales, e_req, n_vec, chunk_vec, sl, k.neg_zero);
         echo_exit_kernel<G, true><<<g_chunk, kThreads, 0, st>>>(
             rcodes, rscales, y, P, mf, ms, e_req, n_vec, chunk_vec, sl, k);
     } else {
         echo_entry_kernel<G, false, false><<<g_entry, kThreads, 0, st>>>(
             x, nullptr, nullptr, codes, scales, nullptr, n_vec, chunk_vec, sl, P, k);
         echo_reduce_kernel<G, P, false><<<g_red, kThreads, 0, st>>>(
-            codes, scales, rcodes, rscales, nullptr, n_vec, chunk_vec, sl);
+            codes, scales, rcodes, rscales, nullptr, n_vec, chunk_vec, sl, k.neg_zero);
         echo_exit_kernel<G, false><<<g_chunk, kThreads, 0, st>>>(
             rcodes, rscales, y, P, nullptr, nullptr, nullptr, n_vec, chunk_vec, sl, k);
     }
@@ -164,6 +164,7 @@ extern "C" echo_status echo_allreduce_noalloc(const echo_config *cfg, const void
         k.one_m_beta_fast = 1.0f - cfg->beta_fast;
         k.beta_slow = cfg->beta_slow;
         k.one_m_beta_slow = 1.0f - cfg->beta_slow;
+        k.neg_zero = -0.0f;
         cudaStream_t st = (cudaStream_t)stream;
         switch (G) {
             case 32: launch_g<32>(P, x, y, m_fast_device, m_slow_device, scratch, L, N, comp, k, st); break;

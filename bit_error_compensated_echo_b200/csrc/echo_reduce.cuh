@@ -26,7 +26,8 @@ template <int G, int P, bool COMP>
 __global__ void __launch_bounds__(kThreads)
 echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
                    uint32_t *__restrict__ rcodes, float *__restrict__ rscales,
-                   float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec, Slab sl) {
+                   float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec, Slab sl,
+                   float neg_zero) {
     constexpr int LANES = G / kRedVec;              // lanes per group
     const int o = blockIdx.y;
     const int64_t n_run = n_vec / 2;                // 16-element runs per rank
@@ -44,21 +45,26 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
         w[r] = valid ? __ldcs(codes2 + (int64_t)r * n_run + j) : make_uint2(0u, 0u);
         sc[r] = valid ? __ldg(scales + (int64_t)r * n_groups + j / LANES) : 0.0f;
     }
-    float s[16];
+    const float2 z = splat2(neg_zero);
+    float2 s2[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s[i] = 0.0f;
+    for (int i = 0; i < 8; ++i) s2[i] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int r = 0; r < P; ++r) {
+        const float2 sc2 = splat2(sc[r]);
         const uint32_t lx = low_nibbles(w[r].x), hx = high_nibbles(w[r].x);
         const uint32_t ly = low_nibbles(w[r].y), hy = high_nibbles(w[r].y);
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            const float2 kx = code_pair(lx, hx, p), ky = code_pair(ly, hy, p);
-            s[2 * p] = __fadd_rn(s[2 * p], __fmul_rn(kx.x, sc[r]));
-            s[2 * p + 1] = __fadd_rn(s[2 * p + 1], __fmul_rn(kx.y, sc[r]));
-            s[8 + 2 * p] = __fadd_rn(s[8 + 2 * p], __fmul_rn(ky.x, sc[r]));
-            s[9 + 2 * p] = __fadd_rn(s[9 + 2 * p], __fmul_rn(ky.y, sc[r]));
+            s2[p] = add2(s2[p], prod2(code_pair(lx, hx, p), sc2, z));
+            s2[4 + p] = add2(s2[4 + p], prod2(code_pair(ly, hy, p), sc2, z));
         }
+    }
+    float s[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        s[2 * i] = s2[i].x;
+        s[2 * i + 1] = s2[i].y;
     }
 
     float a = 0.0f;
@@ -68,8 +74,8 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
     const GroupScale gs = make_group_scale(a);
     const float scale2 = gs.scale;
     float k2[16];
-    const uint32_t w0 = quantize8(s, gs, k2);
-    const uint32_t w1 = quantize8(s + 8, gs, k2 + 8);
+    const uint32_t w0 = quantize8(s, gs, k2, z);
+    const uint32_t w1 = quantize8(s + 8, gs, k2 + 8, z);
     if (!valid) return;
 
     reinterpret_cast<uint2 *>(rcodes)[j] = make_uint2(w0, w1);
