@@ -138,7 +138,7 @@ cudaEvent_t take_event(echo_plan *p) {
 
 template <int G, bool COMP, bool DEFER>
 void launch_entry_t(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st) {
-    dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)(p->cfg.P * p->cfg.P));
+    dim3 grid(entry_blocks<COMP>(sl.v_count), (unsigned)(p->cfg.P * p->cfg.P));
     echo_entry_kernel<G, COMP, DEFER><<<grid, kThreads, 0, st>>>(
         x, p->m_fast, p->m_slow, p->codes, p->scales, p->e_req, p->n_vec, p->chunk_vec, sl,
         p->cfg.P, p->k);

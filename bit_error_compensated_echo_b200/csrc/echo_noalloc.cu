@@ -76,18 +76,19 @@ void launch_all(const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigne
     float *rscales = (float *)(s + L.rscales);
     float *e_req = comp ? (float *)(s + L.e_req) : nullptr;
     const Slab sl{0, chunk_vec};
-    dim3 g_entry((unsigned)((chunk_vec + kThreads - 1) / kThreads), (unsigned)(P * P));
+    dim3 g_entry_c(entry_blocks<true>(chunk_vec), (unsigned)(P * P));
+    dim3 g_entry_o(entry_blocks<false>(chunk_vec), (unsigned)(P * P));
     dim3 g_chunk((unsigned)((chunk_vec + kThreads - 1) / kThreads), (unsigned)P);
     dim3 g_red(reduce_blocks(chunk_vec), (unsigned)P);
     if (comp) {
-        echo_entry_kernel<G, true, false><<<g_entry, kThreads, 0, st>>>(
+        echo_entry_kernel<G, true, false><<<g_entry_c, kThreads, 0, st>>>(
             x, mf, ms, codes, scales, e_req, n_vec, chunk_vec, sl, P, k);
         echo_reduce_kernel<G, P, true><<<g_red, kThreads, 0, st>>>(
             codes, scales, rcodes, rscales, e_req, n_vec, chunk_vec, sl, k.neg_zero);
         echo_exit_kernel<G, true><<<g_chunk, kThreads, 0, st>>>(
             rcodes, rscales, y, P, mf, ms, e_req, n_vec, chunk_vec, sl, k);
     } else {
-        echo_entry_kernel<G, false, false><<<g_entry, kThreads, 0, st>>>(
+        echo_entry_kernel<G, false, false><<<g_entry_o, kThreads, 0, st>>>(
             x, nullptr, nullptr, codes, scales, nullptr, n_vec, chunk_vec, sl, P, k);
         echo_reduce_kernel<G, P, false><<<g_red, kThreads, 0, st>>>(
             codes, scales, rcodes, rscales, nullptr, n_vec, chunk_vec, sl, k.neg_zero);
