@@ -7,4 +7,4 @@ the product library.
 from .oracle import (SOURCE, CallResult, Oracle, Params, allreduce,  # noqa: F401
                      bf16_to_f32, build, compile_source, default, dequant,
                      f32_to_bf16, owner_of_columns, pack, quantize_group,
-                     unpack)
+                     reduce_scatter, unpack)

@@ -142,7 +142,8 @@ typedef struct {
 } eo_params;
 
 /*
- * One all-reduce call, evaluated on ncols group columns.
+ * One call, evaluated on ncols group columns (requantize = 1: the
+ * all-reduce; 0: the reduce-scatter).
  *
  * cols: ncols group-column ids in [0, N/G), or NULL for every column in
  * order (then ncols must be N/G).  Every per-rank array below is dense over
@@ -170,12 +171,11 @@ typedef struct {
  * be NULL) and the correction is zero.
  * Returns 0, or 1 for an invalid argument.
  */
-int eo_allreduce(const eo_params *prm, int64_t ncols, const int64_t *cols,
-                 const uint16_t *x, float *m_fast, float *m_slow,
-                 uint8_t *codes, float *scales, float *xt_out, float *e_in,
-                 float *s,
-                 uint8_t *rcodes, float *rscales, float *e_req, uint16_t *y,
-                 int32_t *qcount)
+static int call_columns(const eo_params *prm, int64_t ncols, const int64_t *cols,
+                        const uint16_t *x, float *m_fast, float *m_slow,
+                        uint8_t *codes, float *scales, float *xt_out, float *e_in,
+                        float *s, uint8_t *rcodes, float *rscales, float *e_req,
+                        uint16_t *y, int32_t *qcount, int requantize)
 {
     const int P = prm->P, G = prm->G;
     const int64_t N = prm->N;
@@ -185,7 +185,9 @@ int eo_allreduce(const eo_params *prm, int64_t ncols, const int64_t *cols,
         return EO_ERR_ARG;
     if (prm->compensate && (m_fast == NULL || m_slow == NULL))
         return EO_ERR_ARG;
-    if (!x || !codes || !scales || !rcodes || !rscales || !e_req || !y)
+    if (!x || !codes || !scales || !e_req || !y)
+        return EO_ERR_ARG;
+    if (requantize && (!rcodes || !rscales))
         return EO_ERR_ARG;
     for (int64_t t = 0; cols && t < ncols; ++t)
         if (cols[t] < 0 || cols[t] >= N / G)
@@ -272,13 +274,18 @@ int eo_allreduce(const eo_params *prm, int64_t ncols, const int64_t *cols,
             }
         }
 
-        /* 8. requantize the owner's sum, deliver it as bf16 */
-        float scale2;
-        eo_quantize_group(sum, G, k, &scale2, qcount ? cnt_req : NULL);
-        eo_pack(k, G, rcodes + base / 2);
-        rscales[t] = scale2;
+        /* 8. all-reduce: requantize the owner's sum for the all-gather and
+         * deliver it as bf16; reduce-scatter: the owner keeps its sum and
+         * receives it as bf16 directly.  er is the owner's output residual. */
+        float scale2 = 0.0f;
+        if (requantize) {
+            eo_quantize_group(sum, G, k, &scale2, qcount ? cnt_req : NULL);
+            eo_pack(k, G, rcodes + base / 2);
+            rscales[t] = scale2;
+        }
         for (int j = 0; j < G; ++j) {
-            uint16_t yb = eo_f32_to_bf16_rne(eo_dequant(k[j], scale2));
+            uint16_t yb = requantize ? eo_f32_to_bf16_rne(eo_dequant(k[j], scale2))
+                                     : eo_f32_to_bf16_rne(sum[j]);
             float er = fsub(sum[j], eo_bf16_to_f32(yb));
             y[base + j] = yb;
             e_req[base + j] = er;
@@ -298,4 +305,36 @@ int eo_allreduce(const eo_params *prm, int64_t ncols, const int64_t *cols,
     free(xt); free(sum); free(k); free(cnt_entry); free(cnt_req);
     free(max_entry_count); free(ein_local);
     return EO_OK;
+}
+
+/*
+ * One all-reduce call (see call_columns above for the arguments): every
+ * rank receives y, the requantized sum as bf16, and e_req = s - float(y)
+ * goes to the owner of each chunk.
+ */
+int eo_allreduce(const eo_params *prm, int64_t ncols, const int64_t *cols,
+                 const uint16_t *x, float *m_fast, float *m_slow,
+                 uint8_t *codes, float *scales, float *xt_out, float *e_in,
+                 float *s, uint8_t *rcodes, float *rscales, float *e_req,
+                 uint16_t *y, int32_t *qcount)
+{
+    return call_columns(prm, ncols, cols, x, m_fast, m_slow, codes, scales,
+                        xt_out, e_in, s, rcodes, rscales, e_req, y, qcount, 1);
+}
+
+/*
+ * One reduce-scatter call: steps 1-7 as for the all-reduce, then the owner
+ * of each chunk receives y = bf16(s) for its own chunk (each value is
+ * quantized once, at entry) and folds its output residual s - float(y)
+ * into its EMAs (returned in e_req).  rcodes and rscales are not used and
+ * may be NULL.  The reduce-scatter of sequence parallelism is named as a
+ * next target on the ai4snews news summary, "Perspective".
+ */
+int eo_reduce_scatter(const eo_params *prm, int64_t ncols, const int64_t *cols,
+                      const uint16_t *x, float *m_fast, float *m_slow,
+                      uint8_t *codes, float *scales, float *xt_out, float *e_in,
+                      float *s, float *e_req, uint16_t *y, int32_t *qcount)
+{
+    return call_columns(prm, ncols, cols, x, m_fast, m_slow, codes, scales,
+                        xt_out, e_in, s, NULL, NULL, e_req, y, qcount, 0);
 }

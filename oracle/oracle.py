@@ -112,6 +112,12 @@ class Oracle:
         L.eo_allreduce.argtypes = [ctypes.POINTER(_Params), ctypes.c_int64,
                                    vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                    vp, vp, vp, vp]
+        self.has_rs = hasattr(L, "eo_reduce_scatter")
+        if self.has_rs:
+            L.eo_reduce_scatter.restype = ctypes.c_int
+            L.eo_reduce_scatter.argtypes = [ctypes.POINTER(_Params), ctypes.c_int64,
+                                            vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                            vp, vp]
         self.L = L
 
     # ------------------------------------------------------------ primitives
@@ -203,6 +209,44 @@ class Oracle:
         return res
 
 
+    def reduce_scatter(self, prm: Params, x_bits: np.ndarray, m_fast, m_slow,
+                       cols=None) -> CallResult:
+        """One reduce-scatter call: y[i] (bf16 bits) is what the owner of
+        element i's chunk receives; e_req holds the owner's output residual;
+        rcodes and rscales are empty."""
+        P, G = prm.P, prm.G
+        if cols is None:
+            ncols, cptr = prm.N // G, None
+        else:
+            cols = np.ascontiguousarray(cols, dtype=np.int64)
+            ncols, cptr = cols.size, _ptr(cols)
+        n = ncols * G
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        assert x_bits.shape == (P, n), (x_bits.shape, (P, n))
+        if prm.compensate:
+            for m in (m_fast, m_slow):
+                assert m is not None and m.dtype == np.float32 and m.shape == (P, n)
+                assert m.flags.c_contiguous
+        res = CallResult(
+            codes=np.zeros((P, n // 2), np.uint8),
+            scales=np.zeros((P, ncols), np.float32),
+            xt=np.zeros((P, n), np.float32), e_in=np.zeros((P, n), np.float32),
+            s=np.zeros(n, np.float32), rcodes=np.zeros(0, np.uint8),
+            rscales=np.zeros(0, np.float32), e_req=np.zeros(n, np.float32),
+            y=np.zeros(n, np.uint16), qcount=np.zeros(n, np.int32))
+        st = prm.c_struct()
+        rc = self.L.eo_reduce_scatter(
+            ctypes.byref(st), ncols, cptr, _ptr(x_bits),
+            _ptr(m_fast) if prm.compensate else None,
+            _ptr(m_slow) if prm.compensate else None,
+            _ptr(res.codes), _ptr(res.scales), _ptr(res.xt), _ptr(res.e_in),
+            _ptr(res.s), _ptr(res.e_req), _ptr(res.y), _ptr(res.qcount))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments (P=%d N=%d G=%d)"
+                             % (P, prm.N, G))
+        return res
+
+
 def owner_of_columns(prm: Params, cols) -> np.ndarray:
     """Owner rank of each group column: floor(col*G / (N/P))."""
     return (np.asarray(cols, np.int64) * prm.G) // (prm.N // prm.P)
@@ -244,3 +288,7 @@ def unpack(b, n):
 
 def allreduce(prm, x_bits, m_fast, m_slow, cols=None):
     return default().allreduce(prm, x_bits, m_fast, m_slow, cols)
+
+
+def reduce_scatter(prm, x_bits, m_fast, m_slow, cols=None):
+    return default().reduce_scatter(prm, x_bits, m_fast, m_slow, cols)

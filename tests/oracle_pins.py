@@ -475,4 +475,72 @@ def pin_determinism(o):
         assert np.array_equal(mfa, mfb) and np.array_equal(msa, msb)
 
 
+# ---------------------------------------------------------------- reduce-scatter
+
+def _run_rs_sequence(o, prm, xs):
+    P, N = prm.P, prm.N
+    mf = np.zeros((P, N), np.float32)
+    ms = np.zeros((P, N), np.float32)
+    out = []
+    for x in xs:
+        r = o.reduce_scatter(prm, x, mf, ms)
+        out.append((r, mf.copy(), ms.copy()))
+    return out
+
+
+def pin_rs_quantized_once(o):
+    """Reduce-scatter: each value is quantized once (at entry), and what the
+    owner receives is its fp32 sum rounded to bf16 -- the all-reduce's sum
+    for the same inputs and state."""
+    rng = np.random.default_rng(22)
+    for P in (1, 2, 4, 8):
+        G = 32
+        N = P * G * 2
+        prm = _params(o, P, N, G, True)
+        x = bf16_bits(rng.normal(0, 1, (P, N)))
+        m0 = rng.normal(0, 0.05, (P, N)).astype(np.float32)
+        a = o.allreduce(prm, x, m0.copy(), m0.copy())
+        r = o.reduce_scatter(prm, x, m0.copy(), m0.copy())
+        assert (r.qcount == 1).all()
+        assert np.array_equal(r.codes, a.codes) and np.array_equal(r.scales, a.scales)
+        assert np.array_equal(r.s.view(np.uint32), a.s.view(np.uint32))
+        assert np.array_equal(r.y, bf16_bits(a.s))
+
+
+def pin_rs_telescoping(o):
+    """The telescoping identity holds for the reduce-scatter too, with y the
+    values the owners receive and their bf16 rounding error as the revealed
+    output residual."""
+    rng = np.random.default_rng(23)
+    for P, G, kw in ((4, 32, DEFAULTS), (2, 64, dict(alpha=0.75, beta_fast=0.5, beta_slow=0.9))):
+        N = P * G * 2
+        T = 16
+        prm = _params(o, P, N, G, True, **kw)
+        xs = _sequence_inputs(rng, P, N, T)
+        a = np.float64(np.float32(kw["alpha"]))
+        bf = np.float64(np.float32(kw["beta_fast"]))
+        bs = np.float64(np.float32(kw["beta_slow"]))
+        S = np.zeros(N)
+        X = np.zeros(N)
+        for t, (x, (r, mf, ms)) in enumerate(zip(xs, _run_rs_sequence(o, prm, xs)), 1):
+            S += bits_to_f64(r.y)
+            X += bits_to_f64(x).sum(axis=0)
+            rhs = -(a * mf.astype(np.float64) / (1 - bf)
+                    + (1 - a) * ms.astype(np.float64) / (1 - bs)).sum(axis=0)
+            tol = 64 * t * P * 2.0 ** -24 * (1 + np.abs(S))
+            assert (np.abs((S - X) - rhs) <= tol).all(), np.abs((S - X) - rhs).max()
+
+
+def pin_rs_grid_exact(o):
+    """Grid-exact inputs reduce-scatter exactly; the states stay 0."""
+    rng = np.random.default_rng(24)
+    for P, G in ((2, 32), (4, 64)):
+        N = P * G * 3
+        prm = _params(o, P, N, G, True)
+        xs = [bf16_bits(grid_exact_inputs(rng, P, N, G)) for _ in range(3)]
+        for x, (r, mf, ms) in zip(xs, _run_rs_sequence(o, prm, xs)):
+            assert np.array_equal(bits_to_f64(r.y), bits_to_f64(x).sum(axis=0))
+            assert not mf.any() and not ms.any()
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

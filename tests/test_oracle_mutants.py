@@ -47,10 +47,17 @@ MUTANTS = {
         "float er = fsub(sum[j], eo_bf16_to_f32(yb));",
         "float er = fsub(sum[j], eo_dequant(k[j], scale2));"),
     "sum_not_requantized": (
-        "uint16_t yb = eo_f32_to_bf16_rne(eo_dequant(k[j], scale2));",
-        "uint16_t yb = eo_f32_to_bf16_rne(sum[j]);"),
+        "uint16_t yb = requantize ? eo_f32_to_bf16_rne(eo_dequant(k[j], scale2))",
+        "uint16_t yb = requantize ? eo_f32_to_bf16_rne(sum[j])"),
     "sum_skips_last_rank": ("sum[j] = fadd(sum[j], d);",
                             "if (r < P - 1 || P == 1) sum[j] = fadd(sum[j], d);"),
+    "rs_output_requantized": (": eo_f32_to_bf16_rne(sum[j]);",
+                              ": eo_f32_to_bf16_rne(fmul(sum[j], 1.0078125f));"),
+    "rs_residual_not_folded": (
+        "/* 9. the owner alone also folds the requantization error in */\n"
+        "            if (prm->compensate) {",
+        "/* 9. the owner alone also folds the requantization error in */\n"
+        "            if (prm->compensate && requantize) {"),
 }
 
 
