@@ -73,6 +73,7 @@ def _load():
         "echo_plan_destroy": (st, [vp]),
         "echo_allreduce": (st, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, vp]),
         "echo_allreduce_host": (st, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp]),
+        "echo_reduce_scatter": (st, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, vp]),
         "echo_reset_state": (st, [vp, vp]),
         "echo_get_state": (st, [vp, vp, vp, vp]),
         "echo_set_state": (st, [vp, vp, vp, vp]),
@@ -131,6 +132,12 @@ def echo_allreduce(plan: int, in_device: Sequence[int], out_device: Sequence[int
                    stream: int = 0, side_stream: int = 0) -> None:
     _check(lib.echo_allreduce(plan, _ptr_array(in_device), _ptr_array(out_device),
                               stream or None, side_stream or None), "echo_allreduce")
+
+
+def echo_reduce_scatter(plan: int, in_device: Sequence[int], out_device: Sequence[int],
+                        stream: int = 0, side_stream: int = 0) -> None:
+    _check(lib.echo_reduce_scatter(plan, _ptr_array(in_device), _ptr_array(out_device),
+                                   stream or None, side_stream or None), "echo_reduce_scatter")
 
 
 def echo_allreduce_host(plan: int, in_host: Sequence[int], out_host: Sequence[int],

@@ -105,6 +105,29 @@ class EchoPlan:
                            _stream_handle(stream, self.device), side)
         return out
 
+    def reduce_scatter(self, xs, out=None, stream: Optional[torch.cuda.Stream] = None,
+                       side_stream: Optional[torch.cuda.Stream] = None):
+        """One reduce-scatter call.  xs: [P, N] bf16 (or P tensors); out:
+        [P, N/P] bf16 (allocated if None), row r = rank r's own chunk of the
+        sum.  Returns out."""
+        xs_l = self._rank_tensors(xs, "inputs")
+        C = self.N // self.P
+        if out is None:
+            out = torch.empty((self.P, C), dtype=torch.bfloat16, device=self.device)
+        out_l = list(out.unbind(0)) if isinstance(out, torch.Tensor) else list(out)
+        if len(out_l) != self.P or any(t.dtype != torch.bfloat16 or t.numel() != C
+                                       or not t.is_contiguous() or t.device != self.device
+                                       for t in out_l):
+            raise ValueError("outputs: P contiguous bf16 tensors of N/P elements on the device")
+        for t in xs_l:
+            if t.device != self.device:
+                raise ValueError("tensors must live on %s" % self.device)
+        side = int(side_stream.cuda_stream) if side_stream is not None else 0
+        abi.echo_reduce_scatter(self.handle, [t.data_ptr() for t in xs_l],
+                                [t.data_ptr() for t in out_l],
+                                _stream_handle(stream, self.device), side)
+        return out
+
     def allreduce_host(self, xs_host, out_host=None, stream: Optional[torch.cuda.Stream] = None):
         """The same call on host tensors (pinned for asynchronous copies);
         the caller synchronizes the stream before reading out_host."""

@@ -225,6 +225,45 @@ void launch_fixup(echo_plan *p, const float *sf, const float *ss, float *df, flo
 
 Slab whole(const echo_plan *p) { return Slab{0, p->chunk_vec}; }
 
+template <int G, int P>
+void launch_rs_t(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+    dim3 grid(reduce_blocks(sl.v_count), (unsigned)P);
+    if (!p->cfg.compensate)
+        echo_rs_kernel<G, P, false, false><<<grid, kThreads, 0, st>>>(
+            p->codes, p->scales, out, p->m_fast, p->m_slow, p->e_req, p->n_vec, p->chunk_vec, sl,
+            p->k);
+    else if (fix)
+        echo_rs_kernel<G, P, true, true><<<grid, kThreads, 0, st>>>(
+            p->codes, p->scales, out, p->m_fast, p->m_slow, p->e_req, p->n_vec, p->chunk_vec, sl,
+            p->k);
+    else
+        echo_rs_kernel<G, P, true, false><<<grid, kThreads, 0, st>>>(
+            p->codes, p->scales, out, p->m_fast, p->m_slow, p->e_req, p->n_vec, p->chunk_vec, sl,
+            p->k);
+}
+
+template <int G>
+void launch_rs_g(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+    switch (p->cfg.P) {
+        case 1: launch_rs_t<G, 1>(p, out, sl, st, fix); break;
+        case 2: launch_rs_t<G, 2>(p, out, sl, st, fix); break;
+        case 3: launch_rs_t<G, 3>(p, out, sl, st, fix); break;
+        case 4: launch_rs_t<G, 4>(p, out, sl, st, fix); break;
+        case 5: launch_rs_t<G, 5>(p, out, sl, st, fix); break;
+        case 6: launch_rs_t<G, 6>(p, out, sl, st, fix); break;
+        case 7: launch_rs_t<G, 7>(p, out, sl, st, fix); break;
+        default: launch_rs_t<G, 8>(p, out, sl, st, fix); break;
+    }
+}
+
+void launch_rs(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+    switch (p->cfg.G) {
+        case 32: launch_rs_g<32>(p, out, sl, st, fix); break;
+        case 64: launch_rs_g<64>(p, out, sl, st, fix); break;
+        default: launch_rs_g<128>(p, out, sl, st, fix); break;
+    }
+}
+
 bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 
 // Wait (on st) for a side-stream fix-up that may still be writing the state.
@@ -405,6 +444,76 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
             p->side_inflight = true;
         } else {
             p->side_inflight = false;
+        }
+    }
+    if (comp && mode == ECHO_FIXUP_DEFERRED) p->pending = true;
+    if (p->profiling) p->records.push_back(rec);
+    return ECHO_OK;
+}
+
+echo_status echo_reduce_scatter(echo_plan *p, const void *const *in, void *const *out,
+                                void *stream, void *side_stream) {
+    if (!p || !in || !out) return ECHO_ERR_INVALID_ARG;
+    const int P = p->cfg.P;
+    const size_t out_bytes = (size_t)p->cfg.N / P * 2;
+    InPtrs xi{};
+    OutPtrs yo{};
+    for (int r = 0; r < P; ++r) {
+        if (!in[r] || !out[r]) return ECHO_ERR_INVALID_ARG;
+        if (!aligned16(in[r]) || !aligned16(out[r])) return ECHO_ERR_ALIGNMENT;
+        xi.p[r] = (const uint4 *)in[r];
+        yo.p[r] = (uint4 *)out[r];
+    }
+    for (int r = 0; r < P; ++r)
+        for (int s2 = r + 1; s2 < P; ++s2) {
+            const char *a = (const char *)out[r], *b = (const char *)out[s2];
+            if (a < b + out_bytes && b < a + out_bytes) return ECHO_ERR_INVALID_ARG;
+        }
+    DeviceGuard guard(p->cfg.device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaStream_t side = (cudaStream_t)side_stream;
+    const bool comp = p->cfg.compensate != 0;
+    const int mode = p->cfg.fixup;
+
+    ProfRecord rec{};
+    if (p->profiling) {
+        for (int i = 0; i < 4; ++i) {
+            rec.ev[i] = take_event(p);
+            if (!rec.ev[i]) return ECHO_ERR_CUDA;
+        }
+    }
+    ECHO_TRY(order_after_side(p, st));
+    const bool defer = comp && mode == ECHO_FIXUP_DEFERRED && p->pending;
+    if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[0], st));
+    launch_entry(p, xi, whole(p), st, defer);
+    ECHO_TRY(cudaGetLastError());
+    if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[1], st));
+    launch_rs(p, yo, whole(p), st, comp && mode == ECHO_FIXUP_EXIT);
+    ECHO_TRY(cudaGetLastError());
+    if (p->profiling) {
+        ECHO_TRY(cudaEventRecord(rec.ev[2], st));
+        ECHO_TRY(cudaEventRecord(rec.ev[3], st));
+    }
+    if (comp && mode == ECHO_FIXUP_SIDE) {
+        cudaStream_t fs = side ? side : st;
+        if (side) {
+            ECHO_TRY(cudaEventRecord(p->ev_reduced, st));
+            ECHO_TRY(cudaStreamWaitEvent(side, p->ev_reduced, 0));
+        }
+        if (p->profiling) {
+            rec.ev[4] = take_event(p);
+            rec.ev[5] = take_event(p);
+            if (!rec.ev[4] || !rec.ev[5]) return ECHO_ERR_CUDA;
+            rec.side = true;
+            ECHO_TRY(cudaEventRecord(rec.ev[4], fs));
+        }
+        launch_fixup(p, p->m_fast, p->m_slow, p->m_fast, p->m_slow, true, true, whole(p), fs);
+        ECHO_TRY(cudaGetLastError());
+        if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[5], fs));
+        if (side) {
+            ECHO_TRY(cudaEventRecord(p->ev_side_done, side));
+            p->side_inflight = true;
         }
     }
     if (comp && mode == ECHO_FIXUP_DEFERRED) p->pending = true;

@@ -22,22 +22,18 @@ inline unsigned reduce_blocks(int64_t v_count) {
     return (unsigned)((v_count / 2 + kThreads - 1) / kThreads);
 }
 
-template <int G, int P, bool COMP>
-__global__ void __launch_bounds__(kThreads)
-echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
-                   uint32_t *__restrict__ rcodes, float *__restrict__ rscales,
-                   float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec, Slab sl,
-                   float neg_zero) {
-    constexpr int LANES = G / kRedVec;              // lanes per group
-    const int o = blockIdx.y;
-    const int64_t n_run = n_vec / 2;                // 16-element runs per rank
-    const int64_t chunk_run = chunk_vec / 2;        // runs per owner chunk
-    const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    const bool valid = local < sl.v_count / 2;
-    const int64_t j = (int64_t)o * chunk_run + sl.v_begin / 2 + local;  // run index in a rank
+// The reduce-scatter sum of one 16-element run j (run index within a rank)
+// of the P ranks: dequantize each rank's codes and add them in fp32 in
+// ascending rank order from +0.  All P code and scale loads are issued
+// before any arithmetic.  Lanes with valid == false produce zeros.
+template <int G, int P>
+__device__ __forceinline__ void sum_run(const uint32_t *__restrict__ codes,
+                                        const float *__restrict__ scales, int64_t n_vec,
+                                        int64_t j, bool valid, float2 z, float s[16]) {
+    constexpr int LANES = G / kRedVec;
+    const int64_t n_run = n_vec / 2;
     const int64_t n_groups = n_run / LANES;
     const uint2 *codes2 = reinterpret_cast<const uint2 *>(codes);
-
     uint2 w[P];
     float sc[P];
 #pragma unroll
@@ -45,7 +41,6 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
         w[r] = valid ? __ldcs(codes2 + (int64_t)r * n_run + j) : make_uint2(0u, 0u);
         sc[r] = valid ? __ldg(scales + (int64_t)r * n_groups + j / LANES) : 0.0f;
     }
-    const float2 z = splat2(neg_zero);
     float2 s2[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) s2[i] = make_float2(0.0f, 0.0f);
@@ -60,12 +55,28 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
             s2[4 + p] = add2(s2[4 + p], prod2(code_pair(ly, hy, p), sc2, z));
         }
     }
-    float s[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         s[2 * i] = s2[i].x;
         s[2 * i + 1] = s2[i].y;
     }
+}
+
+template <int G, int P, bool COMP>
+__global__ void __launch_bounds__(kThreads)
+echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
+                   uint32_t *__restrict__ rcodes, float *__restrict__ rscales,
+                   float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec, Slab sl,
+                   float neg_zero) {
+    constexpr int LANES = G / kRedVec;              // lanes per group
+    const int o = blockIdx.y;
+    const int64_t chunk_run = chunk_vec / 2;        // runs per owner chunk
+    const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    const bool valid = local < sl.v_count / 2;
+    const int64_t j = (int64_t)o * chunk_run + sl.v_begin / 2 + local;  // run index in a rank
+    const float2 z = splat2(neg_zero);
+    float s[16];
+    sum_run<G, P>(codes, scales, n_vec, j, valid, z, s);
 
     float a = 0.0f;
 #pragma unroll
@@ -92,6 +103,69 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
         }
         st8(e_req + j * kRedVec, e);
         st8(e_req + j * kRedVec + 8, e + 8);
+    }
+}
+
+// ------------------------------------------------------------ echo_reduce_scatter
+//
+// The reduce-scatter call's second kernel: the same sum, delivered to the
+// owner as bf16 without a second quantization: out[o] (N/P elements) gets
+// bf16(s) of chunk o.  The owner's output residual e = s - float(bf16(s))
+// is folded into its own EMAs here (FIX) or written to e_req for a
+// side-stream or deferred fix-up (COMP && !FIX).
+// Grid: x over the 16-element runs of the slab, y = owner.
+template <int G, int P, bool COMP, bool FIX>
+__global__ void __launch_bounds__(kThreads)
+echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales, OutPtrs out,
+               float *__restrict__ m_fast, float *__restrict__ m_slow, float *__restrict__ e_req,
+               int64_t n_vec, int64_t chunk_vec, Slab sl, Consts k) {
+    const int o = blockIdx.y;
+    const int64_t chunk_run = chunk_vec / 2;
+    const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (local >= sl.v_count / 2) return;    // no shuffles below: lanes may leave
+    const int64_t lr = sl.v_begin / 2 + local;          // run index within chunk o
+    const int64_t j = (int64_t)o * chunk_run + lr;       // run index within a rank
+    const float2 z = splat2(k.neg_zero);
+    float s[16];
+    sum_run<G, P>(codes, scales, n_vec, j, true, z, s);
+
+    uint32_t yw[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) yw[i] = bf16x2_bits_rn(make_float2(s[2 * i], s[2 * i + 1]));
+    uint4 *dst = out.p[o] + lr * 2;
+    dst[0] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+    dst[1] = make_uint4(yw[4], yw[5], yw[6], yw[7]);
+    if (COMP) {
+        float e[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 d = sub2(make_float2(s[2 * i], s[2 * i + 1]), bf16x2_to_f32(yw[i]));
+            e[2 * i] = d.x;
+            e[2 * i + 1] = d.y;
+        }
+        if (FIX) {
+            const int64_t e0 = ((int64_t)o * n_vec + j * 2) * kVec;   // rank o's own state
+            const float2 obf = splat2(k.one_m_beta_fast), obs = splat2(k.one_m_beta_slow);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float mf[8], ms[8];
+                ld8(m_fast + e0 + 8 * h, mf);
+                ld8(m_slow + e0 + 8 * h, ms);
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) {
+                    const float2 e2 = make_float2(e[8 * h + i], e[8 * h + i + 1]);
+                    const float2 f = add2(make_float2(mf[i], mf[i + 1]), prod2(obf, e2, z));
+                    const float2 g = add2(make_float2(ms[i], ms[i + 1]), prod2(obs, e2, z));
+                    mf[i] = f.x; mf[i + 1] = f.y;
+                    ms[i] = g.x; ms[i + 1] = g.y;
+                }
+                st8(m_fast + e0 + 8 * h, mf);
+                st8(m_slow + e0 + 8 * h, ms);
+            }
+        } else {
+            st8(e_req + j * kRedVec, e);
+            st8(e_req + j * kRedVec + 8, e + 8);
+        }
     }
 }
 

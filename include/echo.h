@@ -139,6 +139,24 @@ echo_status echo_allreduce(echo_plan *plan, const void *const *in_device,
                            void *const *out_device, void *stream,
                            void *side_stream);
 
+/* One reduce-scatter over the P ranks: the reduce-scatter of sequence
+ * parallelism, which the pages name as a next target for the same scheme
+ * (ai4snews news summary, "Perspective").  Steps 1-4 as for
+ * echo_allreduce, then the owner o of chunk [o*N/P, (o+1)*N/P) receives
+ * bf16(s) of that chunk: each value is quantized once, at entry.  The
+ * owner's output residual s - float(bf16(s)) is folded into its own EMAs
+ * like e_req (in the second kernel, on side_stream, or deferred into the
+ * next call's entry pass, by the plan's fix-up mode).
+ *   in_device[r]  : bf16, N elements of rank r (read)
+ *   out_device[r] : bf16, N/P elements: rank r's own chunk of the sum
+ *                   (written); must not overlap each other
+ * A plan's state is shared between its all-reduce and reduce-scatter
+ * calls.  Two kernels per call (three in side-stream mode).
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+echo_status echo_reduce_scatter(echo_plan *plan, const void *const *in_device,
+                                void *const *out_device, void *stream,
+                                void *side_stream);
+
 /* The same call on host buffers, pipelined: the call is cut into up to 16
  * slabs (the same sub-range of every owner chunk); each slab's inputs are
  * copied host -> device, its three kernels run, and its outputs are copied

@@ -121,3 +121,33 @@ def oracle_params(plan: EchoPlan) -> oracle.Params:
     c = plan.cfg
     return oracle.Params(P=c.P, N=c.N, G=c.G, compensate=bool(c.compensate), alpha=c.alpha,
                          beta_fast=c.beta_fast, beta_slow=c.beta_slow)
+
+
+class RSChecker(SequenceChecker):
+    """The same comparison for reduce-scatter calls (and, through
+    step_allreduce, all-reduce calls on the same plan and state)."""
+
+    def step_rs(self, x: torch.Tensor, side_stream=None):
+        plan, prm = self.plan, self.prm
+        out = plan.reduce_scatter(x, side_stream=side_stream)
+        torch.cuda.synchronize()
+        call = self.calls
+        self.calls += 1
+        xb = _bits_u16(self.gather(x, "e"))
+        ref = oracle.reduce_scatter(prm, xb, self.mf, self.ms, self.cols)
+        dv = plan.debug_view()
+        assert_same("entry codes", _u8(self.gather(dv["codes"], "c")), ref.codes, "u8", call)
+        assert_same("entry scales", _f32(self.gather(dv["scales"], "g")), ref.scales, "f32", call)
+        C = prm.N // prm.P
+        owner = torch.from_numpy(self.idx // C).to(plan.device)
+        local = torch.from_numpy(self.idx % C).to(plan.device)
+        got = out[owner, local]
+        assert_same("owner outputs", _bits_u16(got), ref.y, "bf16", call)
+        if prm.compensate:
+            if plan.fixup != "exit":
+                assert_same("output residual", _f32(self.gather(dv["e_req"], "e")), ref.e_req,
+                            "f32", call)
+            mf, ms = plan.get_state()
+            assert_same("m_fast", _f32(self.gather(mf, "e")), self.mf, "f32", call)
+            assert_same("m_slow", _f32(self.gather(ms, "e")), self.ms, "f32", call)
+        return out, ref
