@@ -75,6 +75,16 @@ def call_min_bytes(P: int, N: int, G: int, comp: bool) -> float:
     return P * N * (2 + 2 + 2 * q) + N * 2 * q
 
 
+def rs_min_bytes(P: int, N: int, G: int, comp: bool) -> float:
+    """Minimal HBM bytes of one reduce-scatter call: read x, (read+write both
+    states), write and read the entry transport, write each owner's bf16
+    chunk, (write e_req and read it once in the next entry)."""
+    q = transport_bytes_per_elem(G)
+    if comp:
+        return P * N * (2 + 16 + 2 * q) + N * (2 + 8)
+    return P * N * (2 + 2 * q) + N * 2
+
+
 def entry_bytes(P: int, N: int, G: int, comp: bool, fixup: str) -> float:
     """Algorithmic bytes of one echo_entry launch: read x (2 B), read and
     write both states (16 B), write codes + scales (q B) per rank-element;
@@ -282,9 +292,18 @@ def run_step_mode(args, ws, rank, local):
     plan = EchoPlan(P, N, G, compensate=comp, fixup=fixup, device=local)
     side = torch.cuda.Stream(device=dev) if fixup == "side" else None
     stream = torch.cuda.current_stream(dev)
+    rs = args.op == "reduce-scatter"
+    if rs:
+        out = torch.empty((P, N // P), dtype=torch.bfloat16, device=dev)
+
+    def one_call():
+        if rs:
+            plan.reduce_scatter(x, out=out, side_stream=side)
+        else:
+            plan.allreduce(x, out=out, side_stream=side)
 
     for _ in range(args.warmup):
-        plan.allreduce(x, out=out, side_stream=side)
+        one_call()
     torch.cuda.synchronize(dev)
 
     clocks = ClockSampler(local)
@@ -299,7 +318,7 @@ def run_step_mode(args, ws, rank, local):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(args.steps):
-        plan.allreduce(x, out=out, side_stream=side)
+        one_call()
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(ws)
@@ -313,7 +332,7 @@ def run_step_mode(args, ws, rank, local):
 
     # end to end: host buffers through echo_allreduce_host
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not rs:
         xh = torch.empty((P, N), dtype=torch.bfloat16, pin_memory=True)
         xh.copy_(x)
         yh = torch.empty((P, N), dtype=torch.bfloat16, pin_memory=True)
@@ -349,15 +368,18 @@ def run_step_mode(args, ws, rank, local):
         entry_ms = prof["entry_ms"] / max(calls, 1)
         eb = entry_bytes(P, N, G, comp, fixup)
         achieved = eb / (entry_ms / 1e3) / 1e9
-        bmin = call_min_bytes(P, N, G, comp)
+        bmin = rs_min_bytes(P, N, G, comp) if rs else call_min_bytes(P, N, G, comp)
         traffic = ncu_traffic(w.name, comp, fixup)
+        metric = METRIC if comp else METRIC.replace("compensated", "uncompensated")
+        if rs:
+            metric = metric.replace("reduce input", "reduce-scatter input")
         line = {
-            "metric": METRIC if comp else METRIC.replace("compensated", "uncompensated"),
+            "metric": metric,
             "value": round(value, 3), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, int4 transport, f32 sum+state",
             "data": "synthetic (seeded N(0,0.5^2) bf16 draws, no dataset)",
-            "config": {"workload": w.name, "P": P, "N_per_rank": N, "G": G,
+            "config": {"workload": w.name, "op": args.op, "P": P, "N_per_rank": N, "G": G,
                        "compensate": comp, "fixup": fixup, "alpha": 0.5, "beta_fast": 0.5,
                        "beta_slow": 0.95, "l2": "inputs larger than L2 (%.1f GiB of x per step)"
                        % (2 * P * N / 2**30), "parallelism": "replicas" if ws > 1 else "1 GPU"},
@@ -577,6 +599,7 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="large")
     ap.add_argument("--fixup", choices=("exit", "side", "deferred"), default=BENCH_FIXUP)
     ap.add_argument("--uncompensated", action="store_true")
+    ap.add_argument("--op", choices=("all-reduce", "reduce-scatter"), default="all-reduce")
     ap.add_argument("--mode", choices=("step", "depth-chain", "sweep", "overlap"), default="step")
     ap.add_argument("--sweep-max-mib", type=int, default=0,
                     help="sweep only points up to this many MiB per rank (0: all)")

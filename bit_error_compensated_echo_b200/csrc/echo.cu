@@ -86,6 +86,7 @@ struct DeviceGuard {
 struct ProfRecord {
     cudaEvent_t ev[6];   // entry start, entry end, reduce end, exit end, fixup start, fixup end
     bool side;
+    int kernels;         // kernels on the main stream (3 all-reduce, 2 reduce-scatter)
 };
 
 }  // namespace
@@ -400,6 +401,7 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
     const int mode = p->cfg.fixup;
 
     ProfRecord rec{};
+    rec.kernels = 3;
     if (p->profiling) {
         for (int i = 0; i < 6; ++i) rec.ev[i] = nullptr;
         for (int i = 0; i < 4; ++i) {
@@ -477,6 +479,7 @@ echo_status echo_reduce_scatter(echo_plan *p, const void *const *in, void *const
     const int mode = p->cfg.fixup;
 
     ProfRecord rec{};
+    rec.kernels = 2;
     if (p->profiling) {
         for (int i = 0; i < 4; ++i) {
             rec.ev[i] = take_event(p);
@@ -671,7 +674,7 @@ echo_status echo_profile_read(echo_plan *p, echo_profile *out, int32_t reset) {
         p->totals.reduce_ms += ms;
         ECHO_TRY(cudaEventElapsedTime(&ms, r.ev[2], r.ev[3]));
         p->totals.exit_ms += ms;
-        p->totals.launches += 3;
+        p->totals.launches += r.kernels;
         if (r.side) {
             ECHO_TRY(cudaEventSynchronize(r.ev[5]));
             ECHO_TRY(cudaEventElapsedTime(&ms, r.ev[4], r.ev[5]));

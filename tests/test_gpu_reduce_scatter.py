@@ -62,3 +62,13 @@ def test_rs_llama_shape_sampled():
         chk = RSChecker(plan, oracle_params(plan), W.column_sample(w, 512))
         for t in range(8):
             chk.step_rs(W.generate(w, t, DEV))
+
+
+def test_rs_profile_counts_two_launches():
+    w = W.with_size(W.TINY, P=2, rows=1, hidden=2 * 32 * 64, G=32)
+    with _plan(w.P, w.N, w.G, True, "deferred") as plan:
+        plan.profile_enable(True)
+        for t in range(3):
+            plan.reduce_scatter(W.generate(w, t, DEV))
+        p = plan.profile_read(reset=True)
+        assert p["calls"] == 3 and p["launches"] == 6
