@@ -76,34 +76,43 @@ uint16_t eo_f32_to_bf16_rne(float f)
 }
 
 /*
- * Quantize one group of G fp32 values to symmetric 4-bit codes.
- *   a = max |v|;  scale = a / 7;  k = clamp(rint(v / scale), -7, 7).
+ * Quantize one group of G fp32 values to symmetric codes with L levels on
+ * each side (L = 7 for 4-bit codes, 127 for 8-bit codes).
+ *   a = max |v|;  scale = a / L;  k = clamp(rint(v / scale), -L, L).
  * A group with a == 0 (or whose scale underflows to 0) gets scale 0 and all
  * codes 0.  rintf rounds half to even in the default rounding mode.
  * If count is not NULL, count[j] is incremented for every element j that is
  * quantized (the instrumented oracle counts quantizer applications).
  */
-void eo_quantize_group(const float *v, int G, int8_t *k, float *scale_out,
-                       int32_t *count)
+void eo_quantize_group_levels(const float *v, int G, int L, int8_t *k,
+                              float *scale_out, int32_t *count)
 {
+    const float levels = (float)L;
     float a = 0.0f;
     for (int j = 0; j < G; ++j)
         a = fmaxf(a, fabsf(v[j]));
     float scale = 0.0f;
     if (a != 0.0f)
-        scale = fdiv(a, 7.0f);
+        scale = fdiv(a, levels);
     for (int j = 0; j < G; ++j) {
         int code = 0;
         if (scale != 0.0f) {
             float r = rintf(fdiv(v[j], scale));
-            if (r > 7.0f) r = 7.0f;
-            if (r < -7.0f) r = -7.0f;
+            if (r > levels) r = levels;
+            if (r < -levels) r = -levels;
             code = (int)r;
         }
         k[j] = (int8_t)code;
         if (count) count[j] += 1;
     }
     *scale_out = scale;
+}
+
+/* The 4-bit quantizer: L = 7. */
+void eo_quantize_group(const float *v, int G, int8_t *k, float *scale_out,
+                       int32_t *count)
+{
+    eo_quantize_group_levels(v, G, 7, k, scale_out, count);
 }
 
 /* Dequantize one code: k * scale in fp32. */
@@ -118,6 +127,13 @@ void eo_pack(const int8_t *k, int64_t n, uint8_t *bytes)
         uint8_t hi = (uint8_t)(k[2 * j + 1] & 0x0f);
         bytes[j] = (uint8_t)(lo | (hi << 4));
     }
+}
+
+/* 8-bit codes: one per byte, two's complement. */
+void eo_pack8(const int8_t *k, int64_t n, uint8_t *bytes)
+{
+    for (int64_t j = 0; j < n; ++j)
+        bytes[j] = (uint8_t)k[j];
 }
 
 /* Inverse of eo_pack: sign-extend each nibble. */
@@ -139,6 +155,7 @@ typedef struct {
     float alpha;        /* weight of the fast EMA in the correction */
     float beta_fast;    /* decay of the fast EMA */
     float beta_slow;    /* decay of the slow EMA */
+    int32_t bits;       /* 4: int4 codes, two per byte; 8: int8 codes */
 } eo_params;
 
 /*
@@ -153,12 +170,12 @@ typedef struct {
  *   x       [P][ncols*G]   bf16 bits, input of each rank (read)
  *   m_fast  [P][ncols*G]   fast EMA state (read, updated in place)
  *   m_slow  [P][ncols*G]   slow EMA state (read, updated in place)
- *   codes   [P][ncols*G/2] entry codes, packed (written)
+ *   codes   [P][ncols*G*bits/8] entry codes, packed (written)
  *   scales  [P][ncols]     entry scales (written)
  *   xt      [P][ncols*G]   corrected input x + c (written, may be NULL)
  *   e_in    [P][ncols*G]   entry quantization error (written, may be NULL)
  *   s       [ncols*G]      fp32 sum of the dequantized entries (may be NULL)
- *   rcodes  [ncols*G/2]    requantized sum, packed (written)
+ *   rcodes  [ncols*G*bits/8] requantized sum, packed (written)
  *   rscales [ncols]        requantization scales (written)
  *   e_req   [ncols*G]      requantization error s - float(y) (written)
  *   y       [ncols*G]      bf16 bits of the result every rank receives
@@ -181,6 +198,9 @@ static int call_columns(const eo_params *prm, int64_t ncols, const int64_t *cols
     const int64_t N = prm->N;
     if (P < 1 || G < 2 || (G & 1) || N <= 0 || N % ((int64_t)P * G) != 0)
         return EO_ERR_ARG;
+    if (prm->bits != 4 && prm->bits != 8)
+        return EO_ERR_ARG;
+    const int L = prm->bits == 8 ? 127 : 7;   /* levels on each side */
     if (cols == NULL && ncols != N / G)
         return EO_ERR_ARG;
     if (prm->compensate && (m_fast == NULL || m_slow == NULL))
@@ -247,8 +267,11 @@ static int call_columns(const eo_params *prm, int64_t ncols, const int64_t *cols
             float scale;
             if (qcount)
                 memset(cnt_entry, 0, sizeof(int32_t) * (size_t)G);
-            eo_quantize_group(xt, G, k, &scale, qcount ? cnt_entry : NULL);
-            eo_pack(k, G, codes + ((int64_t)r * n + base) / 2);
+            eo_quantize_group_levels(xt, G, L, k, &scale, qcount ? cnt_entry : NULL);
+            if (prm->bits == 8)
+                eo_pack8(k, G, codes + (int64_t)r * n + base);
+            else
+                eo_pack(k, G, codes + ((int64_t)r * n + base) / 2);
             scales[(int64_t)r * ncols + t] = scale;
             for (int j = 0; j < G; ++j) {
                 float d = eo_dequant(k[j], scale);
@@ -279,8 +302,11 @@ static int call_columns(const eo_params *prm, int64_t ncols, const int64_t *cols
          * receives it as bf16 directly.  er is the owner's output residual. */
         float scale2 = 0.0f;
         if (requantize) {
-            eo_quantize_group(sum, G, k, &scale2, qcount ? cnt_req : NULL);
-            eo_pack(k, G, rcodes + base / 2);
+            eo_quantize_group_levels(sum, G, L, k, &scale2, qcount ? cnt_req : NULL);
+            if (prm->bits == 8)
+                eo_pack8(k, G, rcodes + base);
+            else
+                eo_pack(k, G, rcodes + base / 2);
             rscales[t] = scale2;
         }
         for (int j = 0; j < G; ++j) {

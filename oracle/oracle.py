@@ -52,7 +52,7 @@ class _Params(ctypes.Structure):
     _fields_ = [("P", ctypes.c_int32), ("G", ctypes.c_int32),
                 ("N", ctypes.c_int64), ("compensate", ctypes.c_int32),
                 ("alpha", ctypes.c_float), ("beta_fast", ctypes.c_float),
-                ("beta_slow", ctypes.c_float)]
+                ("beta_slow", ctypes.c_float), ("bits", ctypes.c_int32)]
 
 
 @dataclass
@@ -65,10 +65,11 @@ class Params:
     alpha: float = 0.5
     beta_fast: float = 0.5
     beta_slow: float = 0.95
+    bits: int = 4
 
     def c_struct(self) -> _Params:
         return _Params(self.P, self.G, self.N, int(bool(self.compensate)),
-                       self.alpha, self.beta_fast, self.beta_slow)
+                       self.alpha, self.beta_fast, self.beta_slow, self.bits)
 
 
 @dataclass
@@ -102,6 +103,9 @@ class Oracle:
         L.eo_f32_to_bf16_rne.argtypes = [ctypes.c_float]
         L.eo_quantize_group.restype = None
         L.eo_quantize_group.argtypes = [vp, ctypes.c_int, vp, vp, vp]
+        if hasattr(L, "eo_quantize_group_levels"):
+            L.eo_quantize_group_levels.restype = None
+            L.eo_quantize_group_levels.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp, vp]
         L.eo_dequant.restype = ctypes.c_float
         L.eo_dequant.argtypes = [ctypes.c_int8, ctypes.c_float]
         L.eo_pack.restype = None
@@ -147,6 +151,14 @@ class Oracle:
         self.L.eo_quantize_group(_ptr(v), v.size, _ptr(k), _ptr(sc), _ptr(count))
         return k, np.float32(sc[0])
 
+    def quantize_group_levels(self, v, levels: int, count=None):
+        """Symmetric absmax quantization with `levels` levels per side."""
+        v = np.ascontiguousarray(v, dtype=np.float32)
+        k = np.zeros(v.size, dtype=np.int8)
+        sc = np.zeros(1, dtype=np.float32)
+        self.L.eo_quantize_group_levels(_ptr(v), v.size, levels, _ptr(k), _ptr(sc), _ptr(count))
+        return k, np.float32(sc[0])
+
     def dequant(self, k, scale) -> np.ndarray:
         k = np.asarray(k, dtype=np.int8).ravel()
         return np.array([self.L.eo_dequant(int(c), float(scale)) for c in k],
@@ -188,11 +200,12 @@ class Oracle:
             for m in (m_fast, m_slow):
                 assert m is not None and m.dtype == np.float32 and m.shape == (P, n)
                 assert m.flags.c_contiguous
+        cb = n * prm.bits // 8
         res = CallResult(
-            codes=np.zeros((P, n // 2), np.uint8),
+            codes=np.zeros((P, cb), np.uint8),
             scales=np.zeros((P, ncols), np.float32),
             xt=np.zeros((P, n), np.float32), e_in=np.zeros((P, n), np.float32),
-            s=np.zeros(n, np.float32), rcodes=np.zeros(n // 2, np.uint8),
+            s=np.zeros(n, np.float32), rcodes=np.zeros(cb, np.uint8),
             rscales=np.zeros(ncols, np.float32), e_req=np.zeros(n, np.float32),
             y=np.zeros(n, np.uint16), qcount=np.zeros(n, np.int32))
         st = prm.c_struct()
@@ -228,7 +241,7 @@ class Oracle:
                 assert m is not None and m.dtype == np.float32 and m.shape == (P, n)
                 assert m.flags.c_contiguous
         res = CallResult(
-            codes=np.zeros((P, n // 2), np.uint8),
+            codes=np.zeros((P, n * prm.bits // 8), np.uint8),
             scales=np.zeros((P, ncols), np.float32),
             xt=np.zeros((P, n), np.float32), e_in=np.zeros((P, n), np.float32),
             s=np.zeros(n, np.float32), rcodes=np.zeros(0, np.uint8),

@@ -222,9 +222,9 @@ def pin_golden_call(o):
 
 # ---------------------------------------------------------------- invariants
 
-def grid_exact_inputs(rng, P, N, G):
-    """Inputs on the int4 grid whose sums stay on it (values k*2^e with
-    every rank's group max |k| = 7 and |sum_r k_r| <= 7, reaching 7)."""
+def grid_exact_inputs(rng, P, N, G, L=7):
+    """Inputs on the code grid whose sums stay on it (values k*2^e with
+    every rank's group max |k| = L and |sum_r k_r| <= L, reaching L)."""
     assert G >= P
     x = np.zeros((P, N), np.float64)
     for c in range(N // G):
@@ -233,7 +233,7 @@ def grid_exact_inputs(rng, P, N, G):
         special = pos[:P]
         k = np.zeros((P, G), np.int64)
         for j in pos[P:]:
-            budget = 7
+            budget = L
             for r in rng.permutation(P):
                 if budget == 0:
                     break
@@ -241,7 +241,7 @@ def grid_exact_inputs(rng, P, N, G):
                 k[r, j] = v
                 budget -= abs(v)
         for r in range(P):
-            k[r, special[r]] = 7 * int(rng.choice([-1, 1])) if r else 7
+            k[r, special[r]] = L * int(rng.choice([-1, 1])) if r else L
         x[:, c * G:(c + 1) * G] = k * 2.0 ** e
     return x.astype(np.float32)
 
@@ -473,6 +473,98 @@ def pin_determinism(o):
     for (ra, mfa, msa), (rb, mfb, msb) in zip(a, b):
         assert np.array_equal(ra.y, rb.y) and np.array_equal(ra.codes, rb.codes)
         assert np.array_equal(mfa, mfb) and np.array_equal(msa, msb)
+
+
+# ---------------------------------------------------------------- 8-bit codes
+
+def pin_quantize8_bruteforce(o):
+    """8-bit codes: each code minimises |v - k*scale| over k in -127..127
+    (exact arithmetic), exact midpoints go to the even code, the scale is the
+    fp32 nearest to a/127, and the largest magnitude maps to +-127."""
+    rng = np.random.default_rng(25)
+    for trial in range(24):
+        G = int(rng.choice([2, 4, 8]))
+        kind = trial % 3
+        if kind == 0:
+            v = rng.normal(0, 1, G)
+        elif kind == 1:
+            e = int(rng.integers(-4, 4))
+            v = (rng.integers(-127, 127, G) + 0.5) * 2.0 ** e
+            v[rng.integers(0, G)] = 127.0 * 2.0 ** e
+        else:
+            v = rng.standard_t(3, G) * 100
+        v = np.asarray(v, np.float32)
+        k, scale = o.quantize_group_levels(v, 127)
+        a = np.float32(np.max(np.abs(v)))
+        _nearest_f32_check(Fraction(float(a)) / 127, scale)
+        fs = Fraction(float(scale))
+        for vj, kj in zip(v, k):
+            errs = [(abs(Fraction(float(vj)) - c * fs), c) for c in range(-127, 128)]
+            m = min(e for e, _ in errs)
+            cands = [c for e, c in errs if e == m]
+            q = Fraction(float(vj)) / fs
+            near = abs(q - (q.__floor__() + Fraction(1, 2))) <= Fraction(1, 2**12)
+            if len(cands) == 2:
+                assert int(kj) == [c for c in cands if c % 2 == 0][0], (vj, kj, cands)
+            elif not near:
+                assert int(kj) == cands[0], (vj, kj, cands)
+        assert abs(int(k[int(np.argmax(np.abs(v)))])) == 127
+
+
+def pin_golden_quantize8(o):
+    """Hand-worked 8-bit groups (tests/golden/quantize8_worked.txt)."""
+    for row in _read_golden("quantize8_worked.txt"):
+        vals, codes, scale, packed = [p.strip() for p in row.split("|")]
+        v = np.array([float(t) for t in vals.split()], np.float32)
+        k, sc = o.quantize_group_levels(v, 127)
+        assert k.tolist() == [int(t) for t in codes.split()], (row, k)
+        assert sc == np.float32(float.fromhex(scale)), (row, sc)
+        assert k.view(np.uint8).tolist() == [int(t, 16) for t in packed.split()], row
+
+
+def pin_8bit_calls(o):
+    """8-bit plans: grid-exact inputs reduce exactly with zero states, each
+    value is quantized twice, the transport is (1 + 4/G)/2 of bf16, codes
+    are one byte each, and the telescoping identity holds."""
+    rng = np.random.default_rng(26)
+    for P, G in ((2, 32), (4, 64)):
+        N = P * G * 2
+        prm = _params(o, P, N, G, True, bits=8)
+        xs = [bf16_bits(grid_exact_inputs(rng, P, N, G, L=127)) for _ in range(3)]
+        for x, (r, mf, ms) in zip(xs, _run_sequence(o, prm, xs)):
+            assert np.array_equal(bits_to_f64(r.y), bits_to_f64(x).sum(axis=0))
+            assert not mf.any() and not ms.any()
+            assert (r.qcount == 2).all()
+            assert r.codes.shape == (P, N) and r.rcodes.shape == (N,)
+            assert (r.codes.nbytes + r.scales.nbytes) / (P * N * 2) == (1 + 4 / G) / 2
+    P, G = 4, 32
+    N = P * G * 2
+    prm = _params(o, P, N, G, True, bits=8)
+    S = np.zeros(N)
+    X = np.zeros(N)
+    xs = _sequence_inputs(rng, P, N, 12)
+    for t, (x, (r, mf, ms)) in enumerate(zip(xs, _run_sequence(o, prm, xs)), 1):
+        S += bits_to_f64(r.y)
+        X += bits_to_f64(x).sum(axis=0)
+        rhs = -(0.5 * mf.astype(np.float64) / 0.5
+                + 0.5 * ms.astype(np.float64) / (1 - np.float64(np.float32(0.95)))).sum(axis=0)
+        assert (np.abs((S - X) - rhs) <= 64 * t * P * 2.0 ** -24 * (1 + np.abs(S))).all()
+    # the transport bytes of a call are the quantizer's codes, one byte each
+    prm0 = _params(o, P, N, G, False, bits=8)
+    x0 = _sequence_inputs(rng, P, N, 1)[0]
+    r0 = o.allreduce(prm0, x0, None, None)
+    xf0 = o.bf16_to_f32(x0)
+    for rank in range(P):
+        for c in range(N // G):
+            k, sc = o.quantize_group_levels(xf0[rank, c * G:(c + 1) * G], 127)
+            assert np.array_equal(r0.codes[rank, c * G:(c + 1) * G], k.view(np.uint8))
+            assert r0.scales[rank, c] == sc
+    # 8-bit codes are finer than 4-bit ones: the output residual is smaller
+    x = _sequence_inputs(rng, P, N, 1)[0]
+    r4 = o.allreduce(_params(o, P, N, G, False), x, None, None)
+    r8 = o.allreduce(_params(o, P, N, G, False, bits=8), x, None, None)
+    ex = bits_to_f64(x).sum(axis=0)
+    assert np.abs(bits_to_f64(r8.y) - ex).mean() < 0.2 * np.abs(bits_to_f64(r4.y) - ex).mean()
 
 
 # ---------------------------------------------------------------- reduce-scatter

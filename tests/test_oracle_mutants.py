@@ -28,10 +28,10 @@ MUTANTS = {
         "                                   fmul(alpha, m_slow[row + j]));"),
     "ties_away_from_zero": ("float r = rintf(fdiv(v[j], scale));",
                             "float r = roundf(fdiv(v[j], scale));"),
-    "scale_over_eight": ("scale = fdiv(a, 7.0f);", "scale = fdiv(a, 8.0f);"),
+    "scale_over_eight": ("scale = fdiv(a, levels);", "scale = fdiv(a, levels + 1.0f);"),
     "nibbles_swapped": ("bytes[j] = (uint8_t)(lo | (hi << 4));",
                         "bytes[j] = (uint8_t)(hi | (lo << 4));"),
-    "no_clamp": ("if (r > 7.0f) r = 7.0f;", ""),
+    "no_clamp": ("if (r > levels) r = levels;", ""),
     "ema_decay_swapped": (
         "m_fast[row + j] = fadd(fmul(bf, m_fast[row + j]),\n"
         "                                           fmul(one_m_bf, e));",
@@ -58,6 +58,9 @@ MUTANTS = {
         "            if (prm->compensate) {",
         "/* 9. the owner alone also folds the requantization error in */\n"
         "            if (prm->compensate && requantize) {"),
+    "levels_off_by_one_for_8bit": ("const int L = prm->bits == 8 ? 127 : 7;",
+                                   "const int L = prm->bits == 8 ? 128 : 7;"),
+    "pack8_as_nibbles": ("bytes[j] = (uint8_t)k[j];", "bytes[j] = (uint8_t)(k[j] & 0x0f);"),
 }
 
 
