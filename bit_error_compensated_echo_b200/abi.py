@@ -42,7 +42,8 @@ class echo_config(ctypes.Structure):
     _fields_ = [("P", ctypes.c_int32), ("G", ctypes.c_int32), ("N", ctypes.c_int64),
                 ("compensate", ctypes.c_int32), ("alpha", ctypes.c_float),
                 ("beta_fast", ctypes.c_float), ("beta_slow", ctypes.c_float),
-                ("device", ctypes.c_int32), ("fixup", ctypes.c_int32)]
+                ("device", ctypes.c_int32), ("fixup", ctypes.c_int32),
+                ("bits", ctypes.c_int32)]
 
 
 class echo_debug_view(ctypes.Structure):

@@ -36,7 +36,7 @@ class EchoPlan:
 
     def __init__(self, P: int, N: int, G: int = 128, compensate: bool = True,
                  alpha: float = 0.5, beta_fast: float = 0.5, beta_slow: float = 0.95,
-                 device: Optional[int] = None, fixup: str = "exit"):
+                 device: Optional[int] = None, fixup: str = "exit", bits: int = 4):
         if device is None:
             device = torch.cuda.current_device()
         cfg = abi.echo_config_default()
@@ -47,7 +47,9 @@ class EchoPlan:
         if fixup not in abi.FIXUP_MODES:
             raise ValueError("fixup must be one of %s" % sorted(abi.FIXUP_MODES))
         cfg.fixup = abi.FIXUP_MODES[fixup]
+        cfg.bits = int(bits)
         self.cfg = cfg
+        self.bits = int(bits)
         self.P, self.N, self.G = int(P), int(N), int(G)
         self.compensate = bool(compensate)
         self.fixup = fixup
@@ -175,8 +177,10 @@ class EchoPlan:
 
         return {
             "m_fast": t(v.m_fast, (P, N), "<f4"), "m_slow": t(v.m_slow, (P, N), "<f4"),
-            "codes": t(v.codes, (P, N // 2), "|u1"), "scales": t(v.scales, (P, N // G), "<f4"),
-            "rcodes": t(v.rcodes, (N // 2,), "|u1"), "rscales": t(v.rscales, (N // G,), "<f4"),
+            "codes": t(v.codes, (P, N * self.bits // 8), "|u1"),
+            "scales": t(v.scales, (P, N // G), "<f4"),
+            "rcodes": t(v.rcodes, (N * self.bits // 8,), "|u1"),
+            "rscales": t(v.rscales, (N // G,), "<f4"),
             "e_req": t(v.e_req, (N,), "<f4"), "fixup_pending": bool(v.fixup_pending),
         }
 

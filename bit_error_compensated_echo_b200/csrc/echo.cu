@@ -45,9 +45,10 @@ Layout layout_of(const echo_config &c) {
     };
     L.m_fast = comp ? take(P * N * 4) : 0;
     L.m_slow = comp ? take(P * N * 4) : 0;
-    L.codes = take(P * N / 2);
+    const size_t B = (size_t)c.bits;
+    L.codes = take(P * N * B / 8);
     L.scales = take(P * (N / G) * 4);
-    L.rcodes = take(N / 2);
+    L.rcodes = take(N * B / 8);
     L.rscales = take((N / G) * 4);
     L.e_req = comp ? take(N * 4) : 0;
     L.total = off;
@@ -66,6 +67,7 @@ echo_status validate(const echo_config *c) {
     if (c->fixup < ECHO_FIXUP_EXIT || c->fixup > ECHO_FIXUP_DEFERRED)
         return ECHO_ERR_INVALID_ARG;
     if (c->device < 0) return ECHO_ERR_INVALID_ARG;
+    if (c->bits != 4 && c->bits != 8) return ECHO_ERR_UNSUPPORTED;
     return ECHO_OK;
 }
 
@@ -137,83 +139,101 @@ cudaEvent_t take_event(echo_plan *p) {
     return e;
 }
 
-template <int G, bool COMP, bool DEFER>
+template <int G, bool COMP, bool DEFER, int BITS>
 void launch_entry_t(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st) {
     dim3 grid(entry_blocks<COMP>(sl.v_count), (unsigned)(p->cfg.P * p->cfg.P));
-    echo_entry_kernel<G, COMP, DEFER><<<grid, kThreads, 0, st>>>(
+    echo_entry_kernel<G, COMP, DEFER, BITS><<<grid, kThreads, 0, st>>>(
         x, p->m_fast, p->m_slow, p->codes, p->scales, p->e_req, p->n_vec, p->chunk_vec, sl,
         p->cfg.P, p->k);
 }
 
-template <int G>
+template <int G, int BITS>
 void launch_entry_g(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
-    if (!p->cfg.compensate) launch_entry_t<G, false, false>(p, x, sl, st);
-    else if (defer) launch_entry_t<G, true, true>(p, x, sl, st);
-    else launch_entry_t<G, true, false>(p, x, sl, st);
+    if (!p->cfg.compensate) launch_entry_t<G, false, false, BITS>(p, x, sl, st);
+    else if (defer) launch_entry_t<G, true, true, BITS>(p, x, sl, st);
+    else launch_entry_t<G, true, false, BITS>(p, x, sl, st);
 }
 
-void launch_entry(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
+template <int BITS>
+void launch_entry_b(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
     switch (p->cfg.G) {
-        case 32: launch_entry_g<32>(p, x, sl, st, defer); break;
-        case 64: launch_entry_g<64>(p, x, sl, st, defer); break;
-        default: launch_entry_g<128>(p, x, sl, st, defer); break;
+        case 32: launch_entry_g<32, BITS>(p, x, sl, st, defer); break;
+        case 64: launch_entry_g<64, BITS>(p, x, sl, st, defer); break;
+        default: launch_entry_g<128, BITS>(p, x, sl, st, defer); break;
     }
 }
 
-template <int G, int P>
+void launch_entry(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
+    if (p->cfg.bits == 8) launch_entry_b<8>(p, x, sl, st, defer);
+    else launch_entry_b<4>(p, x, sl, st, defer);
+}
+
+template <int G, int P, int BITS>
 void launch_reduce_t(echo_plan *p, Slab sl, cudaStream_t st) {
     dim3 grid(reduce_blocks(sl.v_count), (unsigned)P);
     if (p->cfg.compensate)
-        echo_reduce_kernel<G, P, true><<<grid, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, true, BITS><<<grid, kThreads, 0, st>>>(
             p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl,
             p->k.neg_zero);
     else
-        echo_reduce_kernel<G, P, false><<<grid, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, false, BITS><<<grid, kThreads, 0, st>>>(
             p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl,
             p->k.neg_zero);
 }
 
-template <int G>
+template <int G, int BITS>
 void launch_reduce_g(echo_plan *p, Slab sl, cudaStream_t st) {
     switch (p->cfg.P) {
-        case 1: launch_reduce_t<G, 1>(p, sl, st); break;
-        case 2: launch_reduce_t<G, 2>(p, sl, st); break;
-        case 3: launch_reduce_t<G, 3>(p, sl, st); break;
-        case 4: launch_reduce_t<G, 4>(p, sl, st); break;
-        case 5: launch_reduce_t<G, 5>(p, sl, st); break;
-        case 6: launch_reduce_t<G, 6>(p, sl, st); break;
-        case 7: launch_reduce_t<G, 7>(p, sl, st); break;
-        default: launch_reduce_t<G, 8>(p, sl, st); break;
+        case 1: launch_reduce_t<G, 1, BITS>(p, sl, st); break;
+        case 2: launch_reduce_t<G, 2, BITS>(p, sl, st); break;
+        case 3: launch_reduce_t<G, 3, BITS>(p, sl, st); break;
+        case 4: launch_reduce_t<G, 4, BITS>(p, sl, st); break;
+        case 5: launch_reduce_t<G, 5, BITS>(p, sl, st); break;
+        case 6: launch_reduce_t<G, 6, BITS>(p, sl, st); break;
+        case 7: launch_reduce_t<G, 7, BITS>(p, sl, st); break;
+        default: launch_reduce_t<G, 8, BITS>(p, sl, st); break;
+    }
+}
+
+template <int BITS>
+void launch_reduce_b(echo_plan *p, Slab sl, cudaStream_t st) {
+    switch (p->cfg.G) {
+        case 32: launch_reduce_g<32, BITS>(p, sl, st); break;
+        case 64: launch_reduce_g<64, BITS>(p, sl, st); break;
+        default: launch_reduce_g<128, BITS>(p, sl, st); break;
     }
 }
 
 void launch_reduce(echo_plan *p, Slab sl, cudaStream_t st) {
-    switch (p->cfg.G) {
-        case 32: launch_reduce_g<32>(p, sl, st); break;
-        case 64: launch_reduce_g<64>(p, sl, st); break;
-        default: launch_reduce_g<128>(p, sl, st); break;
-    }
+    if (p->cfg.bits == 8) launch_reduce_b<8>(p, sl, st);
+    else launch_reduce_b<4>(p, sl, st);
 }
 
-template <int G>
+template <int G, int BITS>
 void launch_exit_g(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
     dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
     if (fix)
-        echo_exit_kernel<G, true><<<grid, kThreads, 0, st>>>(
+        echo_exit_kernel<G, true, BITS><<<grid, kThreads, 0, st>>>(
             p->rcodes, p->rscales, out, p->cfg.P, p->m_fast, p->m_slow, p->e_req, p->n_vec,
             p->chunk_vec, sl, p->k);
     else
-        echo_exit_kernel<G, false><<<grid, kThreads, 0, st>>>(
+        echo_exit_kernel<G, false, BITS><<<grid, kThreads, 0, st>>>(
             p->rcodes, p->rscales, out, p->cfg.P, p->m_fast, p->m_slow, p->e_req, p->n_vec,
             p->chunk_vec, sl, p->k);
 }
 
-void launch_exit(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+template <int BITS>
+void launch_exit_b(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
     switch (p->cfg.G) {
-        case 32: launch_exit_g<32>(p, out, sl, st, fix); break;
-        case 64: launch_exit_g<64>(p, out, sl, st, fix); break;
-        default: launch_exit_g<128>(p, out, sl, st, fix); break;
+        case 32: launch_exit_g<32, BITS>(p, out, sl, st, fix); break;
+        case 64: launch_exit_g<64, BITS>(p, out, sl, st, fix); break;
+        default: launch_exit_g<128, BITS>(p, out, sl, st, fix); break;
     }
+}
+
+void launch_exit(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+    if (p->cfg.bits == 8) launch_exit_b<8>(p, out, sl, st, fix);
+    else launch_exit_b<4>(p, out, sl, st, fix);
 }
 
 void launch_fixup(echo_plan *p, const float *sf, const float *ss, float *df, float *ds, bool apply,
@@ -226,43 +246,49 @@ void launch_fixup(echo_plan *p, const float *sf, const float *ss, float *df, flo
 
 Slab whole(const echo_plan *p) { return Slab{0, p->chunk_vec}; }
 
-template <int G, int P>
+template <int G, int P, int BITS>
 void launch_rs_t(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
     dim3 grid(reduce_blocks(sl.v_count), (unsigned)P);
     if (!p->cfg.compensate)
-        echo_rs_kernel<G, P, false, false><<<grid, kThreads, 0, st>>>(
+        echo_rs_kernel<G, P, false, false, BITS><<<grid, kThreads, 0, st>>>(
             p->codes, p->scales, out, p->m_fast, p->m_slow, p->e_req, p->n_vec, p->chunk_vec, sl,
             p->k);
     else if (fix)
-        echo_rs_kernel<G, P, true, true><<<grid, kThreads, 0, st>>>(
+        echo_rs_kernel<G, P, true, true, BITS><<<grid, kThreads, 0, st>>>(
             p->codes, p->scales, out, p->m_fast, p->m_slow, p->e_req, p->n_vec, p->chunk_vec, sl,
             p->k);
     else
-        echo_rs_kernel<G, P, true, false><<<grid, kThreads, 0, st>>>(
+        echo_rs_kernel<G, P, true, false, BITS><<<grid, kThreads, 0, st>>>(
             p->codes, p->scales, out, p->m_fast, p->m_slow, p->e_req, p->n_vec, p->chunk_vec, sl,
             p->k);
 }
 
-template <int G>
+template <int G, int BITS>
 void launch_rs_g(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
     switch (p->cfg.P) {
-        case 1: launch_rs_t<G, 1>(p, out, sl, st, fix); break;
-        case 2: launch_rs_t<G, 2>(p, out, sl, st, fix); break;
-        case 3: launch_rs_t<G, 3>(p, out, sl, st, fix); break;
-        case 4: launch_rs_t<G, 4>(p, out, sl, st, fix); break;
-        case 5: launch_rs_t<G, 5>(p, out, sl, st, fix); break;
-        case 6: launch_rs_t<G, 6>(p, out, sl, st, fix); break;
-        case 7: launch_rs_t<G, 7>(p, out, sl, st, fix); break;
-        default: launch_rs_t<G, 8>(p, out, sl, st, fix); break;
+        case 1: launch_rs_t<G, 1, BITS>(p, out, sl, st, fix); break;
+        case 2: launch_rs_t<G, 2, BITS>(p, out, sl, st, fix); break;
+        case 3: launch_rs_t<G, 3, BITS>(p, out, sl, st, fix); break;
+        case 4: launch_rs_t<G, 4, BITS>(p, out, sl, st, fix); break;
+        case 5: launch_rs_t<G, 5, BITS>(p, out, sl, st, fix); break;
+        case 6: launch_rs_t<G, 6, BITS>(p, out, sl, st, fix); break;
+        case 7: launch_rs_t<G, 7, BITS>(p, out, sl, st, fix); break;
+        default: launch_rs_t<G, 8, BITS>(p, out, sl, st, fix); break;
+    }
+}
+
+template <int BITS>
+void launch_rs_b(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+    switch (p->cfg.G) {
+        case 32: launch_rs_g<32, BITS>(p, out, sl, st, fix); break;
+        case 64: launch_rs_g<64, BITS>(p, out, sl, st, fix); break;
+        default: launch_rs_g<128, BITS>(p, out, sl, st, fix); break;
     }
 }
 
 void launch_rs(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    switch (p->cfg.G) {
-        case 32: launch_rs_g<32>(p, out, sl, st, fix); break;
-        case 64: launch_rs_g<64>(p, out, sl, st, fix); break;
-        default: launch_rs_g<128>(p, out, sl, st, fix); break;
-    }
+    if (p->cfg.bits == 8) launch_rs_b<8>(p, out, sl, st, fix);
+    else launch_rs_b<4>(p, out, sl, st, fix);
 }
 
 bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
@@ -286,6 +312,7 @@ void echo_config_default(echo_config *cfg) {
     cfg->beta_slow = 0.95f;
     cfg->device = 0;
     cfg->fixup = ECHO_FIXUP_EXIT;
+    cfg->bits = 4;
 }
 
 size_t echo_workspace_bytes(const echo_config *cfg) {

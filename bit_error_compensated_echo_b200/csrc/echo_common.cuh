@@ -121,31 +121,96 @@ __device__ __forceinline__ float2 prod2(float2 a, float2 b, float2 z) {
 // ---- exact integer <-> float steps without conversion instructions
 //
 // In [2^23, 2^24) consecutive floats are consecutive integers, so adding
-// 1.5*2^23 to a float q with |q| <= 7 rounds q to an integer under the
+// 1.5*2^23 to a float q with |q| <= 127 rounds q to an integer under the
 // current rounding (nearest, ties to even -- the same result as rint(q)),
-// and the low nibble of the sum's bit pattern is that integer in 4-bit two's
-// complement (the bits of 1.5*2^23 end in 0x0).  Going back, 2^23 + u with
-// u = (k + 8) in 0..15 has bit pattern 0x4B000000 | u, and subtracting
-// 2^23 + 8 gives k exactly.  Both replace the int<->float conversion
-// instructions, which issue at a fraction of the fp32 add rate.
+// and the low 4 (or 8) bits of the sum's bit pattern are that integer in
+// two's complement (the bits of 1.5*2^23 end in 0x00).  Going back, 2^23 + u
+// with u = k + 8 (k + 128 for 8-bit codes) has bit pattern 0x4B000000 | u,
+// and subtracting 2^23 + 8 (2^23 + 128) gives k exactly.  Both replace the
+// int<->float conversion instructions, which issue at a fraction of the
+// fp32 add rate.
 constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
-constexpr float kCodeMagic = 8388616.0f;     // 2^23 + 8
 
-// Codes 2j and 2j+1 of a packed word, as a float pair.  lo_nibs/hi_nibs
-// are (w ^ 0x88888888) & 0x0F0F0F0F and ((w ^ 0x88888888) >> 4) & 0x0F0F0F0F:
-// byte j of each holds k + 8 of element 2j / 2j+1.  One byte permute per
-// element builds the bit pattern 0x4B0000uu = 2^23 + u, and one packed
-// subtract of 2^23 + 8 leaves k exactly.
-__device__ __forceinline__ float2 code_pair(uint32_t lo_nibs, uint32_t hi_nibs, int j) {
-    const float2 m = make_float2(__uint_as_float(__byte_perm(lo_nibs, 0x4B000000u, 0x7540 + j)),
-                                 __uint_as_float(__byte_perm(hi_nibs, 0x4B000000u, 0x7540 + j)));
-    return sub2(m, splat2(kCodeMagic));
+// ---- code widths
+//
+// BITS = 4: levels -7..7, two codes per byte (element 2j in the low nibble
+// of byte j), 8 codes per 32-bit word.  BITS = 8: levels -127..127, one code
+// per byte, 4 per word.  A thread's 8 (16) codes are BITS/4 (BITS/2) words.
+template <int BITS>
+struct CodeWidth;
+template <>
+struct CodeWidth<4> {
+    static constexpr float levels = 7.0f;
+    static constexpr float offset = 8388616.0f;     // 2^23 + 8
+    static constexpr uint32_t bias = 0x88888888u;   // two's complement -> k + 8
+    static constexpr float tie_window = 0x1p-18f;   // see quantize8
+};
+template <>
+struct CodeWidth<8> {
+    static constexpr float levels = 127.0f;
+    static constexpr float offset = 8388736.0f;     // 2^23 + 128
+    static constexpr uint32_t bias = 0x80808080u;
+    static constexpr float tie_window = 0x1p-13f;
+};
+
+// The codes of 8 elements, packed (BITS/4 words).
+template <int BITS>
+struct Packed8 {
+    uint32_t w[BITS / 4];
+};
+
+template <int BITS>
+__device__ __forceinline__ void put_code(Packed8<BITS> &p, float t, int i) {
+    constexpr uint32_t mask = (1u << BITS) - 1u;
+    p.w[(i * BITS) / 32] |= (__float_as_uint(t) & mask) << ((i * BITS) % 32);
 }
-__device__ __forceinline__ uint32_t low_nibbles(uint32_t w) {
-    return (w ^ 0x88888888u) & 0x0F0F0F0Fu;
+
+// 2^23 + (byte b of word u), as a float
+__device__ __forceinline__ float byte_as_magic(uint32_t u, int b) {
+    return __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540 + b));
 }
-__device__ __forceinline__ uint32_t high_nibbles(uint32_t w) {
-    return ((w ^ 0x88888888u) >> 4) & 0x0F0F0F0Fu;
+
+// Decode 2n codes from n*BITS/16 words (n = 4: 8 codes, n = 8: 16 codes)
+// into n float pairs: pair p holds elements 2p and 2p+1.
+template <int BITS, int NPAIR>
+__device__ __forceinline__ void decode_pairs(const uint32_t *w, float2 k[NPAIR]) {
+    const float2 off = splat2(CodeWidth<BITS>::offset);
+    if (BITS == 4) {
+        // byte j of lo (hi) holds k + 8 of element 2j (2j+1) of that word
+#pragma unroll
+        for (int q = 0; q < NPAIR / 4; ++q) {
+            const uint32_t u = w[q] ^ CodeWidth<4>::bias;
+            const uint32_t lo = u & 0x0F0F0F0Fu, hi = (u >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                k[4 * q + j] = sub2(make_float2(byte_as_magic(lo, j), byte_as_magic(hi, j)), off);
+        }
+    } else {
+        // byte b of a word holds k + 128 of element 4q + b
+#pragma unroll
+        for (int q = 0; q < NPAIR / 2; ++q) {
+            const uint32_t u = w[q] ^ CodeWidth<8>::bias;
+            k[2 * q] = sub2(make_float2(byte_as_magic(u, 0), byte_as_magic(u, 1)), off);
+            k[2 * q + 1] = sub2(make_float2(byte_as_magic(u, 2), byte_as_magic(u, 3)), off);
+        }
+    }
+}
+
+// store / load the packed codes of 8-element vector v (BITS/4 words each)
+template <int BITS>
+__device__ __forceinline__ void store_packed8(uint32_t *base, int64_t v, const Packed8<BITS> &p) {
+    if (BITS == 4) base[v] = p.w[0];
+    else reinterpret_cast<uint2 *>(base)[v] = make_uint2(p.w[0], p.w[BITS / 4 - 1]);
+}
+template <int BITS>
+__device__ __forceinline__ void load_packed8(const uint32_t *base, int64_t v, uint32_t w[BITS / 4]) {
+    if (BITS == 4) {
+        w[0] = __ldg(base + v);
+    } else {
+        const uint2 t = __ldg(reinterpret_cast<const uint2 *>(base) + v);
+        w[0] = t.x;
+        w[BITS / 4 - 1] = t.y;
+    }
 }
 
 // bf16 round-to-nearest-even of a pair, returned as one word (first value in
@@ -158,78 +223,79 @@ __device__ __forceinline__ float2 bf16x2_to_f32(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
-// scale = a / 7, or 0 for an all-zero group
+// scale = a / L, or 0 for an all-zero group
+template <int BITS>
 __device__ __forceinline__ float group_scale(float a) {
-    return a != 0.0f ? __fdiv_rn(a, 7.0f) : 0.0f;
+    return a != 0.0f ? __fdiv_rn(a, CodeWidth<BITS>::levels) : 0.0f;
 }
 
 // Quantize 8 values of a group with one IEEE division per element:
-// k = clamp(rint(v / scale), -7, 7), ties to even, all 0 when scale == 0;
-// packed as quantize8 below, k as floats in kf.  Preferred where the values
-// are short bf16 numbers: their quotients land on or near half-integers
-// often, which would send quantize8 to its exact path most of the time.
-__device__ __forceinline__ uint32_t quantize8_div(const float v[8], float scale, float kf[8]) {
+// k = clamp(rint(v / scale), -L, L), ties to even, all 0 when scale == 0;
+// k as floats in kf.  Preferred where the values are short bf16 numbers.
+template <int BITS>
+__device__ __forceinline__ Packed8<BITS> quantize8_div(const float v[8], float scale, float kf[8]) {
+    constexpr float L = CodeWidth<BITS>::levels;
+    Packed8<BITS> p = {};
     if (scale == 0.0f) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) kf[i] = 0.0f;
-        return 0u;
+        return p;
     }
-    uint32_t w = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float q = fminf(fmaxf(__fdiv_rn(v[i], scale), -7.0f), 7.0f);
+        const float q = fminf(fmaxf(__fdiv_rn(v[i], scale), -L), L);
         const float t = __fadd_rn(q, kRoundMagic);
         kf[i] = __fsub_rn(t, kRoundMagic);
-        w |= (__float_as_uint(t) & 0xfu) << (4 * i);
+        put_code<BITS>(p, t, i);
     }
-    return w;
+    return p;
 }
 
-// Quantize 8 values of a group: k = clamp(rint(v / scale), -7, 7), ties to
-// even, all 0 when scale == 0.  Returns the packed word (element i in bits
-// 4i..4i+3, so byte j holds element 2j in its low nibble and 2j+1 in its
-// high nibble) and k as floats in kf.
+// Quantize 8 values of a group: k = clamp(rint(v / scale), -L, L), ties to
+// even, all 0 when scale == 0; the packed codes and k as floats in kf.
 //
 // inv is 1/scale rounded (0 when scale == 0, which makes every code 0).
 // For a normal scale, q~ = v*inv differs from the rounded quotient
-// fl(v/scale) by less than 2^-20 (both lie within a few units in the last
-// place of |v/scale| <= 7), so the two round to the same integer unless the
-// exact quotient lies within 2^-19 of a half-integer.  The fast path rounds
-// q~ and flags any element whose q~ lies within 2^-18 of a half-integer;
-// then (rarely), and for every group whose scale is subnormal, all 8 codes
-// are taken from the IEEE division itself.  Either way the codes are
-// exactly those of rint(v/scale).
+// fl(v/scale) by less than |q|*2^-22 (2^-20 for |q| <= 7, 2^-15 for
+// |q| <= 127), so the two round to the same integer unless the exact
+// quotient lies that close to a half-integer.  The fast path rounds q~ and
+// flags any element whose q~ lies within twice that (the tie window) of a
+// half-integer; then (rarely), and for every group whose scale is
+// subnormal, all 8 codes are taken from the IEEE division itself.  Either
+// way the codes are exactly those of rint(v/scale).  For a normal scale
+// |q~| <= L*(1 + 2^-22) < L + 1/2, so the fast path needs no clamp.
 struct GroupScale {
-    float scale;  // a / 7 (0 for an all-zero group)
+    float scale;  // a / L (0 for an all-zero group)
     float inv;    // 1 / scale rounded, 0 when scale == 0
     bool exact;   // subnormal scale: always use the division
 };
 
+template <int BITS>
 __device__ __forceinline__ GroupScale make_group_scale(float a) {
     GroupScale g;
-    g.scale = a != 0.0f ? __fdiv_rn(a, 7.0f) : 0.0f;
+    g.scale = a != 0.0f ? __fdiv_rn(a, CodeWidth<BITS>::levels) : 0.0f;
     g.exact = g.scale != 0.0f && g.scale < 1.17549435e-38f;  // below FLT_MIN
     g.inv = (g.scale != 0.0f && !g.exact) ? __frcp_rn(g.scale) : 0.0f;
     return g;
 }
 
-__device__ __forceinline__ uint32_t quantize8_exact(const float v[8], float scale, float kf[8]) {
-    uint32_t w = 0;
+template <int BITS>
+__device__ __forceinline__ Packed8<BITS> quantize8_exact(const float v[8], float scale, float kf[8]) {
+    constexpr float L = CodeWidth<BITS>::levels;
+    Packed8<BITS> p = {};
     for (int i = 0; i < 8; ++i) {
         float t = kRoundMagic;
-        if (scale != 0.0f)
-            t = __fadd_rn(fminf(fmaxf(__fdiv_rn(v[i], scale), -7.0f), 7.0f), kRoundMagic);
+        if (scale != 0.0f) t = __fadd_rn(fminf(fmaxf(__fdiv_rn(v[i], scale), -L), L), kRoundMagic);
         kf[i] = __fsub_rn(t, kRoundMagic);
-        w |= (__float_as_uint(t) & 0xfu) << (4 * i);
+        put_code<BITS>(p, t, i);
     }
-    return w;
+    return p;
 }
 
-// For a normal scale, |v*inv| <= 7*(1 + 2^-22) < 7.5, so no clamp is needed
-// on the fast path (the exact path keeps it).
-__device__ __forceinline__ uint32_t quantize8(const float v[8], const GroupScale &g, float kf[8],
-                                              float2 z) {
-    uint32_t w = 0;
+template <int BITS>
+__device__ __forceinline__ Packed8<BITS> quantize8(const float v[8], const GroupScale &g,
+                                                   float kf[8], float2 z) {
+    Packed8<BITS> p = {};
     const float2 inv2 = splat2(g.inv), magic2 = splat2(kRoundMagic);
     float dmax = 0.0f;
 #pragma unroll
@@ -241,11 +307,11 @@ __device__ __forceinline__ uint32_t quantize8(const float v[8], const GroupScale
         kf[i] = k.x;
         kf[i + 1] = k.y;
         dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
-        w |= (__float_as_uint(t.x) & 0xfu) << (4 * i);
-        w |= (__float_as_uint(t.y) & 0xfu) << (4 * i + 4);
+        put_code<BITS>(p, t.x, i);
+        put_code<BITS>(p, t.y, i + 1);
     }
-    if (g.exact || dmax > 0.5f - 0x1p-18f) w = quantize8_exact(v, g.scale, kf);
-    return w;
+    if (g.exact || dmax > 0.5f - CodeWidth<BITS>::tie_window) p = quantize8_exact<BITS>(v, g.scale, kf);
+    return p;
 }
 
 __device__ __forceinline__ void ld8(const float *p, float v[8]) {

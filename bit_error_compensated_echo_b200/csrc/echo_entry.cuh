@@ -31,7 +31,7 @@ inline unsigned entry_blocks(int64_t v_count) {
     return (unsigned)((v_count + per - 1) / per);
 }
 
-template <int G, bool COMP, bool DEFER>
+template <int G, bool COMP, bool DEFER, int BITS>
 __global__ void __launch_bounds__(kThreads, EntryShape<COMP>::MIN_BLOCKS)
 echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_slow,
                   uint32_t *__restrict__ codes, float *__restrict__ scales,
@@ -98,18 +98,18 @@ echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_sl
         a = group_absmax<LANES>(a);        // every lane of the warp takes part
         float kf[8];
         float scale;
-        uint32_t w;
+        Packed8<BITS> w;
         if (COMP) {   // corrected inputs carry full fp32 mantissas: ties are rare
-            const GroupScale gs = make_group_scale(a);
+            const GroupScale gs = make_group_scale<BITS>(a);
             scale = gs.scale;
-            w = quantize8(xt[v], gs, kf, z);
+            w = quantize8<BITS>(xt[v], gs, kf, z);
         } else {      // raw bf16 inputs: one IEEE division per element
-            scale = group_scale(a);
-            w = quantize8_div(xt[v], scale, kf);
+            scale = group_scale<BITS>(a);
+            w = quantize8_div<BITS>(xt[v], scale, kf);
         }
         if (!valid[v]) continue;
 
-        codes[(int64_t)r * n_vec + j[v]] = w;
+        store_packed8<BITS>(codes, (int64_t)r * n_vec + j[v], w);
         if ((threadIdx.x & (LANES - 1)) == 0)
             scales[(int64_t)r * (n_vec / LANES) + j[v] / LANES] = scale;
 

@@ -12,7 +12,7 @@ namespace echo {
 // to all P outputs.  FIX: also apply the owner's fix-up of both EMAs
 // (state += (1-beta)*e_req) for the owner's chunk.
 // Grid: x over the vectors of the slab, y = owner.
-template <int G, bool FIX>
+template <int G, bool FIX, int BITS>
 __global__ void __launch_bounds__(kThreads)
 echo_exit_kernel(const uint32_t *__restrict__ rcodes, const float *__restrict__ rscales,
                  OutPtrs out, int P, float *__restrict__ m_fast, float *__restrict__ m_slow,
@@ -24,12 +24,14 @@ echo_exit_kernel(const uint32_t *__restrict__ rcodes, const float *__restrict__ 
     if (local >= sl.v_count) return;
     const int64_t j = (int64_t)o * chunk_vec + sl.v_begin + local;
 
-    const uint32_t w = __ldg(rcodes + j);
+    uint32_t w[BITS / 4];
+    load_packed8<BITS>(rcodes, j, w);
     const float2 sc2 = splat2(__ldg(rscales + j / LANES));
-    const uint32_t lo = low_nibbles(w), hi = high_nibbles(w);
+    float2 kp[4];
+    decode_pairs<BITS, 4>(w, kp);
     uint32_t yw[4];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) yw[p] = bf16x2_bits_rn(mul2(code_pair(lo, hi, p), sc2));
+    for (int p = 0; p < 4; ++p) yw[p] = bf16x2_bits_rn(mul2(kp[p], sc2));
     const uint4 y = make_uint4(yw[0], yw[1], yw[2], yw[3]);
 #pragma unroll
     for (int r = 0; r < kMaxRanks; ++r)

@@ -81,18 +81,18 @@ void launch_all(const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigne
     dim3 g_chunk((unsigned)((chunk_vec + kThreads - 1) / kThreads), (unsigned)P);
     dim3 g_red(reduce_blocks(chunk_vec), (unsigned)P);
     if (comp) {
-        echo_entry_kernel<G, true, false><<<g_entry_c, kThreads, 0, st>>>(
+        echo_entry_kernel<G, true, false, 4><<<g_entry_c, kThreads, 0, st>>>(
             x, mf, ms, codes, scales, e_req, n_vec, chunk_vec, sl, P, k);
-        echo_reduce_kernel<G, P, true><<<g_red, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, true, 4><<<g_red, kThreads, 0, st>>>(
             codes, scales, rcodes, rscales, e_req, n_vec, chunk_vec, sl, k.neg_zero);
-        echo_exit_kernel<G, true><<<g_chunk, kThreads, 0, st>>>(
+        echo_exit_kernel<G, true, 4><<<g_chunk, kThreads, 0, st>>>(
             rcodes, rscales, y, P, mf, ms, e_req, n_vec, chunk_vec, sl, k);
     } else {
-        echo_entry_kernel<G, false, false><<<g_entry_o, kThreads, 0, st>>>(
+        echo_entry_kernel<G, false, false, 4><<<g_entry_o, kThreads, 0, st>>>(
             x, nullptr, nullptr, codes, scales, nullptr, n_vec, chunk_vec, sl, P, k);
-        echo_reduce_kernel<G, P, false><<<g_red, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, false, 4><<<g_red, kThreads, 0, st>>>(
             codes, scales, rcodes, rscales, nullptr, n_vec, chunk_vec, sl, k.neg_zero);
-        echo_exit_kernel<G, false><<<g_chunk, kThreads, 0, st>>>(
+        echo_exit_kernel<G, false, 4><<<g_chunk, kThreads, 0, st>>>(
             rcodes, rscales, y, P, nullptr, nullptr, nullptr, n_vec, chunk_vec, sl, k);
     }
 }
@@ -128,6 +128,7 @@ extern "C" echo_status echo_allreduce_noalloc(const echo_config *cfg, const void
         return ECHO_ERR_INVALID_ARG;
     if (cfg->compensate != 0 && cfg->compensate != 1) return ECHO_ERR_INVALID_ARG;
     if (cfg->device < 0 || cfg->device >= kMaxDevices) return ECHO_ERR_INVALID_ARG;
+    if (cfg->bits != 4) return ECHO_ERR_UNSUPPORTED;   // 4-bit codes only
     const bool comp = cfg->compensate != 0;
 
     // the size limit of the shared array, checked before anything else runs

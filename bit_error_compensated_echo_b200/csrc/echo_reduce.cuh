@@ -26,19 +26,32 @@ inline unsigned reduce_blocks(int64_t v_count) {
 // of the P ranks: dequantize each rank's codes and add them in fp32 in
 // ascending rank order from +0.  All P code and scale loads are issued
 // before any arithmetic.  Lanes with valid == false produce zeros.
-template <int G, int P>
+template <int G, int P, int BITS>
 __device__ __forceinline__ void sum_run(const uint32_t *__restrict__ codes,
                                         const float *__restrict__ scales, int64_t n_vec,
                                         int64_t j, bool valid, float2 z, float s[16]) {
     constexpr int LANES = G / kRedVec;
+    constexpr int WORDS = BITS / 2;                 // words holding 16 codes
     const int64_t n_run = n_vec / 2;
     const int64_t n_groups = n_run / LANES;
-    const uint2 *codes2 = reinterpret_cast<const uint2 *>(codes);
-    uint2 w[P];
+    uint32_t w[P][WORDS];
     float sc[P];
 #pragma unroll
     for (int r = 0; r < P; ++r) {
-        w[r] = valid ? __ldcs(codes2 + (int64_t)r * n_run + j) : make_uint2(0u, 0u);
+        const int64_t run = (int64_t)r * n_run + j;
+        if (BITS == 4) {
+            const uint2 t = valid ? __ldcs(reinterpret_cast<const uint2 *>(codes) + run)
+                                  : make_uint2(0u, 0u);
+            w[r][0] = t.x;
+            w[r][WORDS - 1] = t.y;
+        } else {
+            const uint4 t = valid ? __ldcs(reinterpret_cast<const uint4 *>(codes) + run)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+            w[r][0] = t.x;
+            w[r][1 % WORDS] = t.y;
+            w[r][2 % WORDS] = t.z;
+            w[r][WORDS - 1] = t.w;
+        }
         sc[r] = valid ? __ldg(scales + (int64_t)r * n_groups + j / LANES) : 0.0f;
     }
     float2 s2[8];
@@ -47,13 +60,10 @@ __device__ __forceinline__ void sum_run(const uint32_t *__restrict__ codes,
 #pragma unroll
     for (int r = 0; r < P; ++r) {
         const float2 sc2 = splat2(sc[r]);
-        const uint32_t lx = low_nibbles(w[r].x), hx = high_nibbles(w[r].x);
-        const uint32_t ly = low_nibbles(w[r].y), hy = high_nibbles(w[r].y);
+        float2 k[8];
+        decode_pairs<BITS, 8>(w[r], k);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            s2[p] = add2(s2[p], prod2(code_pair(lx, hx, p), sc2, z));
-            s2[4 + p] = add2(s2[4 + p], prod2(code_pair(ly, hy, p), sc2, z));
-        }
+        for (int p = 0; p < 8; ++p) s2[p] = add2(s2[p], prod2(k[p], sc2, z));
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -62,7 +72,7 @@ __device__ __forceinline__ void sum_run(const uint32_t *__restrict__ codes,
     }
 }
 
-template <int G, int P, bool COMP>
+template <int G, int P, bool COMP, int BITS>
 __global__ void __launch_bounds__(kThreads)
 echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
                    uint32_t *__restrict__ rcodes, float *__restrict__ rscales,
@@ -76,20 +86,24 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
     const int64_t j = (int64_t)o * chunk_run + sl.v_begin / 2 + local;  // run index in a rank
     const float2 z = splat2(neg_zero);
     float s[16];
-    sum_run<G, P>(codes, scales, n_vec, j, valid, z, s);
+    sum_run<G, P, BITS>(codes, scales, n_vec, j, valid, z, s);
 
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(s[i]));
     a = group_absmax<LANES>(a);
-    const GroupScale gs = make_group_scale(a);
+    const GroupScale gs = make_group_scale<BITS>(a);
     const float scale2 = gs.scale;
     float k2[16];
-    const uint32_t w0 = quantize8(s, gs, k2, z);
-    const uint32_t w1 = quantize8(s + 8, gs, k2 + 8, z);
+    const Packed8<BITS> w0 = quantize8<BITS>(s, gs, k2, z);
+    const Packed8<BITS> w1 = quantize8<BITS>(s + 8, gs, k2 + 8, z);
     if (!valid) return;
 
-    reinterpret_cast<uint2 *>(rcodes)[j] = make_uint2(w0, w1);
+    if (BITS == 4)
+        reinterpret_cast<uint2 *>(rcodes)[j] = make_uint2(w0.w[0], w1.w[0]);
+    else
+        reinterpret_cast<uint4 *>(rcodes)[j] =
+            make_uint4(w0.w[0], w0.w[BITS / 4 - 1], w1.w[0], w1.w[BITS / 4 - 1]);
     if ((threadIdx.x & (LANES - 1)) == 0) rscales[j / LANES] = scale2;
     if (COMP) {
         float e[16];
@@ -114,7 +128,7 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
 // is folded into its own EMAs here (FIX) or written to e_req for a
 // side-stream or deferred fix-up (COMP && !FIX).
 // Grid: x over the 16-element runs of the slab, y = owner.
-template <int G, int P, bool COMP, bool FIX>
+template <int G, int P, bool COMP, bool FIX, int BITS>
 __global__ void __launch_bounds__(kThreads)
 echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales, OutPtrs out,
                float *__restrict__ m_fast, float *__restrict__ m_slow, float *__restrict__ e_req,
@@ -127,7 +141,7 @@ echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ sca
     const int64_t j = (int64_t)o * chunk_run + lr;       // run index within a rank
     const float2 z = splat2(k.neg_zero);
     float s[16];
-    sum_run<G, P>(codes, scales, n_vec, j, true, z, s);
+    sum_run<G, P, BITS>(codes, scales, n_vec, j, true, z, s);
 
     uint32_t yw[8];
 #pragma unroll

@@ -64,7 +64,7 @@ typedef enum echo_status {
     ECHO_ERR_INVALID_ARG = 1, /* null pointer, value out of range */
     ECHO_ERR_SHAPE = 2,       /* N <= 0 or N % (P*G) != 0 */
     ECHO_ERR_ALIGNMENT = 3,   /* a buffer not 16-byte aligned */
-    ECHO_ERR_UNSUPPORTED = 4, /* P or G outside the supported set */
+    ECHO_ERR_UNSUPPORTED = 4, /* P, G or bits outside the supported set */
     ECHO_ERR_OOM = 5,         /* device allocation failed */
     ECHO_ERR_CUDA = 6,        /* a CUDA runtime call failed */
     ECHO_ERR_TIMEOUT = 7      /* reserved: no kernel here waits on a flag or barrier */
@@ -95,19 +95,24 @@ typedef struct echo_config {
     float beta_slow;    /* decay of the slow EMA, [0,1] */
     int32_t device;     /* CUDA device ordinal the plan lives on */
     int32_t fixup;      /* echo_fixup_mode */
+    int32_t bits;       /* code width: 4 (levels -7..7, two codes per byte) or
+                         * 8 (levels -127..127, one code per byte; the
+                         * pages' serving policy promotes the first half of
+                         * the layers to 8 bits, ai4snews "Perspective") */
 } echo_config;
 
 typedef struct echo_plan echo_plan;
 
 /* Fill *cfg with the defaults: compensate = 1, alpha = 0.5,
- * beta_fast = 0.5, beta_slow = 0.95, device = 0, fixup = ECHO_FIXUP_EXIT;
- * P, G, N are set to 0 and must be filled in. */
+ * beta_fast = 0.5, beta_slow = 0.95, device = 0, fixup = ECHO_FIXUP_EXIT,
+ * bits = 4; P, G, N are set to 0 and must be filled in. */
 void echo_config_default(echo_config *cfg);
 
 /* Bytes of device memory a plan for *cfg allocates: the EMA states
- * (2*P*N fp32 when compensating), the entry transport (P*N/2 code bytes +
- * P*N/G fp32 scales), the reduced transport (N/2 + 4*N/G bytes), e_req
- * (N fp32 when compensating), each sub-buffer 256-byte aligned.
+ * (2*P*N fp32 when compensating), the entry transport (P*N*bits/8 code
+ * bytes + P*N/G fp32 scales), the reduced transport (N*bits/8 + 4*N/G
+ * bytes), e_req (N fp32 when compensating), each sub-buffer 256-byte
+ * aligned.
  * Returns 0 for an invalid config. */
 size_t echo_workspace_bytes(const echo_config *cfg);
 
@@ -196,9 +201,9 @@ echo_status echo_set_state(echo_plan *plan, const float *m_fast_device,
 typedef struct echo_debug_view {
     float *m_fast;      /* [P][N] fp32, or NULL when not compensating */
     float *m_slow;      /* [P][N] fp32, or NULL */
-    uint8_t *codes;     /* [P][N/2] entry codes */
+    uint8_t *codes;     /* [P][N*bits/8] entry codes */
     float *scales;      /* [P][N/G] entry scales */
-    uint8_t *rcodes;    /* [N/2] requantized sum codes */
+    uint8_t *rcodes;    /* [N*bits/8] requantized sum codes */
     float *rscales;     /* [N/G] requantization scales */
     float *e_req;       /* [N] requantization error, or NULL */
     int32_t fixup_pending; /* 1 if a deferred fix-up is pending */
@@ -260,6 +265,7 @@ int32_t echo_launches_per_call(const echo_plan *plan);
  * that overlap on the GPU -- on streams not ordered with each other, or
  * from several host threads at once -- race on it and corrupt each other's
  * results.  Order them on one stream.
+ * 4-bit codes only (cfg->bits must be 4).
  * Calls no cudaMalloc, cudaFree or host allocator.  Errors as for
  * echo_allreduce, plus UNSUPPORTED for the size limit. */
 #define ECHO_NOALLOC_MAX_SCRATCH_BYTES ((size_t)80 << 20)

@@ -63,15 +63,16 @@ class SequenceChecker:
     def __init__(self, plan: EchoPlan, prm: oracle.Params, cols=None):
         self.plan, self.prm = plan, prm
         P, N, G = prm.P, prm.N, prm.G
+        cb = G * prm.bits // 8          # code bytes per group
         if cols is None:
             self.cols = None
             self.idx = np.arange(N)
-            self.cidx = np.arange(N // 2)
+            self.cidx = np.arange(N // G * cb)
             self.gidx = np.arange(N // G)
         else:
             self.cols = np.asarray(cols, np.int64)
             self.idx = workloads.column_elements(self.cols, G)
-            self.cidx = workloads.column_elements(self.cols, G // 2)
+            self.cidx = workloads.column_elements(self.cols, cb)
             self.gidx = self.cols
         n = self.idx.size
         self.mf = np.zeros((P, n), np.float32)
@@ -120,7 +121,7 @@ class SequenceChecker:
 def oracle_params(plan: EchoPlan) -> oracle.Params:
     c = plan.cfg
     return oracle.Params(P=c.P, N=c.N, G=c.G, compensate=bool(c.compensate), alpha=c.alpha,
-                         beta_fast=c.beta_fast, beta_slow=c.beta_slow)
+                         beta_fast=c.beta_fast, beta_slow=c.beta_slow, bits=c.bits)
 
 
 class RSChecker(SequenceChecker):

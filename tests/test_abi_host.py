@@ -62,6 +62,7 @@ def _cfg(abi, **kw):
     (dict(beta_slow=float("nan")), "ECHO_ERR_INVALID_ARG"),
     (dict(fixup=3), "ECHO_ERR_INVALID_ARG"), (dict(compensate=2), "ECHO_ERR_INVALID_ARG"),
     (dict(device=-1), "ECHO_ERR_INVALID_ARG"),
+    (dict(bits=6), "ECHO_ERR_UNSUPPORTED"), (dict(bits=0), "ECHO_ERR_UNSUPPORTED"),
 ])
 def test_invalid_configs_rejected_on_host(abi, kw, status):
     cfg = _cfg(abi, **kw)
@@ -85,11 +86,13 @@ def test_null_arguments(abi):
 def test_workspace_bytes_closed_form(abi):
     def al(b):
         return (b + 255) // 256 * 256
-    for P, G, k, comp in ((8, 128, 64, 1), (2, 32, 3, 0), (5, 64, 7, 1)):
+    for P, G, k, comp, bits in ((8, 128, 64, 1, 4), (2, 32, 3, 0, 4), (5, 64, 7, 1, 4),
+                                (4, 32, 5, 1, 8), (3, 128, 2, 0, 8)):
         N = P * G * k
-        c = _cfg(abi, P=P, G=G, N=N, compensate=comp)
+        c = _cfg(abi, P=P, G=G, N=N, compensate=comp, bits=bits)
         # codes, scales, reduced codes and scales
-        want = al(P * N // 2) + al(P * (N // G) * 4) + al(N // 2) + al((N // G) * 4)
+        want = (al(P * N * bits // 8) + al(P * (N // G) * 4) + al(N * bits // 8)
+                + al((N // G) * 4))
         if comp:
             want += 2 * al(P * N * 4) + al(N * 4)
         assert abi.echo_workspace_bytes(c) == want

@@ -1,0 +1,89 @@
+"""8-bit codes (levels -127..127, one byte per code) against the oracle:
+whole sequences, ragged shapes, the reduce-scatter, the pipelined host
+call, grid-exact inputs and the Llama-shaped workload on sampled columns.
+The pages' serving policy promotes the first half of the layers to 8 bits
+(ai4snews news summary, "Perspective"); a plan is 4- or 8-bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle_pins
+from bit_error_compensated_echo_b200 import workloads as W
+from bit_error_compensated_echo_b200.api import EchoPlan
+from parity import RSChecker, SequenceChecker, oracle_params
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _plan(P, N, G, comp=True, fixup="exit"):
+    return EchoPlan(P, N, G, compensate=comp, fixup=fixup, device=0, bits=8)
+
+
+@pytest.mark.parametrize("comp,fixup", [(True, "exit"), (True, "side"), (True, "deferred"),
+                                        (False, "exit")])
+def test_tiny_sequence_8bit(comp, fixup):
+    w = W.TINY
+    side = torch.cuda.Stream() if fixup == "side" else None
+    with _plan(w.P, w.N, w.G, comp, fixup) as plan:
+        chk = SequenceChecker(plan, oracle_params(plan))
+        for t in range(w.calls):
+            chk.step(W.generate(w, t, DEV), side_stream=side)
+
+
+@pytest.mark.parametrize("P,G,k", [(1, 32, 37), (3, 128, 41), (5, 64, 29), (8, 128, 37),
+                                   (8, 32, 1)], ids=lambda v: str(v))
+def test_ragged_8bit(P, G, k):
+    N = P * G * k
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    with _plan(P, N, G, True, "deferred") as plan:
+        chk = SequenceChecker(plan, oracle_params(plan))
+        for t in range(3):
+            chk.step(W.generate(w, t, DEV))
+
+
+def test_reduce_scatter_8bit():
+    w = W.with_size(W.TINY, P=4, rows=1, hidden=4 * 64 * 24, G=64)
+    with _plan(w.P, w.N, w.G, True, "deferred") as plan:
+        chk = RSChecker(plan, oracle_params(plan))
+        for t, op in enumerate("RARR"):
+            x = W.generate(w, t, DEV)
+            if op == "A":
+                chk.step(x)
+            else:
+                chk.step_rs(x)
+
+
+def test_grid_exact_8bit():
+    rng = np.random.default_rng(9)
+    P, G = 4, 64
+    N = P * G * 6
+    with _plan(P, N, G) as plan:
+        chk = SequenceChecker(plan, oracle_params(plan))
+        for _ in range(3):
+            xf = oracle_pins.grid_exact_inputs(rng, P, N, G, L=127)
+            x = torch.from_numpy(xf).to(torch.bfloat16).to(DEV)
+            out, _ = chk.step(x)
+            exact = torch.from_numpy(xf.astype(np.float64).sum(axis=0))
+            assert torch.equal(out[0].double().cpu(), exact)
+
+
+def test_host_call_8bit():
+    w = W.with_size(W.TINY, P=8, rows=1, hidden=8 * 128 * 9, G=128)
+    with _plan(w.P, w.N, w.G, True, "deferred") as a, _plan(w.P, w.N, w.G, True, "deferred") as b:
+        yh = torch.empty((w.P, w.N), dtype=torch.bfloat16, pin_memory=True)
+        for t in range(3):
+            x = W.generate(w, t, DEV)
+            yd = a.allreduce(x)
+            b.allreduce_host(x.cpu().pin_memory(), yh)
+            torch.cuda.synchronize()
+            assert torch.equal(yd.cpu(), yh)
+
+
+def test_llama_shape_8bit_sampled():
+    w = W.LLAMA
+    with _plan(w.P, w.N, w.G, True, "deferred") as plan:
+        chk = SequenceChecker(plan, oracle_params(plan), W.column_sample(w, 512))
+        for t in range(8):
+            chk.step(W.generate(w, t, DEV))
