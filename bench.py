@@ -59,38 +59,38 @@ WORKLOADS = {"large": W.LARGE, "llama": W.LLAMA, "depth": W.DEPTH, "tiny": W.TIN
 
 # ------------------------------------------------------------ byte counts
 
-def transport_bytes_per_elem(G: int) -> float:
-    """q: packed codes (1/2 byte) + fp32 scale per G elements."""
-    return 0.5 + 4.0 / G
+def transport_bytes_per_elem(G: int, bits: int = 4) -> float:
+    """q: packed codes (bits/8 bytes) + fp32 scale per G elements."""
+    return bits / 8.0 + 4.0 / G
 
 
-def call_min_bytes(P: int, N: int, G: int, comp: bool) -> float:
+def call_min_bytes(P: int, N: int, G: int, comp: bool, bits: int = 4) -> float:
     """Minimal HBM bytes of one call when each stage boundary is an HBM
     wire: read x, (read+write both states), write the P outputs, write and
     read the entry transport, write and read the reduced transport once,
     (write e_req and read it once)."""
-    q = transport_bytes_per_elem(G)
+    q = transport_bytes_per_elem(G, bits)
     if comp:
         return P * N * (2 + 16 + 2 + 2 * q) + N * (2 * q + 8)
     return P * N * (2 + 2 + 2 * q) + N * 2 * q
 
 
-def rs_min_bytes(P: int, N: int, G: int, comp: bool) -> float:
+def rs_min_bytes(P: int, N: int, G: int, comp: bool, bits: int = 4) -> float:
     """Minimal HBM bytes of one reduce-scatter call: read x, (read+write both
     states), write and read the entry transport, write each owner's bf16
     chunk, (write e_req and read it once in the next entry)."""
-    q = transport_bytes_per_elem(G)
+    q = transport_bytes_per_elem(G, bits)
     if comp:
         return P * N * (2 + 16 + 2 * q) + N * (2 + 8)
     return P * N * (2 + 2 * q) + N * 2
 
 
-def entry_bytes(P: int, N: int, G: int, comp: bool, fixup: str) -> float:
+def entry_bytes(P: int, N: int, G: int, comp: bool, fixup: str, bits: int = 4) -> float:
     """Algorithmic bytes of one echo_entry launch: read x (2 B), read and
     write both states (16 B), write codes + scales (q B) per rank-element;
     in deferred mode also read e_req of each rank's own chunk (4 B per
     element of N)."""
-    q = transport_bytes_per_elem(G)
+    q = transport_bytes_per_elem(G, bits)
     b = P * N * (2 + q)
     if comp:
         b += P * N * 16
@@ -251,7 +251,8 @@ def aggregate(per_rank_ms, per_rank_bytes):
 
 # ------------------------------------------------------------ CPU baseline
 
-def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: int = 7):
+def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: int = 7,
+                      bits: int = 4):
     """Time the oracle (as it stands, one host thread) on ``ncols`` group
     columns of workload ``w``; inputs are the device inputs at those columns
     when given, else a host draw of the same distribution."""
@@ -264,7 +265,7 @@ def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: i
     else:
         small = W.with_size(w, rows=1, hidden=idx.size)
         xb = W.bf16_bits(W.generate(small, 0, "cpu"))
-    prm = oracle.Params(P=w.P, N=w.N, G=w.G, compensate=comp)
+    prm = oracle.Params(P=w.P, N=w.N, G=w.G, compensate=comp, bits=bits)
     mf = np.zeros((w.P, idx.size), np.float32)
     ms = np.zeros_like(mf)
     t0 = time.perf_counter()
@@ -289,7 +290,7 @@ def run_step_mode(args, ws, rank, local):
     x = torch.empty((P, N), dtype=torch.bfloat16, device=dev)
     W.generate(w, rank, dev, out=x)
     out = torch.empty_like(x)
-    plan = EchoPlan(P, N, G, compensate=comp, fixup=fixup, device=local)
+    plan = EchoPlan(P, N, G, compensate=comp, fixup=fixup, device=local, bits=args.bits)
     side = torch.cuda.Stream(device=dev) if fixup == "side" else None
     stream = torch.cuda.current_stream(dev)
     rs = args.op == "reduce-scatter"
@@ -336,7 +337,7 @@ def run_step_mode(args, ws, rank, local):
         xh = torch.empty((P, N), dtype=torch.bfloat16, pin_memory=True)
         xh.copy_(x)
         yh = torch.empty((P, N), dtype=torch.bfloat16, pin_memory=True)
-        with EchoPlan(P, N, G, compensate=comp, fixup=fixup, device=local) as hp:
+        with EchoPlan(P, N, G, compensate=comp, fixup=fixup, device=local, bits=args.bits) as hp:
             for _ in range(args.warmup):
                 hp.allreduce_host(xh, yh)
             torch.cuda.synchronize(dev)
@@ -357,7 +358,7 @@ def run_step_mode(args, ws, rank, local):
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        gbs, dt, ncols = oracle_sample_run(w, comp, args.cpu_cols, x_dev=x)
+        gbs, dt, ncols = oracle_sample_run(w, comp, args.cpu_cols, x_dev=x, bits=args.bits)
         cpu = {"value": round(gbs, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "%d of %d group columns (x %d ranks x G=%d) of the same inputs, one "
                          "call from zero state, %.1f s on one host thread" %
@@ -366,20 +367,24 @@ def run_step_mode(args, ws, rank, local):
     if rank == 0:
         calls = prof["calls"]
         entry_ms = prof["entry_ms"] / max(calls, 1)
-        eb = entry_bytes(P, N, G, comp, fixup)
+        eb = entry_bytes(P, N, G, comp, fixup, args.bits)
         achieved = eb / (entry_ms / 1e3) / 1e9
-        bmin = rs_min_bytes(P, N, G, comp) if rs else call_min_bytes(P, N, G, comp)
+        bmin = (rs_min_bytes(P, N, G, comp, args.bits) if rs
+                else call_min_bytes(P, N, G, comp, args.bits))
         traffic = ncu_traffic(w.name, comp, fixup)
         metric = METRIC if comp else METRIC.replace("compensated", "uncompensated")
         if rs:
             metric = metric.replace("reduce input", "reduce-scatter input")
+        if args.bits == 8:
+            metric = metric.replace("4-bit", "8-bit")
         line = {
             "metric": metric,
             "value": round(value, 3), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, int4 transport, f32 sum+state",
             "data": "synthetic (seeded N(0,0.5^2) bf16 draws, no dataset)",
-            "config": {"workload": w.name, "op": args.op, "P": P, "N_per_rank": N, "G": G,
+            "config": {"workload": w.name, "op": args.op, "bits": args.bits, "P": P,
+                       "N_per_rank": N, "G": G,
                        "compensate": comp, "fixup": fixup, "alpha": 0.5, "beta_fast": 0.5,
                        "beta_slow": 0.95, "l2": "inputs larger than L2 (%.1f GiB of x per step)"
                        % (2 * P * N / 2**30), "parallelism": "replicas" if ws > 1 else "1 GPU"},
@@ -600,6 +605,7 @@ def main(argv=None):
     ap.add_argument("--fixup", choices=("exit", "side", "deferred"), default=BENCH_FIXUP)
     ap.add_argument("--uncompensated", action="store_true")
     ap.add_argument("--op", choices=("all-reduce", "reduce-scatter"), default="all-reduce")
+    ap.add_argument("--bits", type=int, choices=(4, 8), default=4)
     ap.add_argument("--mode", choices=("step", "depth-chain", "sweep", "overlap"), default="step")
     ap.add_argument("--sweep-max-mib", type=int, default=0,
                     help="sweep only points up to this many MiB per rank (0: all)")
