@@ -125,10 +125,16 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the dominant kernel's code with comments and whitespace
+    removed, so that only a change of code invalidates an ncu capture."""
+    import re
     h = hashlib.sha256()
     for rel in KERNEL_FILES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

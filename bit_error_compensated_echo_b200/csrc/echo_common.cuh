@@ -1,20 +1,20 @@
-// echo_common.cuh -- shared definitions of the sm_100a kernels of Echo's error-compensated 4-bit
-// all-reduce ("Echo: Error-Compensated 4-Bit Tensor-Parallel Communication",
+// echo_common.cuh -- shared definitions of the sm_100a kernels of Echo's error-compensated
+// 4-bit all-reduce ("Echo: Error-Compensated 4-Bit Tensor-Parallel Communication",
 // ai4snews news summary "Interpretation" and the arXiv abstract on the
 // fugumt mirror).  The operation each kernel computes is written out in
 // include/echo.h; here is how it maps onto the B200.
 //
 // The path is elementwise codec work bound by HBM bandwidth, not a
-// contraction, so there are no tensor cores.  A thread owns a run of
-// consecutive elements of one rank (8 in the entry and exit passes: one
-// 16-byte bf16 vector, two float4 of each EMA state, one 32-bit word of
-// packed codes; 16 in the reduce pass).  A group of G elements is G/8 (or
-// G/16) adjacent lanes of one warp; its absmax is a butterfly of
-// __shfl_xor_sync (max is order-free, so it is exact).  All fp32 arithmetic
-// uses the explicitly rounded intrinsics (__fadd_rn, __fmul_rn, __fdiv_rn),
-// which the compiler never contracts into FMA, so every value is the same
-// IEEE-754 single-precision result as a plain scalar evaluation of the
-// definition.
+// contraction, so there are no tensor cores.  A thread owns runs of
+// consecutive elements of one rank: vectors of 8 in the entry and exit
+// passes (one 16-byte bf16 vector, two float4 of each EMA state, one word of
+// 4-bit or two words of 8-bit codes), runs of 16 in the reduce pass.  A
+// group of G elements is G/8 (or G/16) adjacent lanes of one warp; its
+// absmax is a butterfly of __shfl_xor_sync (max is order-free, so it is
+// exact).  Every fp32 operation rounds once, to nearest even, exactly as a
+// plain scalar evaluation of the definition: scalar work uses the explicitly
+// rounded intrinsics (__fadd_rn, __fmul_rn, __fdiv_rn, never contracted),
+// paired work the sm_100 f32x2 instructions below.
 #pragma once
 
 #include <cuda_bf16.h>

@@ -17,9 +17,10 @@
  *
  * Per call, for P ranks of N elements each, group size G:
  *   1. c_r  = alpha*m_fast_r + (1-alpha)*m_slow_r;  xt_r = float(x_r) + c_r
- *   2. per group of G: a = max|xt|, scale = a/7,
- *      k = clamp(rint_half_even(xt/scale), -7, 7); codes packed two per
- *      byte (element 2j in the low nibble), scales fp32
+ *   2. per group of G: a = max|xt|, scale = a/L,
+ *      k = clamp(rint_half_even(xt/scale), -L, L) with L = 7 for 4-bit
+ *      codes (packed two per byte, element 2j in the low nibble) or
+ *      L = 127 for 8-bit codes (one byte each); scales fp32
  *   3. e_in_r = xt_r - k*scale;  m <- beta*m + (1-beta)*e_in_r (both EMAs)
  *   4. reduce-scatter: the owner o of chunk [o*N/P, (o+1)*N/P) sums
  *      s = sum over r = 0..P-1 (ascending) of k_r*scale_r in fp32
@@ -31,8 +32,8 @@
  * The constants alpha, beta_fast, beta_slow are parameters: the pages do not
  * fix them (defaults 0.5, 0.5, 0.95).
  *
- * All P ranks live on one GPU; the 4-bit "wire" between the stages is the
- * packed codes and scales in HBM.  Every quantity at element i depends only
+ * All P ranks live on one GPU; the "wire" between the stages is the packed
+ * codes and scales in HBM.  Every quantity at element i depends only
  * on the G-element group column of i across the P ranks.
  *
  * Conventions for every entry point:
