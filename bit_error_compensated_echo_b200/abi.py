@@ -1,5 +1,5 @@
-"""ctypes binding of the C ABI in include/echo.h -- same names, argument
-marshalling only.
+"""ctypes binding of the C ABI in include/echo.h and include/echo_rank.h --
+same names, argument marshalling only.
 
 Every function here forwards to the function of the same name in
 libecho_b200.so and raises ``EchoError`` (carrying the status code) when it
@@ -86,6 +86,22 @@ def _load():
         "echo_abi_version": (ctypes.c_int32, []),
         "echo_allreduce_noalloc": (st, [ctypes.POINTER(echo_config), ctypes.POINTER(vp),
                                         ctypes.POINTER(vp), vp, vp, vp]),
+        # include/echo_rank.h
+        "echo_rank_exchange_bytes": (st, [ctypes.POINTER(echo_config),
+                                          ctypes.POINTER(ctypes.c_size_t),
+                                          ctypes.POINTER(ctypes.c_size_t)]),
+        "echo_rank_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(echo_config)]),
+        "echo_rank_plan_create": (st, [ctypes.POINTER(vp), ctypes.POINTER(echo_config),
+                                       ctypes.c_int32]),
+        "echo_rank_plan_destroy": (st, [vp]),
+        "echo_rank_entry": (st, [vp, vp, vp, vp, vp]),
+        "echo_rank_reduce": (st, [vp, vp, vp, vp, vp, vp, vp]),
+        "echo_rank_exit": (st, [vp, vp, vp, vp, vp]),
+        "echo_rank_reduce_scatter": (st, [vp, vp, vp, vp, vp, vp]),
+        "echo_rank_reset_state": (st, [vp, vp]),
+        "echo_rank_get_state": (st, [vp, vp, vp, vp]),
+        "echo_rank_set_state": (st, [vp, vp, vp, vp]),
+        "echo_rank_launches_per_call": (ctypes.c_int32, [vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -201,3 +217,75 @@ def echo_allreduce_noalloc(cfg: echo_config, in_device: Sequence[int],
                                       _ptr_array(out_device), m_fast_device or None,
                                       m_slow_device or None, stream or None),
            "echo_allreduce_noalloc")
+
+
+# ---------------------------------------------------------------- include/echo_rank.h
+
+def echo_rank_exchange_bytes(cfg: echo_config) -> tuple[int, int]:
+    """(code bytes, scale bytes) of one chunk: C*bits/8 and 4*C/G."""
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib.echo_rank_exchange_bytes(ctypes.byref(cfg), ctypes.byref(cb), ctypes.byref(sb)),
+           "echo_rank_exchange_bytes")
+    return int(cb.value), int(sb.value)
+
+
+def echo_rank_workspace_bytes(cfg: echo_config) -> int:
+    return int(lib.echo_rank_workspace_bytes(ctypes.byref(cfg)))
+
+
+def echo_rank_plan_create(cfg: echo_config, rank: int) -> int:
+    h = ctypes.c_void_p()
+    _check(lib.echo_rank_plan_create(ctypes.byref(h), ctypes.byref(cfg), int(rank)),
+           "echo_rank_plan_create")
+    return h.value
+
+
+def echo_rank_plan_destroy(plan: int) -> None:
+    _check(lib.echo_rank_plan_destroy(plan), "echo_rank_plan_destroy")
+
+
+def echo_rank_entry(plan: int, x_device: int, send_codes_device: int, send_scales_device: int,
+                    stream: int = 0) -> None:
+    _check(lib.echo_rank_entry(plan, x_device, send_codes_device, send_scales_device,
+                               stream or None), "echo_rank_entry")
+
+
+def echo_rank_reduce(plan: int, recv_codes_device: int, recv_scales_device: int,
+                     red_codes_device: int, red_scales_device: int, stream: int = 0,
+                     side_stream: int = 0) -> None:
+    _check(lib.echo_rank_reduce(plan, recv_codes_device, recv_scales_device, red_codes_device,
+                                red_scales_device, stream or None, side_stream or None),
+           "echo_rank_reduce")
+
+
+def echo_rank_exit(plan: int, all_codes_device: int, all_scales_device: int, out_device: int,
+                   stream: int = 0) -> None:
+    _check(lib.echo_rank_exit(plan, all_codes_device, all_scales_device, out_device,
+                              stream or None), "echo_rank_exit")
+
+
+def echo_rank_reduce_scatter(plan: int, recv_codes_device: int, recv_scales_device: int,
+                             out_device: int, stream: int = 0, side_stream: int = 0) -> None:
+    _check(lib.echo_rank_reduce_scatter(plan, recv_codes_device, recv_scales_device, out_device,
+                                        stream or None, side_stream or None),
+           "echo_rank_reduce_scatter")
+
+
+def echo_rank_reset_state(plan: int, stream: int = 0) -> None:
+    _check(lib.echo_rank_reset_state(plan, stream or None), "echo_rank_reset_state")
+
+
+def echo_rank_get_state(plan: int, m_fast_device: int, m_slow_device: int,
+                        stream: int = 0) -> None:
+    _check(lib.echo_rank_get_state(plan, m_fast_device, m_slow_device, stream or None),
+           "echo_rank_get_state")
+
+
+def echo_rank_set_state(plan: int, m_fast_device: int, m_slow_device: int,
+                        stream: int = 0) -> None:
+    _check(lib.echo_rank_set_state(plan, m_fast_device, m_slow_device, stream or None),
+           "echo_rank_set_state")
+
+
+def echo_rank_launches_per_call(plan: int) -> int:
+    return int(lib.echo_rank_launches_per_call(plan))

@@ -27,6 +27,21 @@ def _stream_handle(stream: Optional[torch.cuda.Stream], device) -> int:
     return int(stream.cuda_stream)
 
 
+def make_config(P: int, N: int, G: int, compensate: bool, alpha: float, beta_fast: float,
+                beta_slow: float, device: int, fixup: str, bits: int) -> abi.echo_config:
+    """The echo_config of include/echo.h for these parameters."""
+    cfg = abi.echo_config_default()
+    cfg.P, cfg.N, cfg.G = int(P), int(N), int(G)
+    cfg.compensate = int(bool(compensate))
+    cfg.alpha, cfg.beta_fast, cfg.beta_slow = alpha, beta_fast, beta_slow
+    cfg.device = int(device)
+    if fixup not in abi.FIXUP_MODES:
+        raise ValueError("fixup must be one of %s" % sorted(abi.FIXUP_MODES))
+    cfg.fixup = abi.FIXUP_MODES[fixup]
+    cfg.bits = int(bits)
+    return cfg
+
+
 class EchoPlan:
     """A plan for P virtual ranks of N bf16 elements each, group size G.
 
@@ -39,15 +54,7 @@ class EchoPlan:
                  device: Optional[int] = None, fixup: str = "exit", bits: int = 4):
         if device is None:
             device = torch.cuda.current_device()
-        cfg = abi.echo_config_default()
-        cfg.P, cfg.N, cfg.G = int(P), int(N), int(G)
-        cfg.compensate = int(bool(compensate))
-        cfg.alpha, cfg.beta_fast, cfg.beta_slow = alpha, beta_fast, beta_slow
-        cfg.device = int(device)
-        if fixup not in abi.FIXUP_MODES:
-            raise ValueError("fixup must be one of %s" % sorted(abi.FIXUP_MODES))
-        cfg.fixup = abi.FIXUP_MODES[fixup]
-        cfg.bits = int(bits)
+        cfg = make_config(P, N, G, compensate, alpha, beta_fast, beta_slow, device, fixup, bits)
         self.cfg = cfg
         self.bits = int(bits)
         self.P, self.N, self.G = int(P), int(N), int(G)

@@ -20,12 +20,13 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libecho_b200.so")
 
-NVCC_FLAGS = [
+COMPILE_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17", "-fmad=false",
-    "-Xcompiler", "-fPIC", "-Xcompiler", "-O2", "-shared",
-    "-cudart", "static",
+    "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
 ]
+LINK_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static"]
+BUILD_DIR = os.path.join(PKG, "_build")
 
 
 def nvcc() -> str:
@@ -52,15 +53,34 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ into libecho_b200.so (skips if fresh)."""
+    """Compile every .cu under csrc/ (one nvcc per translation unit, in
+    parallel) and link them into libecho_b200.so (skips if fresh)."""
     if not force and up_to_date():
         return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc(), *NVCC_FLAGS, "-I" + INCLUDE, "-I" + CSRC, "-o", tmp, *sources()]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    tag = "%d" % os.getpid()
+    jobs = []
+    for src in sources():
+        obj = os.path.join(BUILD_DIR, os.path.basename(src) + "." + tag + ".o")
+        cmd = [nvcc(), *COMPILE_FLAGS, "-I" + INCLUDE, "-I" + CSRC, "-c", src, "-o", obj]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        jobs.append((obj, subprocess.Popen(cmd)))
+    failed = [obj for obj, proc in jobs if proc.wait() != 0]
+    objs = [obj for obj, _ in jobs]
+    try:
+        if failed:
+            raise subprocess.CalledProcessError(1, "nvcc -c " + " ".join(failed))
+        tmp = LIB + ".tmp" + tag
+        cmd = [nvcc(), *LINK_FLAGS, "-o", tmp, *objs]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.check_call(cmd)
+        os.replace(tmp, LIB)
+    finally:
+        for obj in objs:
+            if os.path.exists(obj):
+                os.remove(obj)
     return LIB
 
 

@@ -16,10 +16,8 @@
 #include <vector>
 
 #include "echo.h"
-#include "echo_entry.cuh"
-#include "echo_exit.cuh"
-#include "echo_fixup.cuh"
-#include "echo_reduce.cuh"
+#include "echo_host.h"
+#include "echo_launch.h"
 
 using namespace echo;
 
@@ -55,7 +53,15 @@ Layout layout_of(const echo_config &c) {
     return L;
 }
 
-echo_status validate(const echo_config *c) {
+struct ProfRecord {
+    cudaEvent_t ev[6];   // entry start, entry end, reduce end, exit end, fixup start, fixup end
+    bool side;
+    int kernels;         // kernels on the main stream (3 all-reduce, 2 reduce-scatter)
+};
+
+}  // namespace
+
+echo_status echo::validate_config(const echo_config *c) {
     if (!c) return ECHO_ERR_INVALID_ARG;
     if (c->P < 1 || c->P > ECHO_MAX_RANKS) return ECHO_ERR_UNSUPPORTED;
     if (c->G != 32 && c->G != 64 && c->G != 128) return ECHO_ERR_UNSUPPORTED;
@@ -71,33 +77,11 @@ echo_status validate(const echo_config *c) {
     return ECHO_OK;
 }
 
-// Restores the caller's current device on scope exit.
-struct DeviceGuard {
-    int prev = -1;
-    cudaError_t err = cudaSuccess;
-    explicit DeviceGuard(int dev) {
-        err = cudaGetDevice(&prev);
-        if (err == cudaSuccess && prev != dev) err = cudaSetDevice(dev);
-    }
-    ~DeviceGuard() {
-        int cur = -1;
-        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
-    }
-};
-
-struct ProfRecord {
-    cudaEvent_t ev[6];   // entry start, entry end, reduce end, exit end, fixup start, fixup end
-    bool side;
-    int kernels;         // kernels on the main stream (3 all-reduce, 2 reduce-scatter)
-};
-
-}  // namespace
-
 struct echo_plan {
     echo_config cfg;
     Layout L;
     int64_t n_vec = 0, chunk_vec = 0;
-    Consts k{};
+    Bufs b;                          // the workspace as the launchers see it
     char *ws = nullptr;
     float *m_fast = nullptr, *m_slow = nullptr, *scales = nullptr, *rscales = nullptr,
           *e_req = nullptr;
@@ -116,18 +100,6 @@ struct echo_plan {
 
 namespace {
 
-echo_status from_cuda(cudaError_t e) {
-    if (e == cudaSuccess) return ECHO_OK;
-    if (e == cudaErrorMemoryAllocation) return ECHO_ERR_OOM;
-    return ECHO_ERR_CUDA;
-}
-
-#define ECHO_TRY(expr)                                   \
-    do {                                                 \
-        cudaError_t e_ = (expr);                         \
-        if (e_ != cudaSuccess) return from_cuda(e_);     \
-    } while (0)
-
 cudaEvent_t take_event(echo_plan *p) {
     if (!p->pool.empty()) {
         cudaEvent_t e = p->pool.back();
@@ -139,159 +111,28 @@ cudaEvent_t take_event(echo_plan *p) {
     return e;
 }
 
-template <int G, bool COMP, bool DEFER, int BITS>
-void launch_entry_t(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st) {
-    dim3 grid(entry_blocks<COMP>(sl.v_count), (unsigned)(p->cfg.P * p->cfg.P));
-    echo_entry_kernel<G, COMP, DEFER, BITS><<<grid, kThreads, 0, st>>>(
-        x, p->m_fast, p->m_slow, p->codes, p->scales, p->e_req, p->n_vec, p->chunk_vec, sl,
-        p->cfg.P, p->k);
+// The plan's launches: all P virtual ranks in one grid, e_req over every
+// owner chunk, the state rows in rank order.
+void plan_entry(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
+    launch_entry(p->b, x, p->cfg.P, 0, p->chunk_vec, sl, defer, st);
 }
 
-template <int G, int BITS>
-void launch_entry_g(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
-    if (!p->cfg.compensate) launch_entry_t<G, false, false, BITS>(p, x, sl, st);
-    else if (defer) launch_entry_t<G, true, true, BITS>(p, x, sl, st);
-    else launch_entry_t<G, true, false, BITS>(p, x, sl, st);
+void plan_reduce(echo_plan *p, Slab sl, cudaStream_t st) { launch_reduce(p->b, p->cfg.P, sl, st); }
+
+void plan_exit(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+    launch_exit(p->b, out, p->cfg.P, p->cfg.P, sl, fix, st);
 }
 
-template <int BITS>
-void launch_entry_b(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
-    switch (p->cfg.G) {
-        case 32: launch_entry_g<32, BITS>(p, x, sl, st, defer); break;
-        case 64: launch_entry_g<64, BITS>(p, x, sl, st, defer); break;
-        default: launch_entry_g<128, BITS>(p, x, sl, st, defer); break;
-    }
+void plan_rs(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+    launch_rs(p->b, out, p->cfg.P, sl, fix, st);
 }
 
-void launch_entry(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool defer) {
-    if (p->cfg.bits == 8) launch_entry_b<8>(p, x, sl, st, defer);
-    else launch_entry_b<4>(p, x, sl, st, defer);
-}
-
-template <int G, int P, int BITS>
-void launch_reduce_t(echo_plan *p, Slab sl, cudaStream_t st) {
-    dim3 grid(reduce_blocks(sl.v_count), (unsigned)P);
-    if (p->cfg.compensate)
-        echo_reduce_kernel<G, P, true, BITS><<<grid, kThreads, 0, st>>>(
-            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl,
-            p->k.neg_zero);
-    else
-        echo_reduce_kernel<G, P, false, BITS><<<grid, kThreads, 0, st>>>(
-            p->codes, p->scales, p->rcodes, p->rscales, p->e_req, p->n_vec, p->chunk_vec, sl,
-            p->k.neg_zero);
-}
-
-template <int G, int BITS>
-void launch_reduce_g(echo_plan *p, Slab sl, cudaStream_t st) {
-    switch (p->cfg.P) {
-        case 1: launch_reduce_t<G, 1, BITS>(p, sl, st); break;
-        case 2: launch_reduce_t<G, 2, BITS>(p, sl, st); break;
-        case 3: launch_reduce_t<G, 3, BITS>(p, sl, st); break;
-        case 4: launch_reduce_t<G, 4, BITS>(p, sl, st); break;
-        case 5: launch_reduce_t<G, 5, BITS>(p, sl, st); break;
-        case 6: launch_reduce_t<G, 6, BITS>(p, sl, st); break;
-        case 7: launch_reduce_t<G, 7, BITS>(p, sl, st); break;
-        default: launch_reduce_t<G, 8, BITS>(p, sl, st); break;
-    }
-}
-
-template <int BITS>
-void launch_reduce_b(echo_plan *p, Slab sl, cudaStream_t st) {
-    switch (p->cfg.G) {
-        case 32: launch_reduce_g<32, BITS>(p, sl, st); break;
-        case 64: launch_reduce_g<64, BITS>(p, sl, st); break;
-        default: launch_reduce_g<128, BITS>(p, sl, st); break;
-    }
-}
-
-void launch_reduce(echo_plan *p, Slab sl, cudaStream_t st) {
-    if (p->cfg.bits == 8) launch_reduce_b<8>(p, sl, st);
-    else launch_reduce_b<4>(p, sl, st);
-}
-
-template <int G, int BITS>
-void launch_exit_g(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
-    if (fix)
-        echo_exit_kernel<G, true, BITS><<<grid, kThreads, 0, st>>>(
-            p->rcodes, p->rscales, out, p->cfg.P, p->m_fast, p->m_slow, p->e_req, p->n_vec,
-            p->chunk_vec, sl, p->k);
-    else
-        echo_exit_kernel<G, false, BITS><<<grid, kThreads, 0, st>>>(
-            p->rcodes, p->rscales, out, p->cfg.P, p->m_fast, p->m_slow, p->e_req, p->n_vec,
-            p->chunk_vec, sl, p->k);
-}
-
-template <int BITS>
-void launch_exit_b(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    switch (p->cfg.G) {
-        case 32: launch_exit_g<32, BITS>(p, out, sl, st, fix); break;
-        case 64: launch_exit_g<64, BITS>(p, out, sl, st, fix); break;
-        default: launch_exit_g<128, BITS>(p, out, sl, st, fix); break;
-    }
-}
-
-void launch_exit(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    if (p->cfg.bits == 8) launch_exit_b<8>(p, out, sl, st, fix);
-    else launch_exit_b<4>(p, out, sl, st, fix);
-}
-
-void launch_fixup(echo_plan *p, const float *sf, const float *ss, float *df, float *ds, bool apply,
-                  bool only_owner, Slab sl, cudaStream_t st) {
-    dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)p->cfg.P);
-    echo_fixup_kernel<<<grid, kThreads, 0, st>>>(sf, ss, df, ds, p->e_req, p->n_vec, p->chunk_vec,
-                                                 sl, p->cfg.P, apply ? 1 : 0, only_owner ? 1 : 0,
-                                                 p->k);
+void plan_fixup(echo_plan *p, const float *sf, const float *ss, float *df, float *ds, bool apply,
+                bool only_owner, Slab sl, cudaStream_t st) {
+    launch_fixup(p->b, sf, ss, df, ds, p->cfg.P, p->cfg.P, apply, only_owner, sl, st);
 }
 
 Slab whole(const echo_plan *p) { return Slab{0, p->chunk_vec}; }
-
-template <int G, int P, int BITS>
-void launch_rs_t(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    dim3 grid(reduce_blocks(sl.v_count), (unsigned)P);
-    if (!p->cfg.compensate)
-        echo_rs_kernel<G, P, false, false, BITS><<<grid, kThreads, 0, st>>>(
-            p->codes, p->scales, out, p->m_fast, p->m_slow, p->e_req, p->n_vec, p->chunk_vec, sl,
-            p->k);
-    else if (fix)
-        echo_rs_kernel<G, P, true, true, BITS><<<grid, kThreads, 0, st>>>(
-            p->codes, p->scales, out, p->m_fast, p->m_slow, p->e_req, p->n_vec, p->chunk_vec, sl,
-            p->k);
-    else
-        echo_rs_kernel<G, P, true, false, BITS><<<grid, kThreads, 0, st>>>(
-            p->codes, p->scales, out, p->m_fast, p->m_slow, p->e_req, p->n_vec, p->chunk_vec, sl,
-            p->k);
-}
-
-template <int G, int BITS>
-void launch_rs_g(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    switch (p->cfg.P) {
-        case 1: launch_rs_t<G, 1, BITS>(p, out, sl, st, fix); break;
-        case 2: launch_rs_t<G, 2, BITS>(p, out, sl, st, fix); break;
-        case 3: launch_rs_t<G, 3, BITS>(p, out, sl, st, fix); break;
-        case 4: launch_rs_t<G, 4, BITS>(p, out, sl, st, fix); break;
-        case 5: launch_rs_t<G, 5, BITS>(p, out, sl, st, fix); break;
-        case 6: launch_rs_t<G, 6, BITS>(p, out, sl, st, fix); break;
-        case 7: launch_rs_t<G, 7, BITS>(p, out, sl, st, fix); break;
-        default: launch_rs_t<G, 8, BITS>(p, out, sl, st, fix); break;
-    }
-}
-
-template <int BITS>
-void launch_rs_b(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    switch (p->cfg.G) {
-        case 32: launch_rs_g<32, BITS>(p, out, sl, st, fix); break;
-        case 64: launch_rs_g<64, BITS>(p, out, sl, st, fix); break;
-        default: launch_rs_g<128, BITS>(p, out, sl, st, fix); break;
-    }
-}
-
-void launch_rs(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    if (p->cfg.bits == 8) launch_rs_b<8>(p, out, sl, st, fix);
-    else launch_rs_b<4>(p, out, sl, st, fix);
-}
-
-bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 
 // Wait (on st) for a side-stream fix-up that may still be writing the state.
 cudaError_t order_after_side(echo_plan *p, cudaStream_t st) {
@@ -316,14 +157,14 @@ void echo_config_default(echo_config *cfg) {
 }
 
 size_t echo_workspace_bytes(const echo_config *cfg) {
-    if (validate(cfg) != ECHO_OK) return 0;
+    if (validate_config(cfg) != ECHO_OK) return 0;
     return layout_of(*cfg).total;
 }
 
 echo_status echo_plan_create(echo_plan **out, const echo_config *cfg) {
     if (!out) return ECHO_ERR_INVALID_ARG;
     *out = nullptr;
-    echo_status v = validate(cfg);
+    echo_status v = validate_config(cfg);
     if (v != ECHO_OK) return v;
 
     DeviceGuard guard(cfg->device);
@@ -335,13 +176,7 @@ echo_status echo_plan_create(echo_plan **out, const echo_config *cfg) {
     p->L = layout_of(*cfg);
     p->n_vec = cfg->N / kVec;
     p->chunk_vec = p->n_vec / cfg->P;
-    p->k.alpha = cfg->alpha;
-    p->k.one_m_alpha = 1.0f - cfg->alpha;
-    p->k.beta_fast = cfg->beta_fast;
-    p->k.one_m_beta_fast = 1.0f - cfg->beta_fast;
-    p->k.beta_slow = cfg->beta_slow;
-    p->k.one_m_beta_slow = 1.0f - cfg->beta_slow;
-    p->k.neg_zero = -0.0f;
+    p->b.k = make_consts(*cfg);
 
     cudaError_t e = cudaMalloc((void **)&p->ws, p->L.total);
     if (e != cudaSuccess) {
@@ -357,6 +192,19 @@ echo_status echo_plan_create(echo_plan **out, const echo_config *cfg) {
     p->rcodes = (uint32_t *)(p->ws + p->L.rcodes);
     p->rscales = (float *)(p->ws + p->L.rscales);
     p->e_req = comp ? (float *)(p->ws + p->L.e_req) : nullptr;
+    p->b.m_fast = p->m_fast;
+    p->b.m_slow = p->m_slow;
+    p->b.codes = p->codes;
+    p->b.scales = p->scales;
+    p->b.rcodes = p->rcodes;
+    p->b.rscales = p->rscales;
+    p->b.e_req = p->e_req;
+    p->b.n_vec = p->n_vec;
+    p->b.chunk_vec = p->chunk_vec;
+    p->b.P = cfg->P;
+    p->b.G = cfg->G;
+    p->b.bits = cfg->bits;
+    p->b.comp = comp;
 
     e = cudaEventCreateWithFlags(&p->ev_reduced, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_side_done, cudaEventDisableTiming);
@@ -441,17 +289,17 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
     const bool defer = comp && mode == ECHO_FIXUP_DEFERRED && p->pending;
 
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[0], st));
-    launch_entry(p, xi, whole(p), st, defer);
+    plan_entry(p, xi, whole(p), st, defer);
     ECHO_TRY(cudaGetLastError());
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[1], st));
-    launch_reduce(p, whole(p), st);
+    plan_reduce(p, whole(p), st);
     ECHO_TRY(cudaGetLastError());
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[2], st));
 
     const bool fix_in_exit = comp && mode == ECHO_FIXUP_EXIT;
     const bool fix_on_side = comp && mode == ECHO_FIXUP_SIDE;
     if (fix_on_side && side) ECHO_TRY(cudaEventRecord(p->ev_reduced, st));
-    launch_exit(p, yo, whole(p), st, fix_in_exit);
+    plan_exit(p, yo, whole(p), st, fix_in_exit);
     ECHO_TRY(cudaGetLastError());
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[3], st));
 
@@ -465,7 +313,7 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
             rec.side = true;
             ECHO_TRY(cudaEventRecord(rec.ev[4], fs));
         }
-        launch_fixup(p, p->m_fast, p->m_slow, p->m_fast, p->m_slow, true, true, whole(p), fs);
+        plan_fixup(p, p->m_fast, p->m_slow, p->m_fast, p->m_slow, true, true, whole(p), fs);
         ECHO_TRY(cudaGetLastError());
         if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[5], fs));
         if (side) {
@@ -516,10 +364,10 @@ echo_status echo_reduce_scatter(echo_plan *p, const void *const *in, void *const
     ECHO_TRY(order_after_side(p, st));
     const bool defer = comp && mode == ECHO_FIXUP_DEFERRED && p->pending;
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[0], st));
-    launch_entry(p, xi, whole(p), st, defer);
+    plan_entry(p, xi, whole(p), st, defer);
     ECHO_TRY(cudaGetLastError());
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[1], st));
-    launch_rs(p, yo, whole(p), st, comp && mode == ECHO_FIXUP_EXIT);
+    plan_rs(p, yo, whole(p), st, comp && mode == ECHO_FIXUP_EXIT);
     ECHO_TRY(cudaGetLastError());
     if (p->profiling) {
         ECHO_TRY(cudaEventRecord(rec.ev[2], st));
@@ -538,7 +386,7 @@ echo_status echo_reduce_scatter(echo_plan *p, const void *const *in, void *const
             rec.side = true;
             ECHO_TRY(cudaEventRecord(rec.ev[4], fs));
         }
-        launch_fixup(p, p->m_fast, p->m_slow, p->m_fast, p->m_slow, true, true, whole(p), fs);
+        plan_fixup(p, p->m_fast, p->m_slow, p->m_fast, p->m_slow, true, true, whole(p), fs);
         ECHO_TRY(cudaGetLastError());
         if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[5], fs));
         if (side) {
@@ -614,9 +462,9 @@ echo_status echo_allreduce_host(echo_plan *p, const void *const *in_host, void *
                                        width, (size_t)P, cudaMemcpyHostToDevice, s_in));
         ECHO_TRY(cudaEventRecord(p->hev[2 * k], s_in));
         ECHO_TRY(cudaStreamWaitEvent(s_comp, p->hev[2 * k], 0));
-        launch_entry(p, xi, sl, s_comp, defer);
-        launch_reduce(p, sl, s_comp);
-        launch_exit(p, yo, sl, s_comp, comp && !deferred);
+        plan_entry(p, xi, sl, s_comp, defer);
+        plan_reduce(p, sl, s_comp);
+        plan_exit(p, yo, sl, s_comp, comp && !deferred);
         ECHO_TRY(cudaGetLastError());
         ECHO_TRY(cudaEventRecord(p->hev[2 * k + 1], s_comp));
         ECHO_TRY(cudaStreamWaitEvent(s_out, p->hev[2 * k + 1], 0));
@@ -651,7 +499,7 @@ echo_status echo_get_state(echo_plan *p, float *m_fast, float *m_slow, void *str
     if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     ECHO_TRY(order_after_side(p, st));
-    launch_fixup(p, p->m_fast, p->m_slow, m_fast, m_slow, p->pending, false, whole(p), st);
+    plan_fixup(p, p->m_fast, p->m_slow, m_fast, m_slow, p->pending, false, whole(p), st);
     ECHO_TRY(cudaGetLastError());
     return ECHO_OK;
 }

@@ -14,6 +14,10 @@ namespace echo {
 //   DEFER : apply the previous call's pending owner fix-up first
 //           (state += (1-beta)*e_req on this rank's own chunk), which is the
 //           same fp32 operation the exit kernel would have done.
+// The kernel serves the P virtual ranks of one plan (grid y = P*P, rank0 = 0,
+// e_req holding every owner chunk: er_chunk_vec = chunk_vec) and one rank of
+// a group spread over processes (grid y = P, rank0 = that rank's index, e_req
+// holding its own chunk only: er_chunk_vec = 0).
 //   VPT   : vectors per thread.  A block covers kThreads*VPT vectors; thread t
 //           takes vectors t, t + kThreads, ... so each load instruction of a
 //           warp is contiguous, and all of a thread's loads are issued before
@@ -36,10 +40,11 @@ __global__ void __launch_bounds__(kThreads, EntryShape<COMP>::MIN_BLOCKS)
 echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_slow,
                   uint32_t *__restrict__ codes, float *__restrict__ scales,
                   const float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec,
-                  Slab sl, int P, Consts k) {
+                  Slab sl, int P, Consts k, int rank0, int64_t er_chunk_vec) {
     constexpr int LANES = G / kVec;
     constexpr int VPT = EntryShape<COMP>::VPT;
-    const int r = blockIdx.y / P, o = blockIdx.y % P;  // rank, owner chunk
+    const int r = blockIdx.y / P, o = blockIdx.y % P;  // rank (row), owner chunk
+    const bool own = (o == r + rank0);                  // this rank owns chunk o
     const int64_t base = (int64_t)blockIdx.x * (kThreads * VPT) + threadIdx.x;
     const float2 z = splat2(k.neg_zero);
 
@@ -59,7 +64,8 @@ echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_sl
                 const int64_t e0 = ((int64_t)r * n_vec + j[v]) * kVec;
                 ld8(m_fast + e0, mf[v]);
                 ld8(m_slow + e0, ms[v]);
-                if (DEFER && o == r) ld8(e_req + j[v] * kVec, er[v]);
+                if (DEFER && own)
+                    ld8(e_req + ((int64_t)o * er_chunk_vec + sl.v_begin + l) * kVec, er[v]);
             }
         } else {
 #pragma unroll
@@ -70,7 +76,7 @@ echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_sl
 #pragma unroll
     for (int v = 0; v < VPT; ++v) {
         if (COMP && valid[v]) {
-            if (DEFER && o == r) {
+            if (DEFER && own) {
                 const float2 obf = splat2(k.one_m_beta_fast), obs = splat2(k.one_m_beta_slow);
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {

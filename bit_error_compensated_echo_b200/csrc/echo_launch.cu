@@ -1,0 +1,174 @@
+// echo_launch.cu -- the one translation unit that instantiates the kernels
+// of echo_*.cuh, behind the launchers declared in echo_launch.h.
+#include "echo_entry.cuh"
+#include "echo_exit.cuh"
+#include "echo_fixup.cuh"
+#include "echo_launch.h"
+#include "echo_reduce.cuh"
+
+namespace echo {
+namespace {
+
+// ---- entry
+template <int G, bool COMP, bool DEFER, int BITS>
+void entry_t(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chunk_vec, Slab sl,
+             cudaStream_t st) {
+    dim3 grid(entry_blocks<COMP>(sl.v_count), (unsigned)(rows * b.P));
+    echo_entry_kernel<G, COMP, DEFER, BITS><<<grid, kThreads, 0, st>>>(
+        x, b.m_fast, b.m_slow, b.codes, b.scales, b.e_req, b.n_vec, b.chunk_vec, sl, b.P, b.k,
+        rank0, er_chunk_vec);
+}
+
+template <int G, int BITS>
+void entry_g(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er, Slab sl, bool defer,
+             cudaStream_t st) {
+    if (!b.comp) entry_t<G, false, false, BITS>(b, x, rows, rank0, er, sl, st);
+    else if (defer) entry_t<G, true, true, BITS>(b, x, rows, rank0, er, sl, st);
+    else entry_t<G, true, false, BITS>(b, x, rows, rank0, er, sl, st);
+}
+
+template <int BITS>
+void entry_b(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er, Slab sl, bool defer,
+             cudaStream_t st) {
+    switch (b.G) {
+        case 32: entry_g<32, BITS>(b, x, rows, rank0, er, sl, defer, st); break;
+        case 64: entry_g<64, BITS>(b, x, rows, rank0, er, sl, defer, st); break;
+        default: entry_g<128, BITS>(b, x, rows, rank0, er, sl, defer, st); break;
+    }
+}
+
+// ---- reduce
+template <int G, int P, int BITS>
+void reduce_t(const Bufs &b, int owners, Slab sl, cudaStream_t st) {
+    dim3 grid(reduce_blocks(sl.v_count), (unsigned)owners);
+    if (b.comp)
+        echo_reduce_kernel<G, P, true, BITS><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl,
+            b.k.neg_zero);
+    else
+        echo_reduce_kernel<G, P, false, BITS><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl,
+            b.k.neg_zero);
+}
+
+template <int G, int BITS>
+void reduce_g(const Bufs &b, int owners, Slab sl, cudaStream_t st) {
+    switch (b.P) {
+        case 1: reduce_t<G, 1, BITS>(b, owners, sl, st); break;
+        case 2: reduce_t<G, 2, BITS>(b, owners, sl, st); break;
+        case 3: reduce_t<G, 3, BITS>(b, owners, sl, st); break;
+        case 4: reduce_t<G, 4, BITS>(b, owners, sl, st); break;
+        case 5: reduce_t<G, 5, BITS>(b, owners, sl, st); break;
+        case 6: reduce_t<G, 6, BITS>(b, owners, sl, st); break;
+        case 7: reduce_t<G, 7, BITS>(b, owners, sl, st); break;
+        default: reduce_t<G, 8, BITS>(b, owners, sl, st); break;
+    }
+}
+
+template <int BITS>
+void reduce_b(const Bufs &b, int owners, Slab sl, cudaStream_t st) {
+    switch (b.G) {
+        case 32: reduce_g<32, BITS>(b, owners, sl, st); break;
+        case 64: reduce_g<64, BITS>(b, owners, sl, st); break;
+        default: reduce_g<128, BITS>(b, owners, sl, st); break;
+    }
+}
+
+// ---- exit
+template <int G, int BITS>
+void exit_g(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, bool fix,
+            cudaStream_t st) {
+    dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)owners);
+    if (fix)
+        echo_exit_kernel<G, true, BITS><<<grid, kThreads, 0, st>>>(
+            b.rcodes, b.rscales, out, n_out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec,
+            sl, b.k);
+    else
+        echo_exit_kernel<G, false, BITS><<<grid, kThreads, 0, st>>>(
+            b.rcodes, b.rscales, out, n_out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec,
+            sl, b.k);
+}
+
+template <int BITS>
+void exit_b(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, bool fix,
+            cudaStream_t st) {
+    switch (b.G) {
+        case 32: exit_g<32, BITS>(b, out, n_out, owners, sl, fix, st); break;
+        case 64: exit_g<64, BITS>(b, out, n_out, owners, sl, fix, st); break;
+        default: exit_g<128, BITS>(b, out, n_out, owners, sl, fix, st); break;
+    }
+}
+
+// ---- reduce-scatter
+template <int G, int P, int BITS>
+void rs_t(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix, cudaStream_t st) {
+    dim3 grid(reduce_blocks(sl.v_count), (unsigned)owners);
+    if (!b.comp)
+        echo_rs_kernel<G, P, false, false, BITS><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec, sl, b.k);
+    else if (fix)
+        echo_rs_kernel<G, P, true, true, BITS><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec, sl, b.k);
+    else
+        echo_rs_kernel<G, P, true, false, BITS><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec, sl, b.k);
+}
+
+template <int G, int BITS>
+void rs_g(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix, cudaStream_t st) {
+    switch (b.P) {
+        case 1: rs_t<G, 1, BITS>(b, out, owners, sl, fix, st); break;
+        case 2: rs_t<G, 2, BITS>(b, out, owners, sl, fix, st); break;
+        case 3: rs_t<G, 3, BITS>(b, out, owners, sl, fix, st); break;
+        case 4: rs_t<G, 4, BITS>(b, out, owners, sl, fix, st); break;
+        case 5: rs_t<G, 5, BITS>(b, out, owners, sl, fix, st); break;
+        case 6: rs_t<G, 6, BITS>(b, out, owners, sl, fix, st); break;
+        case 7: rs_t<G, 7, BITS>(b, out, owners, sl, fix, st); break;
+        default: rs_t<G, 8, BITS>(b, out, owners, sl, fix, st); break;
+    }
+}
+
+template <int BITS>
+void rs_b(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix, cudaStream_t st) {
+    switch (b.G) {
+        case 32: rs_g<32, BITS>(b, out, owners, sl, fix, st); break;
+        case 64: rs_g<64, BITS>(b, out, owners, sl, fix, st); break;
+        default: rs_g<128, BITS>(b, out, owners, sl, fix, st); break;
+    }
+}
+
+}  // namespace
+
+void launch_entry(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chunk_vec,
+                  Slab sl, bool defer, cudaStream_t st) {
+    if (b.bits == 8) entry_b<8>(b, x, rows, rank0, er_chunk_vec, sl, defer, st);
+    else entry_b<4>(b, x, rows, rank0, er_chunk_vec, sl, defer, st);
+}
+
+void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st) {
+    if (b.bits == 8) reduce_b<8>(b, owners, sl, st);
+    else reduce_b<4>(b, owners, sl, st);
+}
+
+void launch_exit(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, bool fix,
+                 cudaStream_t st) {
+    if (b.bits == 8) exit_b<8>(b, out, n_out, owners, sl, fix, st);
+    else exit_b<4>(b, out, n_out, owners, sl, fix, st);
+}
+
+void launch_rs(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix,
+               cudaStream_t st) {
+    if (b.bits == 8) rs_b<8>(b, out, owners, sl, fix, st);
+    else rs_b<4>(b, out, owners, sl, fix, st);
+}
+
+void launch_fixup(const Bufs &b, const float *src_fast, const float *src_slow, float *dst_fast,
+                  float *dst_slow, int ranks, int owners, bool apply, bool only_owner, Slab sl,
+                  cudaStream_t st) {
+    dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)owners);
+    echo_fixup_kernel<<<grid, kThreads, 0, st>>>(src_fast, src_slow, dst_fast, dst_slow, b.e_req,
+                                                 b.n_vec, b.chunk_vec, sl, ranks, apply ? 1 : 0,
+                                                 only_owner ? 1 : 0, b.k);
+}
+
+}  // namespace echo

@@ -1,0 +1,76 @@
+// echo_launch.h -- host-side launchers of the entry, reduce, exit,
+// reduce-scatter and fix-up kernels, shared by the plan of P virtual ranks
+// on one GPU (echo.cu) and the plan of one rank of a group spread over
+// processes (echo_rank.cu).  The kernels are instantiated once, in
+// echo_launch.cu; these functions pick the instance for the run-time code
+// width, group size and rank count and launch it on the given stream.  They
+// do not check errors: the caller reads cudaGetLastError().
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "echo.h"
+#include "echo_common.cuh"
+
+namespace echo {
+
+// The buffers and sizes one launch works on.
+//   n_vec     : 8-element vectors in one row of the codes / state arrays
+//   chunk_vec : vectors in one owner chunk of such a row
+//   P         : ranks summed by the reduce (and chunks per row at entry)
+struct Bufs {
+    float *m_fast = nullptr, *m_slow = nullptr;    // [rows][n_vec*8] fp32
+    uint32_t *codes = nullptr;                     // [rows][n_vec*8*bits/8] bytes
+    float *scales = nullptr;                       // [rows][n_vec*8/G]
+    uint32_t *rcodes = nullptr;                    // reduced codes
+    float *rscales = nullptr;                      // reduced scales
+    float *e_req = nullptr;                        // requantization / output residual
+    int64_t n_vec = 0, chunk_vec = 0;
+    int P = 1, G = 128, bits = 4;
+    bool comp = true;
+    Consts k{};
+};
+
+// The fp32 constants of the definition for *cfg; 1 - beta and 1 - alpha are
+// rounded once, as the oracle rounds them.
+inline Consts make_consts(const echo_config &c) {
+    Consts k{};
+    k.alpha = c.alpha;
+    k.one_m_alpha = 1.0f - c.alpha;
+    k.beta_fast = c.beta_fast;
+    k.one_m_beta_fast = 1.0f - c.beta_fast;
+    k.beta_slow = c.beta_slow;
+    k.one_m_beta_slow = 1.0f - c.beta_slow;
+    k.neg_zero = -0.0f;   // the run-time -0 addend of the packed products
+    return k;
+}
+
+// Entry over `rows` input rows (grid y = rows * P chunks).  rank0: index of
+// row 0 in the group (the owner test for the deferred fix-up);
+// er_chunk_vec: vectors between consecutive owners' e_req chunks (0 when
+// e_req holds one chunk).
+void launch_entry(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chunk_vec,
+                  Slab sl, bool defer, cudaStream_t st);
+
+// Reduce of `owners` chunks (grid y): sum the P rows, requantize, e_req.
+void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st);
+
+// Exit over `owners` chunks (grid y) into n_out outputs; fix: owner fix-up
+// of state row o for chunk o (the virtual-rank layout).
+void launch_exit(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, bool fix,
+                 cudaStream_t st);
+
+// Reduce-scatter second kernel over `owners` chunks (grid y): out.p[o]
+// receives bf16(s) of chunk o; fix: owner residual folded into state row o.
+void launch_rs(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix,
+               cudaStream_t st);
+
+// Owner fix-up (src == dst) or state copy with the fix-up applied on the
+// way, over `owners` chunks of `ranks` state rows.
+void launch_fixup(const Bufs &b, const float *src_fast, const float *src_slow, float *dst_fast,
+                  float *dst_slow, int ranks, int owners, bool apply, bool only_owner, Slab sl,
+                  cudaStream_t st);
+
+}  // namespace echo

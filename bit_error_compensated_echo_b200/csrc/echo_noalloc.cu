@@ -12,9 +12,8 @@
 #include <mutex>
 
 #include "echo.h"
-#include "echo_entry.cuh"
-#include "echo_exit.cuh"
-#include "echo_reduce.cuh"
+#include "echo_host.h"
+#include "echo_launch.h"
 
 using namespace echo;
 
@@ -64,52 +63,28 @@ cudaError_t scratch_address(int dev, unsigned char **out) {
     return cudaSuccess;
 }
 
-bool is_aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
-
-template <int G, int P>
+// The three launches of one call, on the array's carved sub-buffers.
 void launch_all(const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigned char *s,
-                const ScratchLayout &L, int64_t N, bool comp, const Consts &k, cudaStream_t st) {
-    const int64_t n_vec = N / kVec, chunk_vec = n_vec / P;
-    uint32_t *codes = (uint32_t *)(s + L.codes);
-    float *scales = (float *)(s + L.scales);
-    uint32_t *rcodes = (uint32_t *)(s + L.rcodes);
-    float *rscales = (float *)(s + L.rscales);
-    float *e_req = comp ? (float *)(s + L.e_req) : nullptr;
-    const Slab sl{0, chunk_vec};
-    dim3 g_entry_c(entry_blocks<true>(chunk_vec), (unsigned)(P * P));
-    dim3 g_entry_o(entry_blocks<false>(chunk_vec), (unsigned)(P * P));
-    dim3 g_chunk((unsigned)((chunk_vec + kThreads - 1) / kThreads), (unsigned)P);
-    dim3 g_red(reduce_blocks(chunk_vec), (unsigned)P);
-    if (comp) {
-        echo_entry_kernel<G, true, false, 4><<<g_entry_c, kThreads, 0, st>>>(
-            x, mf, ms, codes, scales, e_req, n_vec, chunk_vec, sl, P, k);
-        echo_reduce_kernel<G, P, true, 4><<<g_red, kThreads, 0, st>>>(
-            codes, scales, rcodes, rscales, e_req, n_vec, chunk_vec, sl, k.neg_zero);
-        echo_exit_kernel<G, true, 4><<<g_chunk, kThreads, 0, st>>>(
-            rcodes, rscales, y, P, mf, ms, e_req, n_vec, chunk_vec, sl, k);
-    } else {
-        echo_entry_kernel<G, false, false, 4><<<g_entry_o, kThreads, 0, st>>>(
-            x, nullptr, nullptr, codes, scales, nullptr, n_vec, chunk_vec, sl, P, k);
-        echo_reduce_kernel<G, P, false, 4><<<g_red, kThreads, 0, st>>>(
-            codes, scales, rcodes, rscales, nullptr, n_vec, chunk_vec, sl, k.neg_zero);
-        echo_exit_kernel<G, false, 4><<<g_chunk, kThreads, 0, st>>>(
-            rcodes, rscales, y, P, nullptr, nullptr, nullptr, n_vec, chunk_vec, sl, k);
-    }
-}
-
-template <int G>
-void launch_g(int P, const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigned char *s,
-              const ScratchLayout &L, int64_t N, bool comp, const Consts &k, cudaStream_t st) {
-    switch (P) {
-        case 1: launch_all<G, 1>(x, y, mf, ms, s, L, N, comp, k, st); break;
-        case 2: launch_all<G, 2>(x, y, mf, ms, s, L, N, comp, k, st); break;
-        case 3: launch_all<G, 3>(x, y, mf, ms, s, L, N, comp, k, st); break;
-        case 4: launch_all<G, 4>(x, y, mf, ms, s, L, N, comp, k, st); break;
-        case 5: launch_all<G, 5>(x, y, mf, ms, s, L, N, comp, k, st); break;
-        case 6: launch_all<G, 6>(x, y, mf, ms, s, L, N, comp, k, st); break;
-        case 7: launch_all<G, 7>(x, y, mf, ms, s, L, N, comp, k, st); break;
-        default: launch_all<G, 8>(x, y, mf, ms, s, L, N, comp, k, st); break;
-    }
+                const ScratchLayout &L, const echo_config &c, cudaStream_t st) {
+    Bufs b;
+    b.comp = c.compensate != 0;
+    b.m_fast = b.comp ? mf : nullptr;
+    b.m_slow = b.comp ? ms : nullptr;
+    b.codes = (uint32_t *)(s + L.codes);
+    b.scales = (float *)(s + L.scales);
+    b.rcodes = (uint32_t *)(s + L.rcodes);
+    b.rscales = (float *)(s + L.rscales);
+    b.e_req = b.comp ? (float *)(s + L.e_req) : nullptr;
+    b.n_vec = c.N / kVec;
+    b.chunk_vec = b.n_vec / c.P;
+    b.P = c.P;
+    b.G = c.G;
+    b.bits = 4;
+    b.k = make_consts(c);
+    const Slab sl{0, b.chunk_vec};
+    launch_entry(b, x, c.P, 0, b.chunk_vec, sl, false, st);
+    launch_reduce(b, c.P, sl, st);
+    launch_exit(b, y, c.P, c.P, sl, b.comp, st);
 }
 
 }  // namespace
@@ -118,17 +93,14 @@ extern "C" echo_status echo_allreduce_noalloc(const echo_config *cfg, const void
                                               void *const *out_device, float *m_fast_device,
                                               float *m_slow_device, void *stream) {
     if (!cfg || !in_device || !out_device) return ECHO_ERR_INVALID_ARG;
+    echo_config c = *cfg;
+    c.fixup = ECHO_FIXUP_EXIT;   // the fix-up always runs in the exit kernel here
+    const echo_status v = validate_config(&c);
+    if (v != ECHO_OK) return v;
+    if (cfg->device >= kMaxDevices) return ECHO_ERR_INVALID_ARG;
+    if (cfg->bits != 4) return ECHO_ERR_UNSUPPORTED;   // 4-bit codes only
     const int P = cfg->P, G = cfg->G;
     const int64_t N = cfg->N;
-    if (P < 1 || P > ECHO_MAX_RANKS) return ECHO_ERR_UNSUPPORTED;
-    if (G != 32 && G != 64 && G != 128) return ECHO_ERR_UNSUPPORTED;
-    if (N <= 0 || N % ((int64_t)P * G) != 0) return ECHO_ERR_SHAPE;
-    auto unit = [](float v) { return std::isfinite(v) && v >= 0.0f && v <= 1.0f; };
-    if (!unit(cfg->alpha) || !unit(cfg->beta_fast) || !unit(cfg->beta_slow))
-        return ECHO_ERR_INVALID_ARG;
-    if (cfg->compensate != 0 && cfg->compensate != 1) return ECHO_ERR_INVALID_ARG;
-    if (cfg->device < 0 || cfg->device >= kMaxDevices) return ECHO_ERR_INVALID_ARG;
-    if (cfg->bits != 4) return ECHO_ERR_UNSUPPORTED;   // 4-bit codes only
     const bool comp = cfg->compensate != 0;
 
     // the size limit of the shared array, checked before anything else runs
@@ -136,14 +108,14 @@ extern "C" echo_status echo_allreduce_noalloc(const echo_config *cfg, const void
     if (L.total > (size_t)ECHO_NOALLOC_MAX_SCRATCH_BYTES) return ECHO_ERR_UNSUPPORTED;
 
     if (comp && (!m_fast_device || !m_slow_device)) return ECHO_ERR_INVALID_ARG;
-    if (comp && (!is_aligned16(m_fast_device) || !is_aligned16(m_slow_device)))
+    if (comp && (!aligned16(m_fast_device) || !aligned16(m_slow_device)))
         return ECHO_ERR_ALIGNMENT;
     InPtrs x{};
     OutPtrs y{};
     const size_t bytes = (size_t)N * 2;
     for (int r = 0; r < P; ++r) {
         if (!in_device[r] || !out_device[r]) return ECHO_ERR_INVALID_ARG;
-        if (!is_aligned16(in_device[r]) || !is_aligned16(out_device[r])) return ECHO_ERR_ALIGNMENT;
+        if (!aligned16(in_device[r]) || !aligned16(out_device[r])) return ECHO_ERR_ALIGNMENT;
         x.p[r] = (const uint4 *)in_device[r];
         y.p[r] = (uint4 *)out_device[r];
     }
@@ -159,20 +131,7 @@ extern "C" echo_status echo_allreduce_noalloc(const echo_config *cfg, const void
     unsigned char *scratch = nullptr;
     cudaError_t e = scratch_address(cfg->device, &scratch);
     if (e == cudaSuccess) {
-        Consts k;
-        k.alpha = cfg->alpha;
-        k.one_m_alpha = 1.0f - cfg->alpha;
-        k.beta_fast = cfg->beta_fast;
-        k.one_m_beta_fast = 1.0f - cfg->beta_fast;
-        k.beta_slow = cfg->beta_slow;
-        k.one_m_beta_slow = 1.0f - cfg->beta_slow;
-        k.neg_zero = -0.0f;
-        cudaStream_t st = (cudaStream_t)stream;
-        switch (G) {
-            case 32: launch_g<32>(P, x, y, m_fast_device, m_slow_device, scratch, L, N, comp, k, st); break;
-            case 64: launch_g<64>(P, x, y, m_fast_device, m_slow_device, scratch, L, N, comp, k, st); break;
-            default: launch_g<128>(P, x, y, m_fast_device, m_slow_device, scratch, L, N, comp, k, st); break;
-        }
+        launch_all(x, y, m_fast_device, m_slow_device, scratch, L, *cfg, (cudaStream_t)stream);
         e = cudaGetLastError();
     }
     if (prev != cfg->device) cudaSetDevice(prev);

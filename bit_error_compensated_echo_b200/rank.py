@@ -1,0 +1,225 @@
+"""One rank of an Echo group spread over processes, one GPU each.
+
+The pages' setting is a tensor-parallel group of GPUs whose all-reduce moves
+4-bit integers and sums them in high precision (ai4snews news summary,
+"Interpretation"; arXiv abstract).  ``EchoRankPlan`` runs this rank's part
+of it: the library's kernels (include/echo_rank.h) do every arithmetic
+step, and the two exchange steps between them -- an all-to-all of the packed
+entry chunks and an all-gather of the owners' reduced chunks -- go through a
+transport, by default ``torch.distributed`` (NCCL between GPUs).  Only
+packed codes and fp32 group scales cross between ranks: C*bits/8 + 4*C/G
+bytes per chunk of C = N/P elements, against 2*C for a bf16 all-reduce.
+
+Run by every rank of a group with the same parameters, a call gives every
+rank the output that ``EchoPlan.allreduce`` gives P virtual ranks on one
+GPU, and leaves each rank the state of its virtual counterpart, bit for bit.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+import torch.distributed as dist
+
+from . import abi
+from .api import _stream_handle, make_config
+
+
+class TorchDistTransport:
+    """The two exchange steps over a torch.distributed process group.
+
+    all_to_all(recv, send): equal splits -- part o of ``send`` goes to rank o
+    and part r of ``recv`` comes from rank r.  all_gather(out, inp): part o
+    of ``out`` is rank o's ``inp``.  Both are ordered with the current CUDA
+    stream by torch.distributed (the collectives wait for the work queued on
+    it, and later work on it waits for them)."""
+
+    def __init__(self, group=None):
+        self.group = group
+
+    def all_to_all(self, recv: torch.Tensor, send: torch.Tensor) -> None:
+        dist.all_to_all_single(recv, send, group=self.group)
+
+    def all_gather(self, out: torch.Tensor, inp: torch.Tensor) -> None:
+        dist.all_gather_into_tensor(out, inp, group=self.group)
+
+
+class ExchangeBuffers:
+    """The exchange buffers of one rank (layouts: include/echo_rank.h).
+
+    With cb code bytes and cs scales per chunk:
+      send_codes [P*cb] u8, send_scales [P*cs] f32 : chunk o for rank o
+      recv_codes [P*cb] u8, recv_scales [P*cs] f32 : rank r's copy of this chunk
+      red_codes  [cb] u8,   red_scales  [cs] f32   : this rank's reduced chunk
+      all_codes  [P*cb] u8, all_scales  [P*cs] f32 : owner o's reduced chunk
+    """
+
+    def __init__(self, P: int, chunk_code_bytes: int, chunk_scale_bytes: int, device):
+        cb, cs = int(chunk_code_bytes), int(chunk_scale_bytes) // 4
+        u8, f32 = torch.uint8, torch.float32
+        self.P, self.cb, self.cs = int(P), cb, cs
+        self.send_codes = torch.empty(P * cb, dtype=u8, device=device)
+        self.send_scales = torch.empty(P * cs, dtype=f32, device=device)
+        self.recv_codes = torch.empty(P * cb, dtype=u8, device=device)
+        self.recv_scales = torch.empty(P * cs, dtype=f32, device=device)
+        self.red_codes = torch.empty(cb, dtype=u8, device=device)
+        self.red_scales = torch.empty(cs, dtype=f32, device=device)
+        self.all_codes = torch.empty(P * cb, dtype=u8, device=device)
+        self.all_scales = torch.empty(P * cs, dtype=f32, device=device)
+
+    def wire_bytes(self) -> int:
+        """Bytes this rank sends per all-reduce: (P-1) chunks in the
+        all-to-all and its reduced chunk to P-1 ranks in the all-gather."""
+        chunk = self.cb + 4 * self.cs
+        return 2 * (self.P - 1) * chunk
+
+
+def exchange(bufs: ExchangeBuffers, transport) -> None:
+    """The reduce-scatter exchange: every rank's chunk o to rank o."""
+    transport.all_to_all(bufs.recv_codes, bufs.send_codes)
+    transport.all_to_all(bufs.recv_scales, bufs.send_scales)
+
+
+def gather(bufs: ExchangeBuffers, transport) -> None:
+    """The all-gather exchange: every owner's reduced chunk to every rank."""
+    transport.all_gather(bufs.all_codes, bufs.red_codes)
+    transport.all_gather(bufs.all_scales, bufs.red_scales)
+
+
+class EchoRankPlan:
+    """Rank ``rank`` of a group of P ranks, N bf16 elements per rank.
+
+    Owns this rank's compensator state (two fp32 EMAs of N elements) and
+    its exchange buffers.  The stage methods (entry, reduce, exit,
+    reduce_scatter_finish) are the library calls; ``allreduce`` and
+    ``reduce_scatter`` put the transport's exchanges between them.
+    """
+
+    def __init__(self, P: int, rank: int, N: int, G: int = 128, compensate: bool = True,
+                 alpha: float = 0.5, beta_fast: float = 0.5, beta_slow: float = 0.95,
+                 device: Optional[int] = None, fixup: str = "deferred", bits: int = 4):
+        if device is None:
+            device = torch.cuda.current_device()
+        self.cfg = make_config(P, N, G, compensate, alpha, beta_fast, beta_slow, device, fixup,
+                               bits)
+        self.P, self.rank, self.N, self.G, self.bits = int(P), int(rank), int(N), int(G), int(bits)
+        self.compensate = bool(compensate)
+        self.fixup = fixup
+        self.device = torch.device("cuda", int(device))
+        cb, sb = abi.echo_rank_exchange_bytes(self.cfg)
+        self.handle = abi.echo_rank_plan_create(self.cfg, self.rank)
+        self.bufs = ExchangeBuffers(self.P, cb, sb, self.device)
+
+    # ------------------------------------------------------------ lifetime
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            abi.echo_rank_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    # ------------------------------------------------------------ checks
+    def _check_bf16(self, t: torch.Tensor, n: int, what: str) -> None:
+        if (t.dtype != torch.bfloat16 or t.numel() != n or not t.is_contiguous()
+                or t.device != self.device):
+            raise ValueError("%s: a contiguous bf16 tensor of %d elements on %s"
+                             % (what, n, self.device))
+
+    def _st(self, stream) -> int:
+        return _stream_handle(stream, self.device)
+
+    # ------------------------------------------------------------ stages
+    def entry(self, x: torch.Tensor, stream=None) -> None:
+        """Correction, quantization of every chunk, partial EMA update:
+        writes bufs.send_codes / bufs.send_scales."""
+        self._check_bf16(x, self.N, "input")
+        b = self.bufs
+        abi.echo_rank_entry(self.handle, x.data_ptr(), b.send_codes.data_ptr(),
+                            b.send_scales.data_ptr(), self._st(stream))
+
+    def reduce(self, stream=None, side_stream=None) -> None:
+        """Sum of the received chunks, requantization: writes
+        bufs.red_codes / bufs.red_scales (and the owner fix-up by mode)."""
+        b = self.bufs
+        side = int(side_stream.cuda_stream) if side_stream is not None else 0
+        abi.echo_rank_reduce(self.handle, b.recv_codes.data_ptr(), b.recv_scales.data_ptr(),
+                             b.red_codes.data_ptr(), b.red_scales.data_ptr(), self._st(stream),
+                             side)
+
+    def exit(self, out: torch.Tensor, stream=None) -> None:
+        """Dequantization of the gathered chunks into out (N bf16)."""
+        self._check_bf16(out, self.N, "output")
+        b = self.bufs
+        abi.echo_rank_exit(self.handle, b.all_codes.data_ptr(), b.all_scales.data_ptr(),
+                           out.data_ptr(), self._st(stream))
+
+    def reduce_scatter_finish(self, out: torch.Tensor, stream=None, side_stream=None) -> None:
+        """bf16 sum of this rank's chunk from the received chunks into out."""
+        self._check_bf16(out, self.N // self.P, "output")
+        b = self.bufs
+        side = int(side_stream.cuda_stream) if side_stream is not None else 0
+        abi.echo_rank_reduce_scatter(self.handle, b.recv_codes.data_ptr(),
+                                     b.recv_scales.data_ptr(), out.data_ptr(),
+                                     self._st(stream), side)
+
+    # ------------------------------------------------------------ calls
+    def allreduce(self, x: torch.Tensor, transport=None, out: Optional[torch.Tensor] = None,
+                  side_stream=None) -> torch.Tensor:
+        """One compensated all-reduce of this rank's x ([N] bf16) with the
+        other ranks of the group, on the current stream.  out may be x."""
+        transport = transport if transport is not None else TorchDistTransport()
+        if out is None:
+            out = torch.empty(self.N, dtype=torch.bfloat16, device=self.device)
+        self.entry(x)
+        exchange(self.bufs, transport)
+        self.reduce(side_stream=side_stream)
+        gather(self.bufs, transport)
+        self.exit(out)
+        return out
+
+    def reduce_scatter(self, x: torch.Tensor, transport=None, out: Optional[torch.Tensor] = None,
+                       side_stream=None) -> torch.Tensor:
+        """The reduce-scatter of sequence parallelism: returns this rank's
+        chunk (N/P bf16) of the sum."""
+        transport = transport if transport is not None else TorchDistTransport()
+        if out is None:
+            out = torch.empty(self.N // self.P, dtype=torch.bfloat16, device=self.device)
+        self.entry(x)
+        exchange(self.bufs, transport)
+        self.reduce_scatter_finish(out, side_stream=side_stream)
+        return out
+
+    # ------------------------------------------------------------ state
+    def reset_state(self, stream=None) -> None:
+        abi.echo_rank_reset_state(self.handle, self._st(stream))
+
+    def get_state(self, stream=None):
+        """(m_fast, m_slow) of this rank as new [N] fp32 tensors."""
+        mf = torch.empty(self.N, dtype=torch.float32, device=self.device)
+        ms = torch.empty_like(mf)
+        abi.echo_rank_get_state(self.handle, mf.data_ptr(), ms.data_ptr(), self._st(stream))
+        return mf, ms
+
+    def set_state(self, m_fast: torch.Tensor, m_slow: torch.Tensor, stream=None) -> None:
+        for m in (m_fast, m_slow):
+            if (m.dtype != torch.float32 or m.numel() != self.N or not m.is_contiguous()
+                    or m.device != self.device):
+                raise ValueError("state: a contiguous fp32 tensor of N elements on the device")
+        abi.echo_rank_set_state(self.handle, m_fast.data_ptr(), m_slow.data_ptr(),
+                                self._st(stream))
+
+    def launches_per_call(self) -> int:
+        return abi.echo_rank_launches_per_call(self.handle)
+
+    def workspace_bytes(self) -> int:
+        return abi.echo_rank_workspace_bytes(self.cfg)

@@ -1,0 +1,149 @@
+/*
+ * echo_rank.h -- one rank of an Echo group spread over P processes (one GPU
+ * each), with the two exchange steps left to the caller's collective
+ * library.
+ *
+ * The operation is the one echo.h defines (steps 1-7), for P real ranks
+ * instead of P virtual ranks on one GPU: the pages' setting is a
+ * tensor-parallel group of GPUs on NVLink whose all-reduce moves 4-bit
+ * integers and sums them in high precision (ai4snews news summary,
+ * "Interpretation", paragraph 1; arXiv abstract, "Abstract").  Such an
+ * all-reduce is a reduce-scatter followed by an all-gather; here each half
+ * moves the packed codes and scales, and everything else runs in this
+ * rank's kernels:
+ *
+ *   echo_rank_entry    steps 1-3 on this rank's input: correction, group
+ *                      quantization of every chunk, partial EMA update
+ *   (caller)           all-to-all: chunk o of every rank's codes and scales
+ *                      to rank o
+ *   echo_rank_reduce   steps 4-5 for this rank's own chunk: dequantize the P
+ *                      received chunks, sum in fp32 in ascending rank order,
+ *                      requantize, e_req; and, by fix-up mode, step 7
+ *   (caller)           all-gather of the P owners' reduced codes and scales
+ *   echo_rank_exit     step 6: dequantize every owner's chunk to bf16
+ *
+ * Run by every rank of the group with the same echo_config (P = the group
+ * size), the sequence gives every rank the output, codes and states that
+ * echo_allreduce gives the P virtual ranks of one plan, bit for bit.
+ * echo_rank_reduce_scatter replaces the last three steps for the
+ * reduce-scatter of sequence parallelism (echo_reduce_scatter in echo.h).
+ *
+ * Exchange buffers are owned by the caller (any device memory the collective
+ * library can use).  With C = N/P elements per chunk, cb = C*bits/8 code
+ * bytes and cs = C/G scales per chunk (echo_rank_exchange_bytes):
+ *   send codes  [P][cb] bytes, send scales  [P][cs] fp32: chunk o at o*cb / o*cs
+ *   recv codes  [P][cb] bytes, recv scales  [P][cs] fp32: from rank r at r*cb / r*cs
+ *   red codes   [cb] bytes,    red scales   [cs] fp32:    this rank's chunk
+ *   all codes   [P][cb] bytes, all scales   [P][cs] fp32: owner o's at o*cb / o*cs
+ * so the exchanges are an equal-split all-to-all of the send buffers into
+ * the recv buffers and an all-gather of the red buffers into the all
+ * buffers (for example torch.distributed all_to_all_single and
+ * all_gather_into_tensor, or ncclSend/ncclRecv in a group and
+ * ncclAllGather).  Within a chunk, codes and scales keep the layout of
+ * echo.h (element 2j in the low nibble of byte j for 4-bit codes, one byte
+ * each for 8-bit codes; one fp32 scale per group of G, in element order).
+ * Code buffers, inputs and outputs must be 16-byte aligned; scale buffers
+ * 4-byte aligned.
+ *
+ * Conventions as in echo.h: device pointers on the plan's device,
+ * stream-ordered asynchronous calls, host-side checks that return a status
+ * before any launch, no aborts, not thread-safe.  Nothing here waits on
+ * another rank: ordering between ranks is the collective library's.
+ */
+#ifndef ECHO_RANK_H
+#define ECHO_RANK_H
+
+#include "echo.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct echo_rank_plan echo_rank_plan;
+
+/* Bytes of one chunk's codes (C*bits/8) and scales (4*C/G) for *cfg.
+ * Errors: the same checks as echo_plan_create (INVALID_ARG, UNSUPPORTED,
+ * SHAPE). */
+echo_status echo_rank_exchange_bytes(const echo_config *cfg, size_t *chunk_code_bytes,
+                                     size_t *chunk_scale_bytes);
+
+/* Bytes of device memory a rank plan allocates: this rank's EMA states
+ * (2*N fp32) and e_req of its own chunk (C fp32), when compensating, each
+ * 256-byte aligned; 0 for an invalid config. */
+size_t echo_rank_workspace_bytes(const echo_config *cfg);
+
+/* Plan of rank `rank` (0 <= rank < cfg->P) of a group of cfg->P ranks:
+ * validates *cfg as echo_plan_create does, allocates the workspace on
+ * cfg->device and zeroes the state.  Synchronizes the device.
+ * Errors: INVALID_ARG (also rank out of range), UNSUPPORTED, SHAPE, OOM,
+ * CUDA.  *out is NULL on error. */
+echo_status echo_rank_plan_create(echo_rank_plan **out, const echo_config *cfg, int32_t rank);
+
+/* Free the plan (after synchronizing its device); NULL is ignored. */
+echo_status echo_rank_plan_destroy(echo_rank_plan *plan);
+
+/* Steps 1-3 on this rank's input, writing the send buffers.  With
+ * ECHO_FIXUP_DEFERRED the previous call's owner fix-up is folded in first.
+ *   x_device       : bf16, N elements of this rank (read)
+ *   send_codes     : [P][cb] bytes (written)
+ *   send_scales    : [P][cs] fp32 (written)
+ * One kernel.  Errors: INVALID_ARG (null), ALIGNMENT, CUDA. */
+echo_status echo_rank_entry(echo_rank_plan *plan, const void *x_device, void *send_codes_device,
+                            float *send_scales_device, void *stream);
+
+/* Steps 4-5 for this rank's chunk, from the received buffers, writing the
+ * reduced codes and scales that the all-gather distributes, and keeping
+ * e_req in the plan.  Step 7 by the plan's fix-up mode: EXIT runs it here on
+ * stream after the reduce, SIDE on side_stream (NULL: on stream; the plan's
+ * next call waits for it), DEFERRED folds it into the next entry.
+ *   recv_codes, recv_scales : [P][cb] bytes, [P][cs] fp32 (read)
+ *   red_codes, red_scales   : [cb] bytes, [cs] fp32 (written)
+ * Must follow an echo_rank_entry on the plan (a second reduce without a new
+ * entry would apply the fix-up twice).  One kernel, two with the fix-up.
+ * Errors: INVALID_ARG (null, or no entry since the last reduce),
+ * ALIGNMENT, CUDA. */
+echo_status echo_rank_reduce(echo_rank_plan *plan, const void *recv_codes_device,
+                             const float *recv_scales_device, void *red_codes_device,
+                             float *red_scales_device, void *stream, void *side_stream);
+
+/* Step 6: dequantize the P owners' reduced chunks to bf16.
+ *   all_codes, all_scales : [P][cb] bytes, [P][cs] fp32 (read)
+ *   out_device            : bf16, N elements (written); may be this rank's
+ *                           input
+ * One kernel.  Reads no plan state.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+echo_status echo_rank_exit(echo_rank_plan *plan, const void *all_codes_device,
+                           const float *all_scales_device, void *out_device, void *stream);
+
+/* The reduce-scatter of sequence parallelism, after echo_rank_entry and the
+ * all-to-all: out_device (C bf16 elements) receives bf16(s) of this rank's
+ * chunk, quantized once at entry; the output residual s - float(bf16(s))
+ * enters this rank's EMAs by the fix-up mode, as in echo_rank_reduce.
+ * One kernel, two in side-stream mode.  Errors as echo_rank_reduce. */
+echo_status echo_rank_reduce_scatter(echo_rank_plan *plan, const void *recv_codes_device,
+                                     const float *recv_scales_device, void *out_device,
+                                     void *stream, void *side_stream);
+
+/* Zero this rank's state and drop a pending fix-up, on stream (a no-op when
+ * compensate == 0). */
+echo_status echo_rank_reset_state(echo_rank_plan *plan, void *stream);
+
+/* Copy this rank's states ([N] fp32 each), with a pending fix-up applied,
+ * into caller device buffers; the plan's state is unchanged.
+ * Errors: INVALID_ARG (null, or compensate == 0), ALIGNMENT, CUDA. */
+echo_status echo_rank_get_state(echo_rank_plan *plan, float *m_fast_device,
+                                float *m_slow_device, void *stream);
+
+/* Overwrite this rank's states from caller device buffers ([N] fp32 each)
+ * and drop a pending fix-up.  Errors as echo_rank_get_state. */
+echo_status echo_rank_set_state(echo_rank_plan *plan, const float *m_fast_device,
+                                const float *m_slow_device, void *stream);
+
+/* Kernels one all-reduce (entry + reduce + exit) launches with this plan:
+ * 3, or 4 when the fix-up runs as its own kernel (EXIT and SIDE modes). */
+int32_t echo_rank_launches_per_call(const echo_rank_plan *plan);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ECHO_RANK_H */

@@ -98,6 +98,38 @@ def test_workspace_bytes_closed_form(abi):
         assert abi.echo_workspace_bytes(c) == want
 
 
+def test_rank_plan_sizes_and_host_checks(abi):
+    """The rank path (include/echo_rank.h): chunk sizes and workspace in
+    closed form, and invalid arguments rejected before any CUDA call."""
+    def al(b):
+        return (b + 255) // 256 * 256
+    for P, G, k, comp, bits in ((8, 128, 64, 1, 4), (2, 32, 3, 0, 4), (4, 32, 5, 1, 8)):
+        N = P * G * k
+        c = _cfg(abi, P=P, G=G, N=N, compensate=comp, bits=bits)
+        C = N // P
+        assert abi.echo_rank_exchange_bytes(c) == (C * bits // 8, C // G * 4)
+        want = (2 * al(N * 4) + al(C * 4)) if comp else 0
+        assert abi.echo_rank_workspace_bytes(c) == want
+    c = _cfg(abi)
+    for rank in (-1, 8):
+        with pytest.raises(abi.EchoError) as e:
+            abi.echo_rank_plan_create(c, rank)
+        assert e.value.status == abi.ECHO_ERR_INVALID_ARG
+    with pytest.raises(abi.EchoError) as e:
+        abi.echo_rank_plan_create(_cfg(abi, G=48), 0)
+    assert e.value.status == abi.ECHO_ERR_UNSUPPORTED
+    with pytest.raises(abi.EchoError) as e:
+        abi.echo_rank_exchange_bytes(_cfg(abi, N=100))
+    assert e.value.status == abi.ECHO_ERR_SHAPE
+    L = abi.lib
+    assert L.echo_rank_entry(None, None, None, None, None) == abi.ECHO_ERR_INVALID_ARG
+    assert L.echo_rank_reduce(None, None, None, None, None, None, None) == \
+        abi.ECHO_ERR_INVALID_ARG
+    assert L.echo_rank_exit(None, None, None, None, None) == abi.ECHO_ERR_INVALID_ARG
+    assert L.echo_rank_plan_destroy(None) == abi.ECHO_OK
+    assert L.echo_rank_launches_per_call(None) == 0
+
+
 def test_bench_byte_counts():
     import bench
     # 1 GiB per rank, P=8, G=128: 95.33 GB with the compensator, 22.31 GB off

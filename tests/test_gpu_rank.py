@@ -1,0 +1,183 @@
+"""The rank path (include/echo_rank.h): P rank plans on one GPU, driven in
+lockstep with the exchanges done by copies, against the oracle and against
+the plan of P virtual ranks, call by call, bit for bit -- outputs, the
+packed codes and scales on both wires, and every rank's two EMA states."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_error_compensated_echo_b200 import abi
+from bit_error_compensated_echo_b200 import workloads as W
+from bit_error_compensated_echo_b200.api import EchoPlan
+from bit_error_compensated_echo_b200.rank import EchoRankPlan
+from parity import _bits_u16, _f32, assert_same
+from rank_emulation import EmulatedGroup
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _same(name, a: torch.Tensor, b: torch.Tensor, call: int):
+    a, b = a.contiguous().cpu(), b.contiguous().cpu()
+    if a.dtype == torch.bfloat16:
+        assert_same(name, _bits_u16(a), _bits_u16(b), "bf16", call)
+    elif a.dtype == torch.float32:
+        assert_same(name, _f32(a), _f32(b), "f32", call)
+    else:
+        assert_same(name, a.numpy(), b.numpy(), "u8", call)
+
+
+def _compare_wires(grp: EmulatedGroup, plan: EchoPlan, call: int):
+    """Rank r's send buffers are row r of the virtual entry transport;
+    the gathered reduced chunks are the virtual reduced transport."""
+    dv = plan.debug_view()
+    for r, p in enumerate(grp.plans):
+        _same("send codes r%d" % r, p.bufs.send_codes, dv["codes"][r], call)
+        _same("send scales r%d" % r, p.bufs.send_scales, dv["scales"][r], call)
+        _same("gathered codes r%d" % r, p.bufs.all_codes, dv["rcodes"], call)
+        _same("gathered scales r%d" % r, p.bufs.all_scales, dv["rscales"], call)
+
+
+CASES = [  # P, G, groups per chunk, bits
+    (1, 32, 5, 4), (2, 32, 64, 4), (3, 64, 7, 4), (4, 128, 3, 4), (5, 32, 11, 4),
+    (8, 128, 16, 4), (8, 32, 1, 4), (2, 64, 9, 8), (4, 32, 13, 8), (8, 128, 4, 8)]
+
+
+@pytest.mark.parametrize("P,G,k,bits", CASES, ids=lambda v: str(v))
+@pytest.mark.parametrize("comp,fixup", [(True, "exit"), (True, "side"), (True, "deferred"),
+                                        (False, "deferred")])
+def test_rank_group_equals_virtual_plan(P, G, k, bits, comp, fixup):
+    N = P * G * k
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    side = torch.cuda.Stream() if fixup == "side" else None
+    kw = dict(compensate=comp, fixup=fixup, bits=bits)
+    with EmulatedGroup(P, N, G, **kw) as grp, EchoPlan(P, N, G, device=0, **kw) as plan:
+        for t in range(4):
+            x = W.generate(w, t, DEV)
+            y_rank = grp.allreduce(x, side_stream=side)
+            y_virt = plan.allreduce(x, side_stream=side)
+            torch.cuda.synchronize()
+            _same("outputs", y_rank, y_virt, t)
+            _compare_wires(grp, plan, t)
+            if comp:
+                mf_r, ms_r = grp.get_state()
+                mf_v, ms_v = plan.get_state()
+                _same("m_fast", mf_r, mf_v, t)
+                _same("m_slow", ms_r, ms_v, t)
+
+
+@pytest.mark.parametrize("fixup", ["exit", "side", "deferred"])
+def test_rank_group_against_oracle(fixup):
+    """The tiny workload's 16-call sequence, every rank against the oracle."""
+    w = W.TINY
+    side = torch.cuda.Stream() if fixup == "side" else None
+    prm = oracle.Params(P=w.P, N=w.N, G=w.G, compensate=True)
+    mf = np.zeros((w.P, w.N), np.float32)
+    ms = np.zeros((w.P, w.N), np.float32)
+    with EmulatedGroup(w.P, w.N, w.G, fixup=fixup) as grp:
+        for t in range(w.calls):
+            x = W.generate(w, t, DEV)
+            y = grp.allreduce(x, side_stream=side)
+            torch.cuda.synchronize()
+            ref = oracle.allreduce(prm, _bits_u16(x), mf, ms)
+            yb = _bits_u16(y)
+            assert_same("outputs", yb, np.broadcast_to(ref.y, yb.shape), "bf16", t)
+            for r, p in enumerate(grp.plans):
+                assert_same("send codes r%d" % r, p.bufs.send_codes.cpu().numpy(), ref.codes[r],
+                            "u8", t)
+                assert_same("gathered codes r%d" % r, p.bufs.all_codes.cpu().numpy(),
+                            ref.rcodes, "u8", t)
+            gmf, gms = grp.get_state()
+            assert_same("m_fast", _f32(gmf), mf, "f32", t)
+            assert_same("m_slow", _f32(gms), ms, "f32", t)
+
+
+@pytest.mark.parametrize("fixup", ["exit", "side", "deferred"])
+@pytest.mark.parametrize("P,G,k,bits", [(2, 32, 8, 4), (4, 64, 5, 4), (8, 128, 3, 4),
+                                        (4, 32, 6, 8)], ids=lambda v: str(v))
+def test_rank_reduce_scatter_equals_virtual_plan(P, G, k, bits, fixup):
+    N = P * G * k
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    side = torch.cuda.Stream() if fixup == "side" else None
+    kw = dict(fixup=fixup, bits=bits)
+    with EmulatedGroup(P, N, G, **kw) as grp, EchoPlan(P, N, G, device=0, **kw) as plan:
+        for t, op in enumerate("RRARAR"):
+            x = W.generate(w, t, DEV)
+            if op == "R":
+                a, b = grp.reduce_scatter(x, side_stream=side), plan.reduce_scatter(
+                    x, side_stream=side)
+            else:
+                a, b = grp.allreduce(x, side_stream=side), plan.allreduce(x, side_stream=side)
+            torch.cuda.synchronize()
+            _same("outputs (%s)" % op, a, b, t)
+            mf_r, ms_r = grp.get_state()
+            mf_v, ms_v = plan.get_state()
+            _same("m_fast", mf_r, mf_v, t)
+            _same("m_slow", ms_r, ms_v, t)
+
+
+def test_rank_llama_shape_equals_virtual_plan():
+    """P=8, 2048 x 4096 bf16 per rank, G=128, deferred fix-up: 6 calls."""
+    w = W.LLAMA
+    with EmulatedGroup(w.P, w.N, w.G, fixup="deferred") as grp, \
+            EchoPlan(w.P, w.N, w.G, device=0, fixup="deferred") as plan:
+        for t in range(6):
+            x = W.generate(w, t, DEV)
+            y_rank = grp.allreduce(x)
+            y_virt = plan.allreduce(x)
+            torch.cuda.synchronize()
+            assert torch.equal(y_rank.view(torch.int16), y_virt.view(torch.int16)), t
+        mf_r, ms_r = grp.get_state()
+        mf_v, ms_v = plan.get_state()
+        assert torch.equal(mf_r.view(torch.int32), mf_v.view(torch.int32))
+        assert torch.equal(ms_r.view(torch.int32), ms_v.view(torch.int32))
+
+
+def test_rank_state_calls():
+    """set_state / get_state / reset_state of a rank plan, with a pending
+    deferred fix-up, agree with the virtual plan's."""
+    P, G, N = 4, 64, 4 * 64 * 6
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    g = torch.Generator(device=DEV).manual_seed(7)
+    mf0 = torch.randn((P, N), generator=g, device=DEV) * 0.01
+    ms0 = torch.randn((P, N), generator=g, device=DEV) * 0.01
+    with EmulatedGroup(P, N, G, fixup="deferred") as grp, \
+            EchoPlan(P, N, G, device=0, fixup="deferred") as plan:
+        for r, p in enumerate(grp.plans):
+            p.set_state(mf0[r].contiguous(), ms0[r].contiguous())
+        plan.set_state(mf0.contiguous(), ms0.contiguous())
+        for t in range(3):
+            x = W.generate(w, t, DEV)
+            _same("outputs", grp.allreduce(x), plan.allreduce(x), t)
+            for a, b in zip(grp.get_state(), plan.get_state()):
+                _same("state", a, b, t)
+        for p in grp.plans:
+            p.reset_state()
+        plan.reset_state()
+        x = W.generate(w, 9, DEV)
+        _same("outputs after reset", grp.allreduce(x), plan.allreduce(x), 9)
+
+
+def test_rank_stage_order_and_arguments():
+    P, G, N = 2, 32, 2 * 32 * 4
+    with EchoRankPlan(P, 1, N, G, device=0, fixup="exit") as p:
+        with pytest.raises(abi.EchoError) as e:
+            p.reduce()                         # no entry yet
+        assert e.value.status == abi.ECHO_ERR_INVALID_ARG
+        x = torch.zeros(N, dtype=torch.bfloat16, device=DEV)
+        p.entry(x)
+        p.reduce()
+        with pytest.raises(abi.EchoError):
+            p.reduce()                         # a second reduce needs a new entry
+        with pytest.raises(abi.EchoError) as e:
+            abi.echo_rank_entry(p.handle, x.data_ptr() + 2, p.bufs.send_codes.data_ptr(),
+                                p.bufs.send_scales.data_ptr())
+        assert e.value.status == abi.ECHO_ERR_ALIGNMENT
+        assert p.launches_per_call() == 4
+    cfg = abi.echo_config_default()
+    cfg.P, cfg.N, cfg.G = P, N, G
+    with pytest.raises(abi.EchoError) as e:
+        abi.echo_rank_plan_create(cfg, 2)      # rank outside the group
+    assert e.value.status == abi.ECHO_ERR_INVALID_ARG

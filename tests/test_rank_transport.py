@@ -1,0 +1,183 @@
+"""The rank path's exchanges on the CPU, with gloo ranks (2 and 3 processes).
+
+1. The transport: after ``exchange`` and ``gather`` over torch.distributed,
+   every rank's receive buffers hold what the layout of include/echo_rank.h
+   says (part r of recv = rank r's send part o at rank o; part o of all =
+   owner o's reduced chunk), compared with the lockstep copies the GPU
+   tests use for their single-process group.
+2. The orchestration: ``EchoRankPlan.allreduce`` and ``reduce_scatter``
+   with the library stages replaced by byte-level stand-ins (no CUDA) put
+   the exchanges between the right stages: the stand-ins make the call an
+   exact all-reduce of bytes modulo 256, which the test checks.
+"""
+import os
+import socket
+
+import pytest
+import torch
+
+from bit_error_compensated_echo_b200.rank import (EchoRankPlan, ExchangeBuffers,
+                                                  TorchDistTransport, exchange, gather)
+
+CB, CS = 48, 3          # code bytes and scales per chunk in these tests
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _send_for(rank, P):
+    g = torch.Generator().manual_seed(1000 + rank)
+    codes = torch.randint(0, 256, (P * CB,), generator=g, dtype=torch.uint8)
+    scales = torch.randn(P * CS, generator=g)
+    red_codes = torch.randint(0, 256, (CB,), generator=g, dtype=torch.uint8)
+    red_scales = torch.randn(CS, generator=g)
+    return codes, scales, red_codes, red_scales
+
+
+def _transport_main(rank, ws, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        b = ExchangeBuffers(ws, CB, 4 * CS, "cpu")
+        codes, scales, rc, rs = _send_for(rank, ws)
+        b.send_codes.copy_(codes)
+        b.send_scales.copy_(scales)
+        b.red_codes.copy_(rc)
+        b.red_scales.copy_(rs)
+        t = TorchDistTransport()
+        exchange(b, t)
+        gather(b, t)
+        q.put((rank, b.recv_codes.clone(), b.recv_scales.clone(), b.all_codes.clone(),
+               b.all_scales.clone()))
+    finally:
+        dist.destroy_process_group()
+
+
+class _Bufs:
+    """Stand-in for a rank plan, holding only exchange buffers, for the
+    lockstep copies of tests/rank_emulation.py."""
+
+    def __init__(self, b):
+        self.bufs = b
+
+
+@pytest.mark.parametrize("ws", [2, 3])
+def test_transport_matches_the_buffer_layout(ws):
+    import torch.multiprocessing as mp
+
+    import rank_emulation
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_transport_main, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(ws):
+        r, *bufs = q.get(timeout=120)
+        got[r] = bufs
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+
+    # the same exchanges as lockstep copies
+    emul = []
+    for r in range(ws):
+        b = ExchangeBuffers(ws, CB, 4 * CS, "cpu")
+        codes, scales, rc, rs = _send_for(r, ws)
+        b.send_codes.copy_(codes)
+        b.send_scales.copy_(scales)
+        b.red_codes.copy_(rc)
+        b.red_scales.copy_(rs)
+        emul.append(_Bufs(b))
+    rank_emulation.all_to_all(emul)
+    rank_emulation.all_gather(emul)
+    for r in range(ws):
+        want = emul[r].bufs
+        for g, w in zip(got[r], (want.recv_codes, want.recv_scales, want.all_codes,
+                                 want.all_scales)):
+            assert torch.equal(g, w), r
+    # and spelled out for one part: rank 1's part 0 of recv is rank 0's part 1 of send
+    assert torch.equal(got[1][0][:CB], _send_for(0, ws)[0][CB:2 * CB])
+
+
+class ByteStagePlan(EchoRankPlan):
+    """EchoRankPlan whose stages are byte-level stand-ins on CPU buffers:
+    entry copies chunk o of x (uint8) into send part o; reduce sums the P
+    received parts modulo 256; exit concatenates the gathered parts.  The
+    scales carry the rank index through the same exchanges."""
+
+    def __init__(self, P, rank, C):
+        self.P, self.rank, self.N = P, rank, P * C
+        self.bufs = ExchangeBuffers(P, C, 4, "cpu")
+        self.handle = None
+
+    def entry(self, x, stream=None):
+        self.bufs.send_codes.copy_(x)
+        self.bufs.send_scales.fill_(float(self.rank))
+
+    def reduce(self, stream=None, side_stream=None):
+        b = self.bufs
+        parts = b.recv_codes.view(self.P, b.cb).to(torch.int64)
+        b.red_codes.copy_((parts.sum(0) % 256).to(torch.uint8))
+        b.red_scales.copy_(b.recv_scales.sum().reshape(1))
+
+    def exit(self, out, stream=None):
+        out.copy_(self.bufs.all_codes)
+
+    def reduce_scatter_finish(self, out, stream=None, side_stream=None):
+        parts = self.bufs.recv_codes.view(self.P, self.bufs.cb).to(torch.int64)
+        out.copy_((parts.sum(0) % 256).to(torch.uint8))
+
+
+def _x_for(rank, N):
+    g = torch.Generator().manual_seed(77 + rank)
+    return torch.randint(0, 256, (N,), generator=g, dtype=torch.uint8)
+
+
+def _orchestration_main(rank, ws, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        C = 40
+        plan = ByteStagePlan(ws, rank, C)
+        x = _x_for(rank, ws * C)
+        y = plan.allreduce(x, TorchDistTransport(), out=torch.empty(ws * C, dtype=torch.uint8))
+        scales = plan.bufs.all_scales.clone()
+        z = plan.reduce_scatter(x, TorchDistTransport(), out=torch.empty(C, dtype=torch.uint8))
+        q.put((rank, y, scales, z))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("ws", [2, 3])
+def test_allreduce_orchestration_with_byte_stages(ws):
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_orchestration_main, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(ws):
+        r, y, scales, z = q.get(timeout=120)
+        got[r] = (y, scales, z)
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    C = 40
+    total = sum(_x_for(r, ws * C).to(torch.int64) for r in range(ws)) % 256
+    rank_sum = float(sum(range(ws)))
+    for r in range(ws):
+        y, scales, z = got[r]
+        assert torch.equal(y.to(torch.int64), total), r
+        assert torch.equal(scales, torch.full((ws,), rank_sum)), r
+        assert torch.equal(z.to(torch.int64), total[r * C:(r + 1) * C]), r
