@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload large|llama|depth|tiny] [--fixup exit|side|deferred]
-                    [--uncompensated] [--mode step|sweep|overlap|depth-chain]
+                    [--uncompensated] [--mode step|sweep|overlap|depth-chain|group]
 
 Default (mode "step"): one step = one echo_allreduce call (entry + reduce +
 exit kernels) of P=8 virtual ranks x 2^29 bf16 elements (1 GiB) per rank,
@@ -18,6 +18,12 @@ during the timed region.
 With --gpus N under torchrun every rank runs its own independent call on
 its own GPU (the path is emulated on one GPU; there is no cross-GPU data
 exchange), timed between barriers and reported as the max over ranks.
+
+--mode group runs the rank path instead: the N processes of the torchrun
+form ONE Echo group (P = N real ranks, one GPU each, the workload's N
+elements per rank), the two exchanges go over NCCL, and the line compares
+the call with NCCL's bf16 all-reduce of the same tensors (max over ranks of
+CUDA-event times).  With one GPU it runs a one-rank group.
 
 --impl reference times the CPU oracle on bounded samples of the same
 workload (rank 0 only) and prints the same JSON line with "impl":
@@ -584,6 +590,85 @@ def run_overlap_mode(args, ws, rank, local):
     print(json.dumps(res), flush=True)
 
 
+def run_group_mode(args, ws, rank, local):
+    """The rank path over NCCL: this process is rank ``rank`` of a group of
+    ws ranks; per step one EchoRankPlan.allreduce (entry, all-to-all of the
+    packed chunks, reduce, all-gather, exit), timed with CUDA events between
+    barriers, max over ranks; then NCCL's bf16 all-reduce of the same input,
+    timed the same way."""
+    import torch.distributed as dist
+
+    from bit_error_compensated_echo_b200.rank import EchoRankPlan, TorchDistTransport
+    if ws == 1 and not dist.is_initialized():
+        import datetime
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(29500 + (os.getpid() % 1000)))
+        dist.init_process_group("nccl", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    comp = not args.uncompensated
+    P, N, G = ws, w.N, w.G
+    if N % (P * G):
+        raise SystemExit("N=%d is not a multiple of P*G=%d" % (N, P * G))
+    one = W.with_size(w, P=1)
+    x = W.generate(one, rank, dev)[0].contiguous()
+    out = torch.empty_like(x)
+    plan = EchoRankPlan(P, rank, N, G, compensate=comp, fixup=args.fixup, device=local,
+                        bits=args.bits)
+    transport = TorchDistTransport()
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, steps):
+        times = []
+        for _ in range(steps):
+            dist.barrier()
+            torch.cuda.synchronize(dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            times.append(e0.elapsed_time(e1))
+        return times
+
+    echo_fn = lambda: plan.allreduce(x, transport, out=out)  # noqa: E731
+    y = x.clone()
+    nccl_fn = lambda: dist.all_reduce(y)  # noqa: E731
+    timed(echo_fn, max(args.warmup, 3))
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    t_echo = timed(echo_fn, args.steps)
+    clocks = sampler.stop() if sampler else None
+    timed(nccl_fn, max(args.warmup, 3))
+    t_nccl = timed(nccl_fn, args.steps)
+    ms_echo = max_over_ranks(statistics.median(t_echo), ws, dev)
+    ms_nccl = max_over_ranks(statistics.median(t_nccl), ws, dev)
+    wire = plan.bufs.wire_bytes()
+    if rank == 0:
+        line = {
+            "mode": "group", "metric": "Echo all-reduce over NCCL: input GB/s (P ranks x N bf16 "
+            "/ call time), against NCCL's bf16 all-reduce", "unit": UNIT,
+            "value": round(2.0 * P * N / (ms_echo / 1e3) / 1e9, 3), "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_call": round(ms_echo, 4),
+            "nccl_bf16_allreduce_ms": round(ms_nccl, 4),
+            "speedup_vs_nccl_bf16": round(ms_nccl / ms_echo, 3),
+            "wire_bytes_per_rank": wire, "bf16_ring_wire_bytes_per_rank": 2 * (P - 1) * N * 2 // P,
+            "higher_is_better": True, "scaling": "weak", "data": "synthetic",
+            "config": {"workload": w.name, "P": P, "N_per_rank": N, "G": G, "bits": args.bits,
+                       "compensate": comp, "fixup": args.fixup,
+                       "transport": "torch.distributed NCCL all_to_all_single + "
+                       "all_gather_into_tensor"},
+            "gpu_launches_per_call": plan.launches_per_call(), "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if ws == 1:
+        dist.destroy_process_group()
+
+
 def run_depth_chain_mode(args, ws, rank, local):
     """Deviation from the exact fp32 chain per site, forward and backward."""
     from bit_error_compensated_echo_b200 import depth_chain
@@ -612,7 +697,8 @@ def main(argv=None):
     ap.add_argument("--uncompensated", action="store_true")
     ap.add_argument("--op", choices=("all-reduce", "reduce-scatter"), default="all-reduce")
     ap.add_argument("--bits", type=int, choices=(4, 8), default=4)
-    ap.add_argument("--mode", choices=("step", "depth-chain", "sweep", "overlap"), default="step")
+    ap.add_argument("--mode", choices=("step", "depth-chain", "sweep", "overlap", "group"),
+                    default="step")
     ap.add_argument("--sweep-max-mib", type=int, default=0,
                     help="sweep only points up to this many MiB per rank (0: all)")
     ap.add_argument("--sweep-table", default="", help="also write the sweep as a markdown table")
@@ -637,6 +723,8 @@ def main(argv=None):
             run_sweep_mode(args, ws, rank, local)
         elif args.mode == "overlap":
             run_overlap_mode(args, ws, rank, local)
+        elif args.mode == "group":
+            run_group_mode(args, ws, rank, local)
         else:
             run_step_mode(args, ws, rank, local)
     finally:
