@@ -50,7 +50,8 @@ class echo_debug_view(ctypes.Structure):
     _fields_ = [("m_fast", ctypes.c_void_p), ("m_slow", ctypes.c_void_p),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("rcodes", ctypes.c_void_p), ("rscales", ctypes.c_void_p),
-                ("e_req", ctypes.c_void_p), ("fixup_pending", ctypes.c_int32)]
+                ("e_req", ctypes.c_void_p), ("fixup_pending", ctypes.c_int32),
+                ("bits", ctypes.c_int32)]
 
 
 class echo_profile(ctypes.Structure):
@@ -82,6 +83,7 @@ def _load():
         "echo_profile_enable": (st, [vp, ctypes.c_int32]),
         "echo_profile_read": (st, [vp, ctypes.POINTER(echo_profile), ctypes.c_int32]),
         "echo_launches_per_call": (ctypes.c_int32, [vp]),
+        "echo_plan_set_bits": (st, [vp, ctypes.c_int32]),
         "echo_status_string": (ctypes.c_char_p, [st]),
         "echo_abi_version": (ctypes.c_int32, []),
         "echo_allreduce_noalloc": (st, [ctypes.POINTER(echo_config), ctypes.POINTER(vp),
@@ -102,6 +104,7 @@ def _load():
         "echo_rank_get_state": (st, [vp, vp, vp, vp]),
         "echo_rank_set_state": (st, [vp, vp, vp, vp]),
         "echo_rank_launches_per_call": (ctypes.c_int32, [vp]),
+        "echo_rank_plan_set_bits": (st, [vp, ctypes.c_int32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -191,6 +194,10 @@ def echo_profile_read(plan: int, reset: bool = False) -> echo_profile:
     p = echo_profile()
     _check(lib.echo_profile_read(plan, ctypes.byref(p), int(bool(reset))), "echo_profile_read")
     return p
+
+
+def echo_plan_set_bits(plan: int, bits: int) -> None:
+    _check(lib.echo_plan_set_bits(plan, int(bits)), "echo_plan_set_bits")
 
 
 def echo_launches_per_call(plan: int) -> int:
@@ -289,3 +296,7 @@ def echo_rank_set_state(plan: int, m_fast_device: int, m_slow_device: int,
 
 def echo_rank_launches_per_call(plan: int) -> int:
     return int(lib.echo_rank_launches_per_call(plan))
+
+
+def echo_rank_plan_set_bits(plan: int, bits: int) -> None:
+    _check(lib.echo_rank_plan_set_bits(plan, int(bits)), "echo_rank_plan_set_bits")

@@ -56,7 +56,8 @@ class EchoPlan:
             device = torch.cuda.current_device()
         cfg = make_config(P, N, G, compensate, alpha, beta_fast, beta_slow, device, fixup, bits)
         self.cfg = cfg
-        self.bits = int(bits)
+        self.max_bits = int(bits)   # the transport is sized for this width
+        self.bits = int(bits)       # width of the following calls
         self.P, self.N, self.G = int(P), int(N), int(G)
         self.compensate = bool(compensate)
         self.fixup = fixup
@@ -96,11 +97,23 @@ class EchoPlan:
         return xs
 
     # ------------------------------------------------------------ calls
+    def set_bits(self, bits: int) -> None:
+        """Code width of the following calls (4, or 8 if the plan was made
+        with bits=8); every width shares the plan's one state."""
+        abi.echo_plan_set_bits(self.handle, bits)
+        self.bits = int(bits)
+
+    def _width(self, bits: Optional[int]) -> None:
+        if bits is not None and int(bits) != self.bits:
+            self.set_bits(bits)
+
     def allreduce(self, xs, out=None, stream: Optional[torch.cuda.Stream] = None,
-                  side_stream: Optional[torch.cuda.Stream] = None):
+                  side_stream: Optional[torch.cuda.Stream] = None, bits: Optional[int] = None):
         """One call.  xs: [P, N] bf16 tensor or P tensors on the plan's
         device.  out: same form (allocated if None; may be xs for in place).
+        bits: code width of this call and the following ones (None: keep).
         Returns out."""
+        self._width(bits)
         xs_l = self._rank_tensors(xs, "inputs")
         if out is None:
             out = torch.empty((self.P, self.N), dtype=torch.bfloat16, device=self.device)
@@ -115,10 +128,12 @@ class EchoPlan:
         return out
 
     def reduce_scatter(self, xs, out=None, stream: Optional[torch.cuda.Stream] = None,
-                       side_stream: Optional[torch.cuda.Stream] = None):
+                       side_stream: Optional[torch.cuda.Stream] = None,
+                       bits: Optional[int] = None):
         """One reduce-scatter call.  xs: [P, N] bf16 (or P tensors); out:
         [P, N/P] bf16 (allocated if None), row r = rank r's own chunk of the
         sum.  Returns out."""
+        self._width(bits)
         xs_l = self._rank_tensors(xs, "inputs")
         C = self.N // self.P
         if out is None:
@@ -137,9 +152,11 @@ class EchoPlan:
                                 _stream_handle(stream, self.device), side)
         return out
 
-    def allreduce_host(self, xs_host, out_host=None, stream: Optional[torch.cuda.Stream] = None):
+    def allreduce_host(self, xs_host, out_host=None, stream: Optional[torch.cuda.Stream] = None,
+                       bits: Optional[int] = None):
         """The same call on host tensors (pinned for asynchronous copies);
         the caller synchronizes the stream before reading out_host."""
+        self._width(bits)
         xs_l = self._rank_tensors(xs_host, "host inputs")
         if out_host is None:
             out_host = torch.empty((self.P, self.N), dtype=torch.bfloat16, pin_memory=True)
@@ -175,7 +192,7 @@ class EchoPlan:
         """Zero-copy tensors over the plan's workspace (valid while the plan
         lives; contents as left by the last call)."""
         v = abi.echo_debug_view_get(self.handle)
-        P, N, G = self.P, self.N, self.G
+        P, N, G, bits = self.P, self.N, self.G, v.bits
 
         def t(ptr, shape, typestr):
             if not ptr:
@@ -184,9 +201,9 @@ class EchoPlan:
 
         return {
             "m_fast": t(v.m_fast, (P, N), "<f4"), "m_slow": t(v.m_slow, (P, N), "<f4"),
-            "codes": t(v.codes, (P, N * self.bits // 8), "|u1"),
+            "codes": t(v.codes, (P, N * bits // 8), "|u1"),
             "scales": t(v.scales, (P, N // G), "<f4"),
-            "rcodes": t(v.rcodes, (N * self.bits // 8,), "|u1"),
+            "rcodes": t(v.rcodes, (N * bits // 8,), "|u1"),
             "rscales": t(v.rscales, (N // G,), "<f4"),
             "e_req": t(v.e_req, (N,), "<f4"), "fixup_pending": bool(v.fixup_pending),
         }

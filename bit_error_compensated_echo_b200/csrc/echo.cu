@@ -527,6 +527,14 @@ echo_status echo_debug_view_get(echo_plan *p, echo_debug_view *v) {
     v->rscales = p->rscales;
     v->e_req = p->e_req;
     v->fixup_pending = p->pending ? 1 : 0;
+    v->bits = p->b.bits;
+    return ECHO_OK;
+}
+
+echo_status echo_plan_set_bits(echo_plan *p, int32_t bits) {
+    if (!p) return ECHO_ERR_INVALID_ARG;
+    if ((bits != 4 && bits != 8) || bits > p->cfg.bits) return ECHO_ERR_UNSUPPORTED;
+    p->b.bits = bits;
     return ECHO_OK;
 }
 

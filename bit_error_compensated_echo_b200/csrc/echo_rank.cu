@@ -27,6 +27,7 @@ using namespace echo;
 
 struct echo_rank_plan {
     echo_config cfg;
+    int bits = 4;                     // code width of the calls
     int rank = 0;
     int64_t C = 0;                    // elements per chunk
     int64_t n_vec = 0, chunk_vec = 0; // vectors per row and per chunk
@@ -54,7 +55,7 @@ Bufs base_bufs(const echo_rank_plan *p) {
     Bufs b;
     b.P = p->cfg.P;
     b.G = p->cfg.G;
-    b.bits = p->cfg.bits;
+    b.bits = p->bits;
     b.comp = p->cfg.compensate != 0;
     b.k = p->k;
     b.e_req = p->e_req;
@@ -145,6 +146,7 @@ echo_status echo_rank_plan_create(echo_rank_plan **out, const echo_config *cfg, 
     if (!p) return ECHO_ERR_OOM;
     p->cfg = *cfg;
     p->rank = rank;
+    p->bits = cfg->bits;
     p->C = cfg->N / cfg->P;
     p->n_vec = cfg->N / kVec;
     p->chunk_vec = p->n_vec / cfg->P;
@@ -331,6 +333,13 @@ echo_status echo_rank_set_state(echo_rank_plan *p, const float *m_fast, const fl
     ECHO_TRY(cudaMemcpyAsync(p->m_slow, m_slow, bytes, cudaMemcpyDeviceToDevice, st));
     p->pending = false;
     p->entered = false;
+    return ECHO_OK;
+}
+
+echo_status echo_rank_plan_set_bits(echo_rank_plan *p, int32_t bits) {
+    if (!p) return ECHO_ERR_INVALID_ARG;
+    if ((bits != 4 && bits != 8) || bits > p->cfg.bits) return ECHO_ERR_UNSUPPORTED;
+    p->bits = bits;
     return ECHO_OK;
 }
 

@@ -14,10 +14,13 @@ by the all-reduce of the P ranks' partial products:
 with W_l Haar-orthogonal (QR of a Gaussian, signs fixed, seeded 1000 + l),
 B_r the r-th block of hidden/P features, RMSNorm with unit weight and
 eps = 1e-6, everything else in fp32.  Orthogonal maps and RMSNorm do not
-amplify perturbations, which is the bound's assumption.  Four chains run
+amplify perturbations, which is the bound's assumption.  Five chains run
 side by side: the exact chain (fp32 partials summed in fp32), the
-compensated 4-bit all-reduce, the uncompensated one, and a bf16 all-reduce
-(bf16 partials summed in fp32, rounded to bf16).  Per site it reports the
+compensated 4-bit all-reduce, the uncompensated one, a bf16 all-reduce
+(bf16 partials summed in fp32, rounded to bf16), and "promoted": the
+compensated all-reduce under the pages' serving policy, the first half of
+the layers (two sites each) at 8-bit codes and the rest at 4 bits, on one
+state (ai4snews news summary, "Perspective").  Per site it reports the
 absolute RMS deviation from the exact chain and the relative Frobenius
 deviation.
 
@@ -34,6 +37,7 @@ import torch
 
 from . import workloads as W
 from .api import EchoPlan
+from .policy import LayerPolicy
 
 EPS = 1e-6
 
@@ -74,7 +78,7 @@ class _Chain:
         self.name, self.h, self.plan = name, h0.clone(), plan
 
 
-def _ar(kind: str, parts32: torch.Tensor, plan, buf_bf16, out_bf16) -> torch.Tensor:
+def _ar(kind: str, parts32: torch.Tensor, plan, buf_bf16, out_bf16, bits=None) -> torch.Tensor:
     """The site's all-reduce of the P partials ([P, T, D] fp32) -> [T, D] fp32."""
     if kind == "exact":
         return parts32.sum(dim=0)
@@ -82,7 +86,7 @@ def _ar(kind: str, parts32: torch.Tensor, plan, buf_bf16, out_bf16) -> torch.Ten
     if kind == "bf16":
         return buf_bf16.float().sum(dim=0).to(torch.bfloat16).float()
     P = parts32.shape[0]
-    plan.allreduce(buf_bf16.view(P, -1), out=out_bf16.view(P, -1))
+    plan.allreduce(buf_bf16.view(P, -1), out=out_bf16.view(P, -1), bits=bits)
     return out_bf16[0].float()
 
 
@@ -103,23 +107,31 @@ def run(P: int = 8, tokens: int = 32768, hidden: int = 1024, sites: int = 56, G:
     buf = torch.empty((P, tokens, hidden), dtype=torch.bfloat16, device=dev)
     out = torch.empty_like(buf)
     res: Dict[str, Dict[str, List[float]]] = {}
+    policy = LayerPolicy(max(1, sites // 2), 2, 0.5)
 
     def one_pass(direction: str, start: torch.Tensor, ws, h_exact_fwd=None):
-        plans = {"comp": EchoPlan(P, N, G, compensate=True, device=dev.index or 0, fixup="deferred"),
-                 "off": EchoPlan(P, N, G, compensate=False, device=dev.index or 0)}
+        d = dev.index or 0
+        plans = {"comp": EchoPlan(P, N, G, compensate=True, device=d, fixup="deferred"),
+                 "off": EchoPlan(P, N, G, compensate=False, device=d),
+                 "promoted": EchoPlan(P, N, G, compensate=True, device=d, fixup="deferred",
+                                      bits=8)}
         chains = [_Chain("exact", start), _Chain("comp", start, plans["comp"]),
-                  _Chain("off", start, plans["off"]), _Chain("bf16", start)]
+                  _Chain("off", start, plans["off"]), _Chain("bf16", start),
+                  _Chain("promoted", start, plans["promoted"])]
         rms = {c.name: [] for c in chains if c.name != "exact"}
         rel = {c.name: [] for c in chains if c.name != "exact"}
         try:
             for step, wmat in enumerate(ws):
+                # the site's position in the forward order sets its layer's width
+                site = step if direction == "forward" else len(ws) - 1 - step
                 for c in chains:
+                    bits = policy.bits_for_site(site) if c.name == "promoted" else None
                     if direction == "forward":
                         partials(rmsnorm(c.h), wmat, P, parts)
-                        c.h = c.h + _ar(c.name, parts, c.plan, buf, out)
+                        c.h = c.h + _ar(c.name, parts, c.plan, buf, out, bits)
                     else:
                         partials(c.h, wmat.t().contiguous(), P, parts)
-                        u = _ar(c.name, parts, c.plan, buf, out)
+                        u = _ar(c.name, parts, c.plan, buf, out, bits)
                         c.h = c.h + rmsnorm_jt(h_exact_fwd[len(ws) - 1 - step], u)
                 ref = chains[0].h
                 for c in chains[1:]:

@@ -52,20 +52,33 @@ class ExchangeBuffers:
       recv_codes [P*cb] u8, recv_scales [P*cs] f32 : rank r's copy of this chunk
       red_codes  [cb] u8,   red_scales  [cs] f32   : this rank's reduced chunk
       all_codes  [P*cb] u8, all_scales  [P*cs] f32 : owner o's reduced chunk
+
+    The code buffers are allocated for ``chunk_code_bytes`` (the widest
+    width) and viewed at the width in force (``set_code_bytes``).
     """
 
     def __init__(self, P: int, chunk_code_bytes: int, chunk_scale_bytes: int, device):
         cb, cs = int(chunk_code_bytes), int(chunk_scale_bytes) // 4
         u8, f32 = torch.uint8, torch.float32
-        self.P, self.cb, self.cs = int(P), cb, cs
-        self.send_codes = torch.empty(P * cb, dtype=u8, device=device)
+        self.P, self.cb_max, self.cs = int(P), cb, cs
+        self._codes = {k: torch.empty(P * cb if k != "red" else cb, dtype=u8, device=device)
+                       for k in ("send", "recv", "red", "all")}
         self.send_scales = torch.empty(P * cs, dtype=f32, device=device)
-        self.recv_codes = torch.empty(P * cb, dtype=u8, device=device)
         self.recv_scales = torch.empty(P * cs, dtype=f32, device=device)
-        self.red_codes = torch.empty(cb, dtype=u8, device=device)
         self.red_scales = torch.empty(cs, dtype=f32, device=device)
-        self.all_codes = torch.empty(P * cb, dtype=u8, device=device)
         self.all_scales = torch.empty(P * cs, dtype=f32, device=device)
+        self.set_code_bytes(cb)
+
+    def set_code_bytes(self, cb: int) -> None:
+        """View the code buffers for chunks of cb bytes (cb <= the allocated
+        size): chunk o then starts at o*cb."""
+        if cb > self.cb_max:
+            raise ValueError("chunk of %d code bytes exceeds the %d allocated" % (cb, self.cb_max))
+        P, self.cb = self.P, int(cb)
+        self.send_codes = self._codes["send"][:P * cb]
+        self.recv_codes = self._codes["recv"][:P * cb]
+        self.red_codes = self._codes["red"][:cb]
+        self.all_codes = self._codes["all"][:P * cb]
 
     def wire_bytes(self) -> int:
         """Bytes this rank sends per all-reduce: (P-1) chunks in the
@@ -103,6 +116,7 @@ class EchoRankPlan:
         self.cfg = make_config(P, N, G, compensate, alpha, beta_fast, beta_slow, device, fixup,
                                bits)
         self.P, self.rank, self.N, self.G, self.bits = int(P), int(rank), int(N), int(G), int(bits)
+        self.max_bits = int(bits)
         self.compensate = bool(compensate)
         self.fixup = fixup
         self.device = torch.device("cuda", int(device))
@@ -127,6 +141,14 @@ class EchoRankPlan:
 
     def __exit__(self, *exc):
         self.close()
+
+    def set_bits(self, bits: int) -> None:
+        """Code width of the following calls (4, or 8 if the plan was made
+        with bits=8), one state for every width.  Every rank of the group
+        must use the same width for a call."""
+        abi.echo_rank_plan_set_bits(self.handle, bits)
+        self.bits = int(bits)
+        self.bufs.set_code_bytes(self.N // self.P * self.bits // 8)
 
     # ------------------------------------------------------------ checks
     def _check_bf16(self, t: torch.Tensor, n: int, what: str) -> None:
@@ -174,9 +196,12 @@ class EchoRankPlan:
 
     # ------------------------------------------------------------ calls
     def allreduce(self, x: torch.Tensor, transport=None, out: Optional[torch.Tensor] = None,
-                  side_stream=None) -> torch.Tensor:
+                  side_stream=None, bits: Optional[int] = None) -> torch.Tensor:
         """One compensated all-reduce of this rank's x ([N] bf16) with the
-        other ranks of the group, on the current stream.  out may be x."""
+        other ranks of the group, on the current stream.  out may be x.
+        bits: code width of this call and the following ones (None: keep)."""
+        if bits is not None and int(bits) != self.bits:
+            self.set_bits(bits)
         transport = transport if transport is not None else TorchDistTransport()
         if out is None:
             out = torch.empty(self.N, dtype=torch.bfloat16, device=self.device)
@@ -188,9 +213,11 @@ class EchoRankPlan:
         return out
 
     def reduce_scatter(self, x: torch.Tensor, transport=None, out: Optional[torch.Tensor] = None,
-                       side_stream=None) -> torch.Tensor:
+                       side_stream=None, bits: Optional[int] = None) -> torch.Tensor:
         """The reduce-scatter of sequence parallelism: returns this rank's
         chunk (N/P bf16) of the sum."""
+        if bits is not None and int(bits) != self.bits:
+            self.set_bits(bits)
         transport = transport if transport is not None else TorchDistTransport()
         if out is None:
             out = torch.empty(self.N // self.P, dtype=torch.bfloat16, device=self.device)

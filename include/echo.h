@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define ECHO_ABI_VERSION 1
+#define ECHO_ABI_VERSION 2
 #define ECHO_MAX_RANKS 8
 
 typedef enum echo_status {
@@ -99,7 +99,11 @@ typedef struct echo_config {
     int32_t bits;       /* code width: 4 (levels -7..7, two codes per byte) or
                          * 8 (levels -127..127, one code per byte; the
                          * pages' serving policy promotes the first half of
-                         * the layers to 8 bits, ai4snews "Perspective") */
+                         * the layers to 8 bits, ai4snews "Perspective").
+                         * The widest width of the plan's calls: the
+                         * transport is sized for it, and a plan with
+                         * bits = 8 can run any call at 4 bits
+                         * (echo_plan_set_bits) on the same state. */
 } echo_config;
 
 typedef struct echo_plan echo_plan;
@@ -208,6 +212,7 @@ typedef struct echo_debug_view {
     float *rscales;     /* [N/G] requantization scales */
     float *e_req;       /* [N] requantization error, or NULL */
     int32_t fixup_pending; /* 1 if a deferred fix-up is pending */
+    int32_t bits;       /* code width of the calls (echo_plan_set_bits) */
 } echo_debug_view;
 
 echo_status echo_debug_view_get(echo_plan *plan, echo_debug_view *view);
@@ -227,6 +232,15 @@ typedef struct echo_profile {
 
 echo_status echo_profile_enable(echo_plan *plan, int32_t on);
 echo_status echo_profile_read(echo_plan *plan, echo_profile *out, int32_t reset);
+
+/* Code width of the plan's following calls: 4, or 8 when cfg.bits == 8
+ * (per-call promotion: the pages' serving policy runs the first half of the
+ * layers at 8 bits, ai4snews news summary, "Perspective").  Every width
+ * shares the plan's one compensator state and any pending fix-up: the
+ * state and e_req are fp32 whatever the width.  Takes effect for calls made
+ * after it; launches nothing.  A new plan runs at cfg.bits.
+ * Errors: INVALID_ARG (null), UNSUPPORTED (not 4 or 8, or above cfg.bits). */
+echo_status echo_plan_set_bits(echo_plan *plan, int32_t bits);
 
 /* Kernels launched by one echo_allreduce call with this plan. */
 int32_t echo_launches_per_call(const echo_plan *plan);

@@ -138,6 +138,13 @@ echo_status echo_rank_get_state(echo_rank_plan *plan, float *m_fast_device,
 echo_status echo_rank_set_state(echo_rank_plan *plan, const float *m_fast_device,
                                 const float *m_slow_device, void *stream);
 
+/* Code width of the following calls, as echo_plan_set_bits (4, or 8 when
+ * cfg.bits == 8; one state for every width).  The chunk sizes of the
+ * exchange buffers follow the width: cb = C*bits/8 with the width in force,
+ * so buffers sized for cfg.bits hold any call, at the offsets of that call's
+ * width.  Errors: INVALID_ARG (null), UNSUPPORTED. */
+echo_status echo_rank_plan_set_bits(echo_rank_plan *plan, int32_t bits);
+
 /* Kernels one all-reduce (entry + reduce + exit) launches with this plan:
  * 3, or 4 when the fix-up runs as its own kernel (EXIT and SIDE modes). */
 int32_t echo_rank_launches_per_call(const echo_rank_plan *plan);

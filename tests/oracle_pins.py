@@ -567,6 +567,50 @@ def pin_8bit_calls(o):
     assert np.abs(bits_to_f64(r8.y) - ex).mean() < 0.2 * np.abs(bits_to_f64(r4.y) - ex).mean()
 
 
+def pin_mixed_width_sequence(o):
+    """One state across calls of both code widths (the serving policy's
+    per-layer promotion): the telescoping identity and the EMA closed form
+    hold over the mixed sequence, and every call's transport is that of its
+    own width -- 8-bit calls reduce 8-bit grid-exact inputs exactly, 4-bit
+    calls the 4-bit ones."""
+    rng = np.random.default_rng(27)
+    P, G = 4, 32
+    N = P * G * 2
+    widths = [8, 8, 8, 8, 4, 4, 4, 4, 8, 4, 8, 4, 8, 8, 4, 4]
+    kw = DEFAULTS
+    bf = np.float64(np.float32(kw["beta_fast"]))
+    bs = np.float64(np.float32(kw["beta_slow"]))
+    a = np.float64(np.float32(kw["alpha"]))
+    own = _owner(_params(o, P, N, G, True), np.arange(N))
+    mf = np.zeros((P, N), np.float32)
+    ms = np.zeros((P, N), np.float32)
+    S = np.zeros(N)
+    X = np.zeros(N)
+    rhos = []
+    for t, bits in enumerate(widths, 1):
+        prm = _params(o, P, N, G, True, bits=bits, **kw)
+        x = _sequence_inputs(rng, P, N, 1)[0]
+        r = o.allreduce(prm, x, mf, ms)
+        assert r.codes.shape == (P, N * bits // 8) and (r.qcount == 2).all()
+        S += bits_to_f64(r.y)
+        X += bits_to_f64(x).sum(axis=0)
+        rhs = -(a * mf.astype(np.float64) / (1 - bf)
+                + (1 - a) * ms.astype(np.float64) / (1 - bs)).sum(axis=0)
+        assert (np.abs((S - X) - rhs) <= 64 * t * P * 2.0 ** -24 * (1 + np.abs(S))).all()
+        rho = r.e_in.astype(np.float64).copy()
+        rho[own, np.arange(N)] += r.e_req
+        rhos.append(rho)
+        cf = sum((1 - bf) * bf ** (t - 1 - k) * rhos[k] for k in range(t))
+        scale = np.abs(np.stack(rhos)).max() + 1e-30
+        assert np.allclose(mf, cf, rtol=1e-6, atol=1e-6 * scale)
+    for bits, L in ((8, 127), (4, 7)):
+        prm = _params(o, P, N, G, True, bits=bits)
+        x = bf16_bits(grid_exact_inputs(rng, P, N, G, L=L))
+        z = np.zeros((P, N), np.float32)
+        r = o.allreduce(prm, x, z, z.copy())
+        assert np.array_equal(bits_to_f64(r.y), bits_to_f64(x).sum(axis=0))
+
+
 # ---------------------------------------------------------------- reduce-scatter
 
 def _run_rs_sequence(o, prm, xs):

@@ -63,36 +63,53 @@ class SequenceChecker:
     def __init__(self, plan: EchoPlan, prm: oracle.Params, cols=None):
         self.plan, self.prm = plan, prm
         P, N, G = prm.P, prm.N, prm.G
-        cb = G * prm.bits // 8          # code bytes per group
         if cols is None:
             self.cols = None
             self.idx = np.arange(N)
-            self.cidx = np.arange(N // G * cb)
             self.gidx = np.arange(N // G)
         else:
             self.cols = np.asarray(cols, np.int64)
             self.idx = workloads.column_elements(self.cols, G)
-            self.cidx = workloads.column_elements(self.cols, cb)
             self.gidx = self.cols
         n = self.idx.size
         self.mf = np.zeros((P, n), np.float32)
         self.ms = np.zeros((P, n), np.float32)
         self.t_idx = torch.from_numpy(self.idx).to(plan.device)
-        self.t_cidx = torch.from_numpy(self.cidx).to(plan.device)
         self.t_gidx = torch.from_numpy(self.gidx).to(plan.device)
+        self._t_cidx = {}
         self.calls = 0
 
+    def cidx(self, bits: int) -> torch.Tensor:
+        """Byte indices of the sampled columns in a code row of this width."""
+        if bits not in self._t_cidx:
+            cb = self.prm.G * bits // 8          # code bytes per group
+            if self.cols is None:
+                c = np.arange(self.prm.N // self.prm.G * cb)
+            else:
+                c = workloads.column_elements(self.cols, cb)
+            self._t_cidx[bits] = torch.from_numpy(c).to(self.plan.device)
+        return self._t_cidx[bits]
+
+    def _prm(self) -> oracle.Params:
+        """The oracle's parameters for the plan's current code width."""
+        if self.prm.bits == self.plan.bits:
+            return self.prm
+        import dataclasses
+        return dataclasses.replace(self.prm, bits=self.plan.bits)
+
     def gather(self, t: torch.Tensor, which: str) -> torch.Tensor:
-        ix = {"e": self.t_idx, "c": self.t_cidx, "g": self.t_gidx}[which]
+        ix = {"e": self.t_idx, "c": self.cidx(self.plan.bits), "g": self.t_gidx}[which]
         if self.cols is None:
             return t
         return t.index_select(t.dim() - 1, ix)
 
     def step(self, x: torch.Tensor, out: torch.Tensor | None = None, side_stream=None,
-             check_states: bool = True):
-        """One call on x ([P, N] bf16 on the plan's device) and its check."""
-        plan, prm = self.plan, self.prm
-        out = plan.allreduce(x, out=out, side_stream=side_stream)
+             check_states: bool = True, bits: int | None = None):
+        """One call on x ([P, N] bf16 on the plan's device) and its check
+        (bits: the call's code width, None for the plan's current one)."""
+        plan = self.plan
+        out = plan.allreduce(x, out=out, side_stream=side_stream, bits=bits)
+        prm = self._prm()
         torch.cuda.synchronize()
         call = self.calls
         self.calls += 1
@@ -128,9 +145,10 @@ class RSChecker(SequenceChecker):
     """The same comparison for reduce-scatter calls (and, through
     step_allreduce, all-reduce calls on the same plan and state)."""
 
-    def step_rs(self, x: torch.Tensor, side_stream=None):
-        plan, prm = self.plan, self.prm
-        out = plan.reduce_scatter(x, side_stream=side_stream)
+    def step_rs(self, x: torch.Tensor, side_stream=None, bits: int | None = None):
+        plan = self.plan
+        out = plan.reduce_scatter(x, side_stream=side_stream, bits=bits)
+        prm = self._prm()
         torch.cuda.synchronize()
         call = self.calls
         self.calls += 1

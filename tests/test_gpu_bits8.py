@@ -2,14 +2,18 @@
 whole sequences, ragged shapes, the reduce-scatter, the pipelined host
 call, grid-exact inputs and the Llama-shaped workload on sampled columns.
 The pages' serving policy promotes the first half of the layers to 8 bits
-(ai4snews news summary, "Perspective"); a plan is 4- or 8-bit."""
+(ai4snews news summary, "Perspective"): a plan made with bits=8 runs each
+call at 4 or 8 bits on one compensator state, which the mixed-width
+sequences below check call by call, following the layer policy."""
 import numpy as np
 import pytest
 import torch
 
 import oracle_pins
 from bit_error_compensated_echo_b200 import workloads as W
+from bit_error_compensated_echo_b200 import abi
 from bit_error_compensated_echo_b200.api import EchoPlan
+from bit_error_compensated_echo_b200.policy import LayerPolicy
 from parity import RSChecker, SequenceChecker, oracle_params
 
 pytestmark = pytest.mark.gpu
@@ -87,3 +91,55 @@ def test_llama_shape_8bit_sampled():
         chk = SequenceChecker(plan, oracle_params(plan), W.column_sample(w, 512))
         for t in range(8):
             chk.step(W.generate(w, t, DEV))
+
+
+@pytest.mark.parametrize("fixup", ["exit", "side", "deferred"])
+def test_layer_policy_sequence_one_state(fixup):
+    """Two passes over a 6-layer model (2 sites per layer), the first 3
+    layers at 8 bits: 24 calls of both widths on one state, each against the
+    oracle at the call's width."""
+    pol = LayerPolicy(6, 2, 0.5)
+    w = W.with_size(W.TINY, P=4, rows=1, hidden=4 * 64 * 10, G=64)
+    side = torch.cuda.Stream() if fixup == "side" else None
+    with _plan(w.P, w.N, w.G, True, fixup) as plan:
+        chk = SequenceChecker(plan, oracle_params(plan))
+        for t in range(2 * pol.sites):
+            chk.step(W.generate(w, t, DEV), side_stream=side, bits=pol.bits_for_site(t))
+        assert plan.bits == 4
+
+
+def test_mixed_widths_reduce_scatter_and_allreduce():
+    w = W.with_size(W.TINY, P=8, rows=1, hidden=8 * 128 * 5, G=128)
+    with _plan(w.P, w.N, w.G, True, "deferred") as plan:
+        chk = RSChecker(plan, oracle_params(plan))
+        for t, (op, bits) in enumerate([("A", 8), ("R", 4), ("A", 4), ("R", 8), ("A", 8),
+                                        ("A", 4), ("R", 4), ("R", 8)]):
+            x = W.generate(w, t, DEV)
+            if op == "A":
+                chk.step(x, bits=bits)
+            else:
+                chk.step_rs(x, bits=bits)
+
+
+def test_llama_policy_sampled():
+    """The Llama-shaped workload's 64 calls (2 per layer x 32 layers) with
+    the first 16 layers at 8 bits, sampled columns against the oracle."""
+    w = W.LLAMA
+    pol = LayerPolicy(32, 2, 0.5)
+    with _plan(w.P, w.N, w.G, True, "deferred") as plan:
+        chk = SequenceChecker(plan, oracle_params(plan), W.column_sample(w, 256))
+        for t in range(0, pol.sites, 4):        # every 4th site, both widths
+            chk.step(W.generate(w, t, DEV), bits=pol.bits_for_site(t))
+
+
+def test_set_bits_limits():
+    with EchoPlan(2, 2 * 32 * 4, 32, device=0, bits=4) as p4:
+        with pytest.raises(abi.EchoError) as e:
+            p4.set_bits(8)                       # transport sized for 4 bits
+        assert e.value.status == abi.ECHO_ERR_UNSUPPORTED
+    with EchoPlan(2, 2 * 32 * 4, 32, device=0, bits=8) as p8:
+        for bad in (0, 5, 16):
+            with pytest.raises(abi.EchoError):
+                p8.set_bits(bad)
+        p8.set_bits(4)
+        assert p8.debug_view()["codes"].shape == (2, 2 * 32 * 4 // 2)

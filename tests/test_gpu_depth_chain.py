@@ -41,3 +41,19 @@ def test_backward_deviation_smaller_with_compensation(chain):
     comp, off = chain["backward_rel"]["comp"], chain["backward_rel"]["off"]
     assert comp[-1] <= 0.75 * off[-1], (comp[-1], off[-1])
     assert sum(comp) < 0.75 * sum(off)
+
+
+def test_layer_policy_promotion(chain):
+    """The serving policy (first half of the layers at 8 bits, one state;
+    ai4snews news summary, "Perspective"): forward, the 8-bit half stays far
+    below the 4-bit chain and the end of the chain is well below it;
+    backward runs the 4-bit layers first, so the promoted chain equals the
+    4-bit chain there and drops below it once the 8-bit layers come."""
+    comp, prom = chain["forward_rel"]["comp"], chain["forward_rel"]["promoted"]
+    half = len(comp) // 2
+    assert prom[half - 1] < 0.1 * comp[half - 1], (prom[half - 1], comp[half - 1])
+    assert prom[-1] < 0.6 * comp[-1], (prom[-1], comp[-1])
+    bcomp, bprom = chain["backward_rel"]["comp"], chain["backward_rel"]["promoted"]
+    for a, b in zip(bcomp[:half], bprom[:half]):
+        assert abs(a - b) <= 1e-6 * a, (a, b)
+    assert bprom[-1] < 0.5 * bcomp[-1], (bprom[-1], bcomp[-1])

@@ -181,3 +181,21 @@ def test_rank_stage_order_and_arguments():
     with pytest.raises(abi.EchoError) as e:
         abi.echo_rank_plan_create(cfg, 2)      # rank outside the group
     assert e.value.status == abi.ECHO_ERR_INVALID_ARG
+
+
+def test_rank_group_mixed_widths():
+    """Rank plans made with bits=8 follow a per-call width schedule on one
+    state, bit-identical to the virtual-rank plan."""
+    P, G, N = 4, 64, 4 * 64 * 7
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    with EmulatedGroup(P, N, G, fixup="deferred", bits=8) as grp, \
+            EchoPlan(P, N, G, device=0, fixup="deferred", bits=8) as plan:
+        for t, bits in enumerate([8, 8, 4, 4, 8, 4, 4, 8]):
+            for p in grp.plans:
+                p.set_bits(bits)
+            plan.set_bits(bits)
+            x = W.generate(w, t, DEV)
+            _same("outputs", grp.allreduce(x), plan.allreduce(x), t)
+            _compare_wires(grp, plan, t)
+            for a, b in zip(grp.get_state(), plan.get_state()):
+                _same("state", a, b, t)
