@@ -287,6 +287,60 @@ def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: i
     return nbytes / dt / 1e9, dt, cols.size
 
 
+def _oracle_part(job):
+    """Worker of oracle_parallel_run: the oracle on one column range of the
+    shared input sample; returns its own compute seconds."""
+    from multiprocessing import shared_memory
+
+    import oracle
+    name, shape, prm_kw, c0, c1, G, cols = job
+    shm = shared_memory.SharedMemory(name=name)
+    try:
+        xb = np.ndarray(shape, dtype=np.uint16, buffer=shm.buf)[:, c0 * G:c1 * G].copy()
+    finally:
+        shm.close()
+    prm = oracle.Params(**prm_kw)
+    mf = np.zeros(xb.shape, np.float32)
+    ms = np.zeros_like(mf)
+    t0 = time.perf_counter()
+    oracle.allreduce(prm, xb, mf, ms, np.asarray(cols[c0:c1], np.int64))
+    return time.perf_counter() - t0
+
+
+def oracle_parallel_run(w: W.Workload, comp: bool, ncols: int, x_dev, bits: int = 4,
+                        workers: int = 0, reps: int = 3):
+    """The same oracle, as it stands, on the same column sample split over
+    all host cores (processes started with spawn, inputs in shared memory):
+    every quantity depends only on its group column, so the split is exact.
+    Returns (GB/s, median wall seconds, workers)."""
+    import multiprocessing as mp
+    from multiprocessing import shared_memory
+    workers = workers or len(os.sched_getaffinity(0))
+    cols = W.column_sample(w, ncols, seed=7)
+    idx = W.column_elements(cols, w.G)
+    ti = torch.from_numpy(idx).to(x_dev.device)
+    xb = W.bf16_bits(x_dev.index_select(1, ti))
+    shm = shared_memory.SharedMemory(create=True, size=xb.nbytes)
+    try:
+        np.ndarray(xb.shape, dtype=np.uint16, buffer=shm.buf)[:] = xb
+        prm_kw = dict(P=w.P, N=w.N, G=w.G, compensate=comp, bits=bits)
+        bounds = np.linspace(0, cols.size, workers + 1).astype(int)
+        jobs = [(shm.name, xb.shape, prm_kw, int(bounds[i]), int(bounds[i + 1]), w.G, cols)
+                for i in range(workers) if bounds[i + 1] > bounds[i]]
+        times = []
+        with mp.get_context("spawn").Pool(len(jobs)) as pool:
+            pool.map(_oracle_part, jobs)                 # start-up and warm-up
+            for _ in range(reps):
+                t0 = time.perf_counter()
+                pool.map(_oracle_part, jobs)
+                times.append(time.perf_counter() - t0)
+    finally:
+        shm.close()
+        shm.unlink()
+    dt = statistics.median(times)
+    return 2 * w.P * idx.size / dt / 1e9, dt, len(jobs)
+
+
 # ------------------------------------------------------------ modes
 
 def run_step_mode(args, ws, rank, local):
@@ -368,13 +422,19 @@ def run_step_mode(args, ws, rank, local):
                "d2h_bytes_per_step": 2 * P * N}
         del xh, yh
 
-    cpu = None
+    cpu = cpu_par = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         gbs, dt, ncols = oracle_sample_run(w, comp, args.cpu_cols, x_dev=x, bits=args.bits)
         cpu = {"value": round(gbs, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "%d of %d group columns (x %d ranks x G=%d) of the same inputs, one "
                          "call from zero state, %.1f s on one host thread" %
                          (ncols, N // G, P, G, dt)}
+        if not args.no_cpu_parallel:
+            pg, pdt, nw = oracle_parallel_run(w, comp, args.cpu_cols, x, bits=args.bits)
+            cpu_par = {"value": round(pg, 5), "unit": UNIT, "cores": nw, "kind": "oracle",
+                       "sample": "the same %d columns split over %d spawned processes (one "
+                                 "per host core), median of 3 runs, %.2f s wall" %
+                                 (ncols, nw, pdt)}
 
     if rank == 0:
         calls = prof["calls"]
@@ -410,7 +470,7 @@ def run_step_mode(args, ws, rank, local):
             "kernels_ms": {k: round(prof[k] / max(calls, 1), 4)
                            for k in ("entry_ms", "reduce_ms", "exit_ms", "fixup_ms")},
             "gpu_launches": int(prof["launches"]),
-            "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
+            "e2e": e2e, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_par, "clocks": clk,
         }
         print(json.dumps(line), flush=True)
     plan.close()
@@ -705,6 +765,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cpu-parallel", action="store_true",
+                    help="skip the all-cores run of the oracle beside the CPU baseline")
     ap.add_argument("--cpu-cols", type=int, default=655360,
                     help="group columns of the CPU-baseline sample")
     ap.add_argument("--ref-cols", type=int, default=131072,

@@ -23,3 +23,13 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"] == "large_p8_1gib_g128"
+
+
+def test_oracle_all_cores_run_on_cpu():
+    """The all-cores CPU baseline: the oracle over column ranges in spawned
+    processes, inputs in shared memory (here 2 workers, tiny workload)."""
+    import bench
+    from bit_error_compensated_echo_b200 import workloads as W
+    x = W.generate(W.TINY, 0, "cpu")
+    gbs, dt, nw = bench.oracle_parallel_run(W.TINY, True, 64, x, workers=2, reps=1)
+    assert nw == 2 and gbs > 0 and dt > 0
