@@ -20,9 +20,15 @@ namespace echo {
 // holding its own chunk only: er_chunk_vec = 0).
 //   VPT   : vectors per thread.  A block covers kThreads*VPT vectors; thread t
 //           takes vectors t, t + kThreads, ... so each load instruction of a
-//           warp is contiguous, and all of a thread's loads are issued before
-//           any arithmetic: the bytes in flight per SM grow with VPT, which is
-//           what bounds the uncompensated pass (2.5 bytes per element).
+//           warp is contiguous, and all of a thread's input and state loads
+//           are issued before any arithmetic: the bytes in flight per SM grow
+//           with VPT, which is what bounds the uncompensated pass (2.5 bytes
+//           per element).
+// x is a __grid_constant__ parameter: the block's rank selects its pointer
+// straight from the parameter bank.  Indexing a by-value array parameter
+// with a run-time index otherwise copies the whole array to every thread's
+// local memory first (64 bytes per thread, 2^28 threads per 1 GiB-per-rank
+// launch), which measured 7% of the entry's time.
 template <bool COMP>
 struct EntryShape {
     static constexpr int VPT = COMP ? 2 : 4;
@@ -37,7 +43,7 @@ inline unsigned entry_blocks(int64_t v_count) {
 
 template <int G, bool COMP, bool DEFER, int BITS>
 __global__ void __launch_bounds__(kThreads, EntryShape<COMP>::MIN_BLOCKS)
-echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_slow,
+echo_entry_kernel(const __grid_constant__ InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_slow,
                   uint32_t *__restrict__ codes, float *__restrict__ scales,
                   const float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec,
                   Slab sl, int P, Consts k, int rank0, int64_t er_chunk_vec) {
@@ -48,7 +54,7 @@ echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_sl
     const int64_t base = (int64_t)blockIdx.x * (kThreads * VPT) + threadIdx.x;
     const float2 z = splat2(k.neg_zero);
 
-    float xt[VPT][8], mf[COMP ? VPT : 1][8], ms[COMP ? VPT : 1][8], er[DEFER ? VPT : 1][8];
+    float xt[VPT][8], mf[COMP ? VPT : 1][8], ms[COMP ? VPT : 1][8];
     int64_t j[VPT];
     bool valid[VPT];
 
@@ -64,8 +70,6 @@ echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_sl
                 const int64_t e0 = ((int64_t)r * n_vec + j[v]) * kVec;
                 ld8(m_fast + e0, mf[v]);
                 ld8(m_slow + e0, ms[v]);
-                if (DEFER && own)
-                    ld8(e_req + ((int64_t)o * er_chunk_vec + sl.v_begin + l) * kVec, er[v]);
             }
         } else {
 #pragma unroll
@@ -77,10 +81,16 @@ echo_entry_kernel(InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_sl
     for (int v = 0; v < VPT; ++v) {
         if (COMP && valid[v]) {
             if (DEFER && own) {
+                // e_req is loaded here, not with the other operands: only the
+                // owner's blocks (1/P of them) read it, and keeping its 8
+                // values live across the loads would cost every block registers
+                float er[8];
+                const int64_t l = base + (int64_t)v * kThreads;
+                ld8(e_req + ((int64_t)o * er_chunk_vec + sl.v_begin + l) * kVec, er);
                 const float2 obf = splat2(k.one_m_beta_fast), obs = splat2(k.one_m_beta_slow);
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {
-                    const float2 e2 = make_float2(er[v][i], er[v][i + 1]);
+                    const float2 e2 = make_float2(er[i], er[i + 1]);
                     const float2 f = add2(make_float2(mf[v][i], mf[v][i + 1]), prod2(obf, e2, z));
                     const float2 g = add2(make_float2(ms[v][i], ms[v][i + 1]), prod2(obs, e2, z));
                     mf[v][i] = f.x; mf[v][i + 1] = f.y;

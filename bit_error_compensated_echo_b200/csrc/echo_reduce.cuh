@@ -127,10 +127,12 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
 // bf16(s) of chunk o.  The owner's output residual e = s - float(bf16(s))
 // is folded into its own EMAs here (FIX) or written to e_req for a
 // side-stream or deferred fix-up (COMP && !FIX).
-// Grid: x over the 16-element runs of the slab, y = owner.
+// Grid: x over the 16-element runs of the slab, y = owner (out is a
+// __grid_constant__ parameter, indexed by the owner without a local copy).
 template <int G, int P, bool COMP, bool FIX, int BITS>
 __global__ void __launch_bounds__(kThreads)
-echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales, OutPtrs out,
+echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
+               const __grid_constant__ OutPtrs out,
                float *__restrict__ m_fast, float *__restrict__ m_slow, float *__restrict__ e_req,
                int64_t n_vec, int64_t chunk_vec, Slab sl, Consts k) {
     const int o = blockIdx.y;
