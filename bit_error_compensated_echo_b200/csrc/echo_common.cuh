@@ -107,6 +107,8 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
 }
 __device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
 
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c);
+
 // the separately rounded products a.x*b.x, a.y*b.y; z must hold the run-time
 // value (-0.0f, -0.0f)
 __device__ __forceinline__ float2 prod2(float2 a, float2 b, float2 z) {
@@ -117,6 +119,9 @@ __device__ __forceinline__ float2 prod2(float2 a, float2 b, float2 z) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(z.x), "f"(z.y));
     return d;
 }
+
+// a*b + c rounded once, for a pair
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return prod2(a, b, c); }
 
 // ---- exact integer <-> float steps without conversion instructions
 //
@@ -223,34 +228,6 @@ __device__ __forceinline__ float2 bf16x2_to_f32(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
-// scale = a / L, or 0 for an all-zero group
-template <int BITS>
-__device__ __forceinline__ float group_scale(float a) {
-    return a != 0.0f ? __fdiv_rn(a, CodeWidth<BITS>::levels) : 0.0f;
-}
-
-// Quantize 8 values of a group with one IEEE division per element:
-// k = clamp(rint(v / scale), -L, L), ties to even, all 0 when scale == 0;
-// k as floats in kf.  Preferred where the values are short bf16 numbers.
-template <int BITS>
-__device__ __forceinline__ Packed8<BITS> quantize8_div(const float v[8], float scale, float kf[8]) {
-    constexpr float L = CodeWidth<BITS>::levels;
-    Packed8<BITS> p = {};
-    if (scale == 0.0f) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) kf[i] = 0.0f;
-        return p;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float q = fminf(fmaxf(__fdiv_rn(v[i], scale), -L), L);
-        const float t = __fadd_rn(q, kRoundMagic);
-        kf[i] = __fsub_rn(t, kRoundMagic);
-        put_code<BITS>(p, t, i);
-    }
-    return p;
-}
-
 // Quantize 8 values of a group: k = clamp(rint(v / scale), -L, L), ties to
 // even, all 0 when scale == 0; the packed codes and k as floats in kf.
 //
@@ -260,21 +237,21 @@ __device__ __forceinline__ Packed8<BITS> quantize8_div(const float v[8], float s
 // |q| <= 127), so the two round to the same integer unless the exact
 // quotient lies that close to a half-integer.  The fast path rounds q~ and
 // flags any element whose q~ lies within twice that (the tie window) of a
-// half-integer; then (rarely), and for every group whose scale is
-// subnormal, all 8 codes are taken from the IEEE division itself.  Either
-// way the codes are exactly those of rint(v/scale).  For a normal scale
-// |q~| <= L*(1 + 2^-22) < L + 1/2, so the fast path needs no clamp.
+// half-integer; then (rarely), and for every group whose scale lies outside
+// [2^-100, 2^100], all 8 codes are taken from the IEEE division itself.
+// Either way the codes are exactly those of rint(v/scale).  For a normal
+// scale |q~| <= L*(1 + 2^-22) < L + 1/2, so the fast path needs no clamp.
 struct GroupScale {
     float scale;  // a / L (0 for an all-zero group)
     float inv;    // 1 / scale rounded, 0 when scale == 0
-    bool exact;   // subnormal scale: always use the division
+    bool exact;   // scale outside [2^-100, 2^100]: always use the division
 };
 
 template <int BITS>
 __device__ __forceinline__ GroupScale make_group_scale(float a) {
     GroupScale g;
     g.scale = a != 0.0f ? __fdiv_rn(a, CodeWidth<BITS>::levels) : 0.0f;
-    g.exact = g.scale != 0.0f && g.scale < 1.17549435e-38f;  // below FLT_MIN
+    g.exact = g.scale != 0.0f && (g.scale < 0x1p-100f || g.scale > 0x1p100f);
     g.inv = (g.scale != 0.0f && !g.exact) ? __frcp_rn(g.scale) : 0.0f;
     return g;
 }
@@ -311,6 +288,45 @@ __device__ __forceinline__ Packed8<BITS> quantize8(const float v[8], const Group
         put_code<BITS>(p, t.y, i + 1);
     }
     if (g.exact || dmax > 0.5f - CodeWidth<BITS>::tie_window) p = quantize8_exact<BITS>(v, g.scale, kf);
+    return p;
+}
+
+// Quantize 8 values of a group through the correctly rounded quotient,
+// computed without a division by Markstein's method (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990; the theorem as stated in
+// Muller et al., "Handbook of Floating-Point Arithmetic", 2nd ed.):
+// with y = RN(1/s) and q within one ulp of v/s, the remainder v - q*s is
+// exact in one fma and RN(q + (v - q*s)*y) = RN(v/s).  q0 = RN(v*y) is
+// within 1.5 ulp of v/s, one correction brings it within one ulp (its error
+// shrinks by the factor |1 - s*y| <= 2^-24, plus half an ulp of rounding),
+// and a second correction yields RN(v/s).  For s in [2^-100, 2^100] no
+// intermediate overflows, and the remainders of the elements that can
+// round to a nonzero code (|v| >= s/2) are normal numbers.  Then
+// k = rint(RN(v/s)) exactly as the definition's division, and
+// |RN(v/s)| <= L + ulp(L) rounds to at most L: no clamp.  A zero scale
+// (inv = 0) gives q = 0 and all codes 0.  Other scales use the division.
+template <int BITS>
+__device__ __forceinline__ Packed8<BITS> quantize8_q(const float v[8], const GroupScale &g,
+                                                     float kf[8], float2 z) {
+    if (g.exact) return quantize8_exact<BITS>(v, g.scale, kf);
+    Packed8<BITS> p = {};
+    const float2 y = splat2(g.inv), ns = splat2(-g.scale), magic2 = splat2(kRoundMagic);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const float2 x = make_float2(v[i], v[i + 1]);
+        float2 q = prod2(x, y, z);     // RN(v*y)
+        float2 r = fma2(q, ns, x);     // v - q*s, exact
+        q = fma2(r, y, q);
+        r = fma2(q, ns, x);
+        q = fma2(r, y, q);             // RN(v/s)
+        const float2 t = add2(q, magic2);
+        const float2 k = sub2(t, magic2);
+        kf[i] = k.x;
+        kf[i + 1] = k.y;
+        put_code<BITS>(p, t.x, i);
+        put_code<BITS>(p, t.y, i + 1);
+    }
     return p;
 }
 

@@ -115,13 +115,13 @@ echo_entry_kernel(const __grid_constant__ InPtrs x, float *__restrict__ m_fast, 
         float kf[8];
         float scale;
         Packed8<BITS> w;
-        if (COMP) {   // corrected inputs carry full fp32 mantissas: ties are rare
+        {
             const GroupScale gs = make_group_scale<BITS>(a);
             scale = gs.scale;
-            w = quantize8<BITS>(xt[v], gs, kf, z);
-        } else {      // raw bf16 inputs: one IEEE division per element
-            scale = group_scale<BITS>(a);
-            w = quantize8_div<BITS>(xt[v], scale, kf);
+            if (COMP)   // corrected inputs carry full fp32 mantissas: ties are rare
+                w = quantize8<BITS>(xt[v], gs, kf, z);
+            else        // raw bf16 inputs sit on ties often: the exact quotient
+                w = quantize8_q<BITS>(xt[v], gs, kf, z);
         }
         if (!valid[v]) continue;
 

@@ -95,8 +95,8 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
     const GroupScale gs = make_group_scale<BITS>(a);
     const float scale2 = gs.scale;
     float k2[16];
-    const Packed8<BITS> w0 = quantize8<BITS>(s, gs, k2, z);
-    const Packed8<BITS> w1 = quantize8<BITS>(s + 8, gs, k2 + 8, z);
+    const Packed8<BITS> w0 = quantize8_q<BITS>(s, gs, k2, z);
+    const Packed8<BITS> w1 = quantize8_q<BITS>(s + 8, gs, k2 + 8, z);
     if (!valid) return;
 
     if (BITS == 4)
