@@ -164,10 +164,30 @@ struct Packed8 {
     uint32_t w[BITS / 4];
 };
 
+// Pack the codes of 8 elements from their magic sums t (the low bits of each
+// sum's bit pattern are its code): byte permutes gather the low bytes, four
+// to a word; for 4-bit codes one bitwise select then merges the odd
+// elements' nibbles (shifted up by 4) into the even elements' bytes.
 template <int BITS>
-__device__ __forceinline__ void put_code(Packed8<BITS> &p, float t, int i) {
-    constexpr uint32_t mask = (1u << BITS) - 1u;
-    p.w[(i * BITS) / 32] |= (__float_as_uint(t) & mask) << ((i * BITS) % 32);
+__device__ __forceinline__ Packed8<BITS> pack_codes(const float t[8]) {
+    Packed8<BITS> p;
+    uint32_t u[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u[i] = __float_as_uint(t[i]);
+    if (BITS == 4) {
+        // even elements: {u0, u2, u4, u6}.b0; odd elements: {u1, u3, u5, u7}.b0
+        const uint32_t e = __byte_perm(__byte_perm(u[0], u[2], 0x0040),
+                                       __byte_perm(u[4], u[6], 0x0040), 0x5410);
+        const uint32_t o = __byte_perm(__byte_perm(u[1], u[3], 0x0040),
+                                       __byte_perm(u[5], u[7], 0x0040), 0x5410);
+        p.w[0] = (e & 0x0F0F0F0Fu) | ((o << 4) & 0xF0F0F0F0u);
+    } else {
+        p.w[0] = __byte_perm(__byte_perm(u[0], u[1], 0x0040),
+                             __byte_perm(u[2], u[3], 0x0040), 0x5410);
+        p.w[BITS / 4 - 1] = __byte_perm(__byte_perm(u[4], u[5], 0x0040),
+                                        __byte_perm(u[6], u[7], 0x0040), 0x5410);
+    }
+    return p;
 }
 
 // 2^23 + (byte b of word u), as a float
@@ -259,20 +279,20 @@ __device__ __forceinline__ GroupScale make_group_scale(float a) {
 template <int BITS>
 __device__ __forceinline__ Packed8<BITS> quantize8_exact(const float v[8], float scale, float kf[8]) {
     constexpr float L = CodeWidth<BITS>::levels;
-    Packed8<BITS> p = {};
+    float t[8];
     for (int i = 0; i < 8; ++i) {
-        float t = kRoundMagic;
-        if (scale != 0.0f) t = __fadd_rn(fminf(fmaxf(__fdiv_rn(v[i], scale), -L), L), kRoundMagic);
-        kf[i] = __fsub_rn(t, kRoundMagic);
-        put_code<BITS>(p, t, i);
+        t[i] = kRoundMagic;
+        if (scale != 0.0f)
+            t[i] = __fadd_rn(fminf(fmaxf(__fdiv_rn(v[i], scale), -L), L), kRoundMagic);
+        kf[i] = __fsub_rn(t[i], kRoundMagic);
     }
-    return p;
+    return pack_codes<BITS>(t);
 }
 
 template <int BITS>
 __device__ __forceinline__ Packed8<BITS> quantize8(const float v[8], const GroupScale &g,
                                                    float kf[8], float2 z) {
-    Packed8<BITS> p = {};
+    float tt[8];
     const float2 inv2 = splat2(g.inv), magic2 = splat2(kRoundMagic);
     float dmax = 0.0f;
 #pragma unroll
@@ -284,11 +304,12 @@ __device__ __forceinline__ Packed8<BITS> quantize8(const float v[8], const Group
         kf[i] = k.x;
         kf[i + 1] = k.y;
         dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
-        put_code<BITS>(p, t.x, i);
-        put_code<BITS>(p, t.y, i + 1);
+        tt[i] = t.x;
+        tt[i + 1] = t.y;
     }
-    if (g.exact || dmax > 0.5f - CodeWidth<BITS>::tie_window) p = quantize8_exact<BITS>(v, g.scale, kf);
-    return p;
+    if (g.exact || dmax > 0.5f - CodeWidth<BITS>::tie_window)
+        return quantize8_exact<BITS>(v, g.scale, kf);
+    return pack_codes<BITS>(tt);
 }
 
 // Quantize 8 values of a group through the correctly rounded quotient,
@@ -310,7 +331,7 @@ template <int BITS>
 __device__ __forceinline__ Packed8<BITS> quantize8_q(const float v[8], const GroupScale &g,
                                                      float kf[8], float2 z) {
     if (g.exact) return quantize8_exact<BITS>(v, g.scale, kf);
-    Packed8<BITS> p = {};
+    float tt[8];
     const float2 y = splat2(g.inv), ns = splat2(-g.scale), magic2 = splat2(kRoundMagic);
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
@@ -324,10 +345,10 @@ __device__ __forceinline__ Packed8<BITS> quantize8_q(const float v[8], const Gro
         const float2 k = sub2(t, magic2);
         kf[i] = k.x;
         kf[i + 1] = k.y;
-        put_code<BITS>(p, t.x, i);
-        put_code<BITS>(p, t.y, i + 1);
+        tt[i] = t.x;
+        tt[i + 1] = t.y;
     }
-    return p;
+    return pack_codes<BITS>(tt);
 }
 
 __device__ __forceinline__ void ld8(const float *p, float v[8]) {
