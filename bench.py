@@ -4,8 +4,9 @@
                     [--workload large|llama|depth|tiny] [--fixup exit|side|deferred]
                     [--uncompensated] [--mode step|sweep|overlap|depth-chain|group]
 
-Default (mode "step"): one step = one echo_allreduce call (entry + reduce +
-exit kernels) of P=8 virtual ranks x 2^29 bf16 elements (1 GiB) per rank,
+Default (mode "step"): one step = one echo_allreduce call (entry kernel, then
+the reduce kernel that also writes every rank's output) of P=8 virtual ranks
+x 2^29 bf16 elements (1 GiB) per rank,
 G=128, compensator on, inputs resident in HBM.  Prints ONE JSON line with
 the input GB/s per call (all ranks' input bytes / call time), the whole-call
 fraction of the HBM roofline (minimal bytes of a call / measured copy
@@ -105,17 +106,25 @@ def entry_bytes(P: int, N: int, G: int, comp: bool, fixup: str, bits: int = 4) -
     return b
 
 
-def reduce_bytes(P: int, N: int, G: int, comp: bool) -> float:
-    q = transport_bytes_per_elem(G)
-    return P * N * q + N * q + (N * 4 if comp else 0)
-
-
-def exit_bytes(P: int, N: int, G: int, comp: bool, fixup: str) -> float:
-    q = transport_bytes_per_elem(G)
-    b = N * q + P * N * 2
-    if comp and fixup == "exit":
-        b += N * (4 + 16)
+def reduce_bytes(P: int, N: int, G: int, comp: bool, fixup: str, bits: int = 4) -> float:
+    """Algorithmic bytes of one echo_reduce launch of the virtual plan: read
+    the entry transport (P*q per element of N), write the reduced transport
+    (q); uncompensated also the P bf16 outputs (2P); compensated, write
+    e_req (4) or, with the fix-up in the kernel, read and write the owner's
+    states (16)."""
+    q = transport_bytes_per_elem(G, bits)
+    b = P * N * q + N * q
+    if comp:
+        b += N * (16 if fixup == "exit" else 4)
+    else:
+        b += P * N * 2
     return b
+
+
+def exit_bytes(P: int, N: int, G: int, bits: int = 4) -> float:
+    """echo_exit (compensated calls): read the reduced transport, write the
+    P bf16 outputs."""
+    return N * transport_bytes_per_elem(G, bits) + P * N * 2
 
 
 # ------------------------------------------------------------ environment
@@ -583,7 +592,7 @@ def run_sweep_mode(args, ws, rank, local):
 
 def run_overlap_mode(args, ws, rank, local):
     """1 GiB per rank, P=8: the stand-in next matmul (bf16 8192^3) after each
-    call, with the owner fix-up in the exit kernel, on a side stream beside
+    call, with the owner fix-up in the reduce kernel, on a side stream beside
     the matmul, or deferred; plus the fused compensation cost (compensated
     minus uncompensated call) and the compensator written as separate torch
     operations, for context."""

@@ -38,64 +38,68 @@ void entry_b(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er, Sl
 }
 
 // ---- reduce
+// the run-time part of a reduce launch: outputs and in-kernel fix-up
+struct ReduceOut {
+    OutPtrs out;
+    int n_out;
+    int fix;
+};
+
 template <int G, int P, int BITS>
-void reduce_t(const Bufs &b, int owners, Slab sl, cudaStream_t st) {
+void reduce_t(const Bufs &b, int owners, Slab sl, cudaStream_t st, const ReduceOut &ro) {
     dim3 grid(reduce_blocks(sl.v_count), (unsigned)owners);
+    // compensated reduces never write the outputs (the exit pass does)
     if (b.comp)
-        echo_reduce_kernel<G, P, true, BITS><<<grid, kThreads, 0, st>>>(
-            b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl,
-            b.k.neg_zero);
+        echo_reduce_kernel<G, P, true, false, BITS><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
+            ro.out, 0, b.m_fast, b.m_slow, ro.fix);
+    else if (ro.n_out > 0)
+        echo_reduce_kernel<G, P, false, true, BITS><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
+            ro.out, ro.n_out, nullptr, nullptr, 0);
     else
-        echo_reduce_kernel<G, P, false, BITS><<<grid, kThreads, 0, st>>>(
-            b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl,
-            b.k.neg_zero);
+        echo_reduce_kernel<G, P, false, false, BITS><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
+            ro.out, 0, nullptr, nullptr, 0);
 }
 
 template <int G, int BITS>
-void reduce_g(const Bufs &b, int owners, Slab sl, cudaStream_t st) {
+void reduce_g(const Bufs &b, int owners, Slab sl, cudaStream_t st, const ReduceOut &ro) {
     switch (b.P) {
-        case 1: reduce_t<G, 1, BITS>(b, owners, sl, st); break;
-        case 2: reduce_t<G, 2, BITS>(b, owners, sl, st); break;
-        case 3: reduce_t<G, 3, BITS>(b, owners, sl, st); break;
-        case 4: reduce_t<G, 4, BITS>(b, owners, sl, st); break;
-        case 5: reduce_t<G, 5, BITS>(b, owners, sl, st); break;
-        case 6: reduce_t<G, 6, BITS>(b, owners, sl, st); break;
-        case 7: reduce_t<G, 7, BITS>(b, owners, sl, st); break;
-        default: reduce_t<G, 8, BITS>(b, owners, sl, st); break;
+        case 1: reduce_t<G, 1, BITS>(b, owners, sl, st, ro); break;
+        case 2: reduce_t<G, 2, BITS>(b, owners, sl, st, ro); break;
+        case 3: reduce_t<G, 3, BITS>(b, owners, sl, st, ro); break;
+        case 4: reduce_t<G, 4, BITS>(b, owners, sl, st, ro); break;
+        case 5: reduce_t<G, 5, BITS>(b, owners, sl, st, ro); break;
+        case 6: reduce_t<G, 6, BITS>(b, owners, sl, st, ro); break;
+        case 7: reduce_t<G, 7, BITS>(b, owners, sl, st, ro); break;
+        default: reduce_t<G, 8, BITS>(b, owners, sl, st, ro); break;
     }
 }
 
 template <int BITS>
-void reduce_b(const Bufs &b, int owners, Slab sl, cudaStream_t st) {
+void reduce_b(const Bufs &b, int owners, Slab sl, cudaStream_t st, const ReduceOut &ro) {
     switch (b.G) {
-        case 32: reduce_g<32, BITS>(b, owners, sl, st); break;
-        case 64: reduce_g<64, BITS>(b, owners, sl, st); break;
-        default: reduce_g<128, BITS>(b, owners, sl, st); break;
+        case 32: reduce_g<32, BITS>(b, owners, sl, st, ro); break;
+        case 64: reduce_g<64, BITS>(b, owners, sl, st, ro); break;
+        default: reduce_g<128, BITS>(b, owners, sl, st, ro); break;
     }
 }
 
 // ---- exit
 template <int G, int BITS>
-void exit_g(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, bool fix,
-            cudaStream_t st) {
+void exit_g(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, cudaStream_t st) {
     dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)owners);
-    if (fix)
-        echo_exit_kernel<G, true, BITS><<<grid, kThreads, 0, st>>>(
-            b.rcodes, b.rscales, out, n_out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec,
-            sl, b.k);
-    else
-        echo_exit_kernel<G, false, BITS><<<grid, kThreads, 0, st>>>(
-            b.rcodes, b.rscales, out, n_out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec,
-            sl, b.k);
+    echo_exit_kernel<G, BITS><<<grid, kThreads, 0, st>>>(b.rcodes, b.rscales, out, n_out,
+                                                          b.chunk_vec, sl);
 }
 
 template <int BITS>
-void exit_b(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, bool fix,
-            cudaStream_t st) {
+void exit_b(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, cudaStream_t st) {
     switch (b.G) {
-        case 32: exit_g<32, BITS>(b, out, n_out, owners, sl, fix, st); break;
-        case 64: exit_g<64, BITS>(b, out, n_out, owners, sl, fix, st); break;
-        default: exit_g<128, BITS>(b, out, n_out, owners, sl, fix, st); break;
+        case 32: exit_g<32, BITS>(b, out, n_out, owners, sl, st); break;
+        case 64: exit_g<64, BITS>(b, out, n_out, owners, sl, st); break;
+        default: exit_g<128, BITS>(b, out, n_out, owners, sl, st); break;
     }
 }
 
@@ -145,15 +149,22 @@ void launch_entry(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t e
     else entry_b<4>(b, x, rows, rank0, er_chunk_vec, sl, defer, st);
 }
 
-void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st) {
-    if (b.bits == 8) reduce_b<8>(b, owners, sl, st);
-    else reduce_b<4>(b, owners, sl, st);
+void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st, const OutPtrs *out,
+                   int n_out, bool fix) {
+    ReduceOut ro{};
+    if (out && n_out > 0) {
+        ro.out = *out;
+        ro.n_out = n_out;
+    }
+    ro.fix = (fix && b.comp) ? 1 : 0;
+    if (b.bits == 8) reduce_b<8>(b, owners, sl, st, ro);
+    else reduce_b<4>(b, owners, sl, st, ro);
 }
 
-void launch_exit(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, bool fix,
+void launch_exit(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl,
                  cudaStream_t st) {
-    if (b.bits == 8) exit_b<8>(b, out, n_out, owners, sl, fix, st);
-    else exit_b<4>(b, out, n_out, owners, sl, fix, st);
+    if (b.bits == 8) exit_b<8>(b, out, n_out, owners, sl, st);
+    else exit_b<4>(b, out, n_out, owners, sl, st);
 }
 
 void launch_rs(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix,

@@ -54,12 +54,17 @@ inline Consts make_consts(const echo_config &c) {
 void launch_entry(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chunk_vec,
                   Slab sl, bool defer, cudaStream_t st);
 
-// Reduce of `owners` chunks (grid y): sum the P rows, requantize, e_req.
-void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st);
+// Reduce of `owners` chunks (grid y): sum the P rows, requantize;
+// uncompensated with n_out > 0 also write the dequantized sum to the n_out
+// outputs (compensated reduces leave that to launch_exit); compensating,
+// either write e_req or, with fix, apply the owner fix-up to state row o
+// of each chunk o.
+void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st,
+                   const OutPtrs *out = nullptr, int n_out = 0, bool fix = false);
 
-// Exit over `owners` chunks (grid y) into n_out outputs; fix: owner fix-up
-// of state row o for chunk o (the virtual-rank layout).
-void launch_exit(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, bool fix,
+// Exit over `owners` chunks (grid y): dequantize the reduced transport into
+// n_out outputs.
+void launch_exit(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl,
                  cudaStream_t st);
 
 // Reduce-scatter second kernel over `owners` chunks (grid y): out.p[o]

@@ -63,7 +63,7 @@ cudaError_t scratch_address(int dev, unsigned char **out) {
     return cudaSuccess;
 }
 
-// The three launches of one call, on the array's carved sub-buffers.
+// The launches of one call, on the array's carved sub-buffers.
 void launch_all(const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigned char *s,
                 const ScratchLayout &L, const echo_config &c, cudaStream_t st) {
     Bufs b;
@@ -83,8 +83,12 @@ void launch_all(const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigne
     b.k = make_consts(c);
     const Slab sl{0, b.chunk_vec};
     launch_entry(b, x, c.P, 0, b.chunk_vec, sl, false, st);
-    launch_reduce(b, c.P, sl, st);
-    launch_exit(b, y, c.P, c.P, sl, b.comp, st);
+    if (b.comp) {   // owner fix-up in the reduce, outputs in the exit pass
+        launch_reduce(b, c.P, sl, st, nullptr, 0, true);
+        launch_exit(b, y, c.P, c.P, sl, st);
+    } else {        // the reduce writes the outputs
+        launch_reduce(b, c.P, sl, st, &y, c.P, false);
+    }
 }
 
 }  // namespace

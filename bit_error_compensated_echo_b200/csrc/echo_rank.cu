@@ -10,8 +10,9 @@
 //            elements with a single owner chunk
 //   exit   : the gathered reduced chunks are the virtual plan's reduced
 //            transport; one output instead of P
-// The owner fix-up of the EXIT and SIDE modes works on this rank's chunk of
-// the state through pointers offset by rank*C.
+// The owner fix-up of the EXIT mode runs in the reduce kernel, and that of
+// the SIDE mode in its own kernel; both work on this rank's chunk of the
+// state through pointers offset by rank*C.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -82,8 +83,7 @@ void own_chunk_fixup(echo_rank_plan *p, const float *src_f, const float *src_s, 
 }
 
 // Step 7 after a reduce or reduce-scatter, by the plan's mode.  in_kernel:
-// the launch just made already applied it (the reduce-scatter kernel in
-// EXIT mode).
+// the launch just made already applied it (EXIT mode).
 echo_status after_reduce(echo_rank_plan *p, cudaStream_t st, cudaStream_t side, bool in_kernel) {
     if (!p->cfg.compensate) return ECHO_OK;
     switch (p->cfg.fixup) {
@@ -233,10 +233,16 @@ echo_status echo_rank_reduce(echo_rank_plan *p, const void *recv_codes, const fl
     b.rscales = red_scales;
     b.n_vec = p->chunk_vec;       // a received row is one chunk
     b.chunk_vec = p->chunk_vec;
-    launch_reduce(b, 1, chunk_slab(p), st);
+    const bool fix = p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_EXIT;
+    if (fix) {                    // the fix-up in the reduce: this rank's chunk of its state
+        const int64_t off = (int64_t)p->rank * p->C;
+        b.m_fast = p->m_fast + off;
+        b.m_slow = p->m_slow + off;
+    }
+    launch_reduce(b, 1, chunk_slab(p), st, nullptr, 0, fix);
     ECHO_TRY(cudaGetLastError());
     p->entered = false;
-    return after_reduce(p, st, (cudaStream_t)side_stream, false);
+    return after_reduce(p, st, (cudaStream_t)side_stream, fix);
 }
 
 echo_status echo_rank_exit(echo_rank_plan *p, const void *all_codes, const float *all_scales,
@@ -253,7 +259,7 @@ echo_status echo_rank_exit(echo_rank_plan *p, const void *all_codes, const float
     b.chunk_vec = p->chunk_vec;
     OutPtrs yo{};
     yo.p[0] = (uint4 *)out;
-    launch_exit(b, yo, 1, p->cfg.P, chunk_slab(p), false, (cudaStream_t)stream);
+    launch_exit(b, yo, 1, p->cfg.P, chunk_slab(p), (cudaStream_t)stream);
     ECHO_TRY(cudaGetLastError());
     return ECHO_OK;
 }
@@ -345,7 +351,7 @@ echo_status echo_rank_plan_set_bits(echo_rank_plan *p, int32_t bits) {
 
 int32_t echo_rank_launches_per_call(const echo_rank_plan *p) {
     if (!p) return 0;
-    const bool own_kernel = p->cfg.compensate && p->cfg.fixup != ECHO_FIXUP_DEFERRED;
+    const bool own_kernel = p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_SIDE;
     return own_kernel ? 4 : 3;
 }
 

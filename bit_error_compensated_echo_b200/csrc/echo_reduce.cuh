@@ -9,8 +9,13 @@ namespace echo {
 // ------------------------------------------------------------ echo_reduce
 //
 // Reduce-scatter half: for every element, dequantize the P ranks' codes,
-// sum them in fp32 in ascending rank order from +0, requantize the sum,
-// pack it, and (compensating) write e_req = s - float(bf16(k2*scale2)).
+// sum them in fp32 in ascending rank order from +0, requantize the sum and
+// pack it (the reduced transport).  The dequantized sum y = bf16(k2*scale2)
+// is what every rank receives, so on one GPU the kernel can also write it to
+// the n_out outputs itself (OUT), with no second pass over the reduced
+// codes; without OUT that is the exit kernel's job.  Compensating, the output residual e_req = s - float(y) is either
+// written out (for a side-stream or deferred fix-up) or, with fix, folded
+// into the owner's states here (state row o, the owner's own chunk).
 // Each thread owns 16 consecutive elements: one 8-byte word pair of codes
 // per rank, all P loads issued before any arithmetic so that every thread
 // keeps P*8 bytes of the transport in flight.
@@ -72,19 +77,20 @@ __device__ __forceinline__ void sum_run(const uint32_t *__restrict__ codes,
     }
 }
 
-template <int G, int P, bool COMP, int BITS>
+template <int G, int P, bool COMP, bool OUT, int BITS>
 __global__ void __launch_bounds__(kThreads)
 echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
                    uint32_t *__restrict__ rcodes, float *__restrict__ rscales,
                    float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec, Slab sl,
-                   float neg_zero) {
+                   Consts k, const __grid_constant__ OutPtrs out, int n_out,
+                   float *__restrict__ m_fast, float *__restrict__ m_slow, int fix) {
     constexpr int LANES = G / kRedVec;              // lanes per group
     const int o = blockIdx.y;
     const int64_t chunk_run = chunk_vec / 2;        // runs per owner chunk
     const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     const bool valid = local < sl.v_count / 2;
     const int64_t j = (int64_t)o * chunk_run + sl.v_begin / 2 + local;  // run index in a rank
-    const float2 z = splat2(neg_zero);
+    const float2 z = splat2(k.neg_zero);
     float s[16];
     sum_run<G, P, BITS>(codes, scales, n_vec, j, valid, z, s);
 
@@ -105,18 +111,52 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
         reinterpret_cast<uint4 *>(rcodes)[j] =
             make_uint4(w0.w[0], w0.w[BITS / 4 - 1], w1.w[0], w1.w[BITS / 4 - 1]);
     if ((threadIdx.x & (LANES - 1)) == 0) rscales[j / LANES] = scale2;
+    uint32_t yw[8];                                 // y = bf16(k2*scale2), pairs
+    const float2 sc2 = splat2(scale2);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        yw[i] = bf16x2_bits_rn(mul2(make_float2(k2[2 * i], k2[2 * i + 1]), sc2));
+    if (OUT) {
+#pragma unroll
+        for (int r = 0; r < kMaxRanks; ++r) {
+            if (r < n_out) {
+                uint4 *dst = out.p[r] + j * 2;
+                __stcs(dst, make_uint4(yw[0], yw[1], yw[2], yw[3]));
+                __stcs(dst + 1, make_uint4(yw[4], yw[5], yw[6], yw[7]));
+            }
+        }
+    }
     if (COMP) {
         float e[16];
-        const float2 sc2 = splat2(scale2);
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-            const float2 y = bf16x2_to_f32(bf16x2_bits_rn(mul2(make_float2(k2[i], k2[i + 1]), sc2)));
-            const float2 d = sub2(make_float2(s[i], s[i + 1]), y);
-            e[i] = d.x;
-            e[i + 1] = d.y;
+        for (int i = 0; i < 8; ++i) {
+            const float2 d = sub2(make_float2(s[2 * i], s[2 * i + 1]), bf16x2_to_f32(yw[i]));
+            e[2 * i] = d.x;
+            e[2 * i + 1] = d.y;
         }
-        st8(e_req + j * kRedVec, e);
-        st8(e_req + j * kRedVec + 8, e + 8);
+        if (fix) {   // the owner's own states, this run's 16 elements
+            const int64_t e0 = ((int64_t)o * n_vec + j * 2) * kVec;
+            const float2 obf = splat2(k.one_m_beta_fast), obs = splat2(k.one_m_beta_slow);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float mf[8], ms[8];
+                ld8(m_fast + e0 + 8 * h, mf);
+                ld8(m_slow + e0 + 8 * h, ms);
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) {
+                    const float2 e2 = make_float2(e[8 * h + i], e[8 * h + i + 1]);
+                    const float2 f = add2(make_float2(mf[i], mf[i + 1]), prod2(obf, e2, z));
+                    const float2 g = add2(make_float2(ms[i], ms[i + 1]), prod2(obs, e2, z));
+                    mf[i] = f.x; mf[i + 1] = f.y;
+                    ms[i] = g.x; ms[i + 1] = g.y;
+                }
+                st8(m_fast + e0 + 8 * h, mf);
+                st8(m_slow + e0 + 8 * h, ms);
+            }
+        } else {
+            st8(e_req + j * kRedVec, e);
+            st8(e_req + j * kRedVec + 8, e + 8);
+        }
     }
 }
 

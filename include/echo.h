@@ -74,7 +74,8 @@ typedef enum echo_status {
 /* Where the owner's requantization error enters its EMA states (step 7).
  * All three give bit-identical states, outputs and codes. */
 typedef enum echo_fixup_mode {
-    /* inside the exit kernel that writes the outputs */
+    /* inside the kernel that sums and requantizes (the reduce), before the
+     * call returns; e_req is then consumed there and not stored */
     ECHO_FIXUP_EXIT = 0,
     /* in its own kernel on the side stream given to echo_allreduce, so it
      * can run beside the caller's next matrix multiplication (the pages'
@@ -137,6 +138,8 @@ echo_status echo_plan_destroy(echo_plan *plan);
  *   out_device[r] : bf16, N contiguous elements (written with y); may equal
  *                   in_device[r] (in-place)
  *   stream        : stream the entry, reduce and exit kernels run on
+ *                   (uncompensated, the reduce writes the outputs and there
+ *                   is no exit pass)
  *   side_stream   : used with ECHO_FIXUP_SIDE only (the owner fix-up runs
  *                   there after an event on stream); NULL runs the fix-up
  *                   on stream.  Ignored by the other modes.
@@ -169,7 +172,7 @@ echo_status echo_reduce_scatter(echo_plan *plan, const void *const *in_device,
 
 /* The same call on host buffers, pipelined: the call is cut into up to 16
  * slabs (the same sub-range of every owner chunk); each slab's inputs are
- * copied host -> device, its three kernels run, and its outputs are copied
+ * copied host -> device, its kernels run, and its outputs are copied
  * device -> host, on three internal streams, so copies in both directions
  * overlap each other and the kernels.  The staging area (2*P*N*2 bytes) and
  * the internal streams and events are created on first use and kept until
@@ -178,7 +181,7 @@ echo_status echo_reduce_scatter(echo_plan *plan, const void *const *in_device,
  * out_host.  in_host[r], out_host[r]: N bf16 elements each; pinned host
  * memory makes the copies asynchronous, pageable memory makes them
  * synchronous.  Results, codes and states equal echo_allreduce's; with
- * ECHO_FIXUP_SIDE the fix-up runs in the exit kernel here.
+ * ECHO_FIXUP_SIDE the fix-up runs in the reduce kernel here.
  * Errors: INVALID_ARG, OOM (staging), CUDA. */
 echo_status echo_allreduce_host(echo_plan *plan, const void *const *in_host,
                                 void *const *out_host, void *stream);
@@ -225,7 +228,9 @@ typedef struct echo_profile {
     int64_t calls;          /* calls recorded */
     double entry_ms;        /* total time of echo_entry launches */
     double reduce_ms;       /* total time of echo_reduce launches */
-    double exit_ms;         /* total time of echo_exit launches */
+    double exit_ms;         /* total time of echo_exit launches (0 for
+                             * uncompensated calls: the reduce writes the
+                             * outputs) */
     double fixup_ms;        /* total time of side-stream fix-up launches */
     int64_t launches;       /* kernels launched by the recorded calls */
 } echo_profile;
@@ -263,7 +268,7 @@ int32_t echo_launches_per_call(const echo_plan *plan);
  *                                 before the first call, updated in place
  *                                 (ignored, may be NULL, when
  *                                 cfg->compensate == 0)
- *   stream                      : where the three kernels run
+ *   stream                      : where the kernels run
  * The scratch the kernels hand each other (entry codes and scales, the
  * requantized codes and scales and, compensating, e_req) lives in one
  * file-scope device array of ECHO_NOALLOC_MAX_SCRATCH_BYTES, which every
