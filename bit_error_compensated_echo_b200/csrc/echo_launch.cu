@@ -1,6 +1,7 @@
 // echo_launch.cu -- the one translation unit that instantiates the kernels
 // of echo_*.cuh, behind the launchers declared in echo_launch.h.
 #include "echo_entry.cuh"
+#include "echo_entry_raw.cuh"
 #include "echo_exit.cuh"
 #include "echo_fixup.cuh"
 #include "echo_launch.h"
@@ -20,9 +21,16 @@ void entry_t(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chu
 }
 
 template <int G, int BITS>
+void entry_raw_t(const Bufs &b, const InPtrs &x, int rows, Slab sl, cudaStream_t st) {
+    dim3 grid(entry_raw_blocks(sl.v_count), (unsigned)(rows * b.P));
+    echo_entry_raw_kernel<G, BITS><<<grid, kThreads, 0, st>>>(x, b.codes, b.scales, b.n_vec,
+                                                               b.chunk_vec, sl, b.P, b.k);
+}
+
+template <int G, int BITS>
 void entry_g(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er, Slab sl, bool defer,
              cudaStream_t st) {
-    if (!b.comp) entry_t<G, false, false, BITS>(b, x, rows, rank0, er, sl, st);
+    if (!b.comp) entry_raw_t<G, BITS>(b, x, rows, sl, st);
     else if (defer) entry_t<G, true, true, BITS>(b, x, rows, rank0, er, sl, st);
     else entry_t<G, true, false, BITS>(b, x, rows, rank0, er, sl, st);
 }
