@@ -153,9 +153,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str, comp: bool, fixup: str):
+def ncu_traffic(workload: str, comp: bool, fixup: str, bits: int = 4):
     """DRAM bytes per echo_entry launch from the committed ncu summary, if
-    it was captured from the current kernel sources (else None)."""
+    it was captured from the current kernel sources for this workload, mode
+    and code width (else None)."""
     path = os.path.join(ROOT, "profiles", "echo_entry_traffic.md")
     if not os.path.exists(path):
         return None
@@ -164,11 +165,11 @@ def ncu_traffic(workload: str, comp: bool, fixup: str):
     with open(path) as f:
         for line in f:
             if line.startswith("traffic:"):
-                # traffic: <workload> comp=<0|1> fixup=<mode> src=<hash> bytes=<int>
+                # traffic: <workload> comp=<0|1> fixup=<mode> [bits=<4|8>] src=<hash> bytes=<int>
                 parts = line.split()
                 key = " ".join(parts[1:4])
                 kv = dict(p.split("=", 1) for p in parts[4:] if "=" in p)
-                if key == want and kv.get("src") == src:
+                if key == want and kv.get("src") == src and kv.get("bits", "4") == str(bits):
                     return float(kv["bytes"])
     return None
 
@@ -452,7 +453,7 @@ def run_step_mode(args, ws, rank, local):
         achieved = eb / (entry_ms / 1e3) / 1e9
         bmin = (rs_min_bytes(P, N, G, comp, args.bits) if rs
                 else call_min_bytes(P, N, G, comp, args.bits))
-        traffic = ncu_traffic(w.name, comp, fixup)
+        traffic = ncu_traffic(w.name, comp, fixup, args.bits)
         metric = METRIC if comp else METRIC.replace("compensated", "uncompensated")
         if rs:
             metric = metric.replace("reduce input", "reduce-scatter input")
