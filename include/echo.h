@@ -178,9 +178,10 @@ echo_status echo_reduce_scatter(echo_plan *plan, const void *const *in_device,
  * the internal streams and events are created on first use and kept until
  * echo_plan_destroy.  The work starts after everything already queued on
  * stream, and stream waits for its end: synchronize stream before reading
- * out_host.  in_host[r], out_host[r]: N bf16 elements each; pinned host
- * memory makes the copies asynchronous, pageable memory makes them
- * synchronous.  Results, codes and states equal echo_allreduce's; with
+ * out_host.  in_host[r], out_host[r]: N bf16 elements each; out_host[r] may
+ * equal in_host[r] (a slab's outputs are copied back only after its inputs
+ * were copied in, and later slabs read other parts); pinned host memory
+ * makes the copies asynchronous, pageable memory makes them synchronous.  Results, codes and states equal echo_allreduce's; with
  * ECHO_FIXUP_SIDE the fix-up runs in the reduce kernel here.
  * Errors: INVALID_ARG, OOM (staging), CUDA. */
 echo_status echo_allreduce_host(echo_plan *plan, const void *const *in_host,

@@ -233,6 +233,24 @@ def test_host_call_uncompensated_large_slabs():
         assert torch.equal(yd.cpu(), yh)
 
 
+@pytest.mark.parametrize("comp", [True, False])
+def test_host_call_in_place(comp):
+    """The host call with out_host == in_host (the bench's end-to-end leg)
+    gives the device call's outputs and states over a sequence."""
+    w = W.with_size(W.TINY, P=4, rows=1, hidden=4 * 64 * 300, G=64)
+    with _plan(w.P, w.N, w.G, comp, "deferred") as a, _plan(w.P, w.N, w.G, comp, "deferred") as b:
+        for t in range(3):
+            x = W.generate(w, t, DEV)
+            yd = a.allreduce(x)
+            buf = x.cpu().pin_memory()
+            b.allreduce_host(buf, buf)
+            torch.cuda.synchronize()
+            assert torch.equal(yd.cpu().view(torch.int16), buf.view(torch.int16)), t
+        if comp:
+            for sa, sb in zip(a.get_state(), b.get_state()):
+                assert torch.equal(sa.view(torch.int32), sb.view(torch.int32))
+
+
 def test_profile_counts_launches():
     w = W.with_size(W.TINY, P=2, rows=1, hidden=2 * 32 * 64, G=32)
     side = torch.cuda.Stream()
