@@ -118,16 +118,20 @@ void plan_entry(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool de
     launch_entry(p->b, x, p->cfg.P, 0, p->chunk_vec, sl, defer, st);
 }
 
-// The reduce; fix applies the owner fix-up in it.  Uncompensated, it also
-// writes every rank's output (there is no state traffic to hide the extra
-// writes behind, and the merged pass measured 6% faster per call); with the
-// compensator the separate exit pass measured faster.
-void plan_reduce(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    const int n_out = p->cfg.compensate ? 0 : p->cfg.P;
-    launch_reduce(p->b, p->cfg.P, sl, st, &out, n_out, fix);
+// Whether the reduce also writes every rank's output (no exit pass):
+// always uncompensated (no state traffic, the merged pass measured 6% faster
+// per call at 1 GiB per rank), and for small compensated calls.
+bool outputs_in_reduce(const echo_plan *p) {
+    return !p->cfg.compensate || p->cfg.N <= kMergeMaxN;
 }
 
-bool exit_pass(const echo_plan *p) { return p->cfg.compensate != 0; }
+bool exit_pass(const echo_plan *p) { return !outputs_in_reduce(p); }
+
+// The reduce; fix applies the owner fix-up in it.
+void plan_reduce(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
+    const int n_out = outputs_in_reduce(p) ? p->cfg.P : 0;
+    launch_reduce(p->b, p->cfg.P, sl, st, &out, n_out, fix);
+}
 
 void plan_exit(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st) {
     launch_exit(p->b, out, p->cfg.P, p->cfg.P, sl, st);
@@ -254,8 +258,8 @@ echo_status echo_plan_destroy(echo_plan *p) {
 
 int32_t echo_launches_per_call(const echo_plan *p) {
     if (!p) return 0;
-    if (!p->cfg.compensate) return 2;
-    return p->cfg.fixup == ECHO_FIXUP_SIDE ? 4 : 3;
+    const int side = (p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_SIDE) ? 1 : 0;
+    return (exit_pass(p) ? 3 : 2) + side;
 }
 
 echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out, void *stream,

@@ -56,8 +56,11 @@ struct ReduceOut {
 template <int G, int P, int BITS>
 void reduce_t(const Bufs &b, int owners, Slab sl, cudaStream_t st, const ReduceOut &ro) {
     dim3 grid(reduce_blocks(sl.v_count), (unsigned)owners);
-    // compensated reduces never write the outputs (the exit pass does)
-    if (b.comp)
+    if (b.comp && ro.n_out > 0)
+        echo_reduce_kernel<G, P, true, true, BITS><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
+            ro.out, ro.n_out, b.m_fast, b.m_slow, ro.fix);
+    else if (b.comp)
         echo_reduce_kernel<G, P, true, false, BITS><<<grid, kThreads, 0, st>>>(
             b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
             ro.out, 0, b.m_fast, b.m_slow, ro.fix);

@@ -54,11 +54,17 @@ inline Consts make_consts(const echo_config &c) {
 void launch_entry(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chunk_vec,
                   Slab sl, bool defer, cudaStream_t st);
 
-// Reduce of `owners` chunks (grid y): sum the P rows, requantize;
-// uncompensated with n_out > 0 also write the dequantized sum to the n_out
-// outputs (compensated reduces leave that to launch_exit); compensating,
-// either write e_req or, with fix, apply the owner fix-up to state row o
-// of each chunk o.
+// Compensated calls of at most this many elements per rank (1 MiB of bf16)
+// let the reduce write the outputs too, as uncompensated calls always do:
+// there the saved exit launch wins (1 MiB per rank, P=8: 34.6 -> 31.9 us
+// per call); above it the separate exit pass measured faster (4 MiB: +1.5%,
+// 16 MiB: +4% merged).
+constexpr int64_t kMergeMaxN = int64_t(1) << 19;
+
+// Reduce of `owners` chunks (grid y): sum the P rows, requantize; with
+// n_out > 0 also write the dequantized sum to the n_out outputs (else that
+// is launch_exit's job); compensating, either write e_req or, with fix,
+// apply the owner fix-up to state row o of each chunk o.
 void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st,
                    const OutPtrs *out = nullptr, int n_out = 0, bool fix = false);
 

@@ -83,11 +83,11 @@ void launch_all(const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigne
     b.k = make_consts(c);
     const Slab sl{0, b.chunk_vec};
     launch_entry(b, x, c.P, 0, b.chunk_vec, sl, false, st);
-    if (b.comp) {   // owner fix-up in the reduce, outputs in the exit pass
+    if (b.comp && c.N > kMergeMaxN) {   // owner fix-up in the reduce, outputs in the exit
         launch_reduce(b, c.P, sl, st, nullptr, 0, true);
         launch_exit(b, y, c.P, c.P, sl, st);
-    } else {        // the reduce writes the outputs
-        launch_reduce(b, c.P, sl, st, &y, c.P, false);
+    } else {                            // the reduce writes the outputs
+        launch_reduce(b, c.P, sl, st, &y, c.P, b.comp);
     }
 }
 

@@ -138,8 +138,8 @@ echo_status echo_plan_destroy(echo_plan *plan);
  *   out_device[r] : bf16, N contiguous elements (written with y); may equal
  *                   in_device[r] (in-place)
  *   stream        : stream the entry, reduce and exit kernels run on
- *                   (uncompensated, the reduce writes the outputs and there
- *                   is no exit pass)
+ *                   (uncompensated, or compensated with N <= 2^19, the
+ *                   reduce writes the outputs and there is no exit pass)
  *   side_stream   : used with ECHO_FIXUP_SIDE only (the owner fix-up runs
  *                   there after an event on stream); NULL runs the fix-up
  *                   on stream.  Ignored by the other modes.
@@ -229,9 +229,9 @@ typedef struct echo_profile {
     int64_t calls;          /* calls recorded */
     double entry_ms;        /* total time of echo_entry launches */
     double reduce_ms;       /* total time of echo_reduce launches */
-    double exit_ms;         /* total time of echo_exit launches (0 for
-                             * uncompensated calls: the reduce writes the
-                             * outputs) */
+    double exit_ms;         /* total time of echo_exit launches (0 when the
+                             * reduce writes the outputs: uncompensated
+                             * calls, compensated calls with N <= 2^19) */
     double fixup_ms;        /* total time of side-stream fix-up launches */
     int64_t launches;       /* kernels launched by the recorded calls */
 } echo_profile;

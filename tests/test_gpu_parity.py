@@ -251,11 +251,16 @@ def test_host_call_in_place(comp):
                 assert torch.equal(sa.view(torch.int32), sb.view(torch.int32))
 
 
-def test_profile_counts_launches():
-    w = W.with_size(W.TINY, P=2, rows=1, hidden=2 * 32 * 64, G=32)
+@pytest.mark.parametrize("N", [2 * 32 * 64, 1 << 20], ids=["small", "large"])
+def test_profile_counts_launches(N):
+    """Entry, reduce and (compensated calls above 2^19 elements per rank)
+    exit, plus the side-stream fix-up; the reduce writes the outputs
+    otherwise."""
+    w = W.with_size(W.TINY, P=2, rows=1, hidden=N, G=32)
     side = torch.cuda.Stream()
-    for comp, mode, per in ((True, "exit", 3), (True, "side", 4), (True, "deferred", 3),
-                            (False, "exit", 2)):
+    for comp, mode in ((True, "exit"), (True, "side"), (True, "deferred"), (False, "exit")):
+        exit_pass = comp and N > (1 << 19)
+        per = 2 + int(exit_pass) + int(comp and mode == "side")
         with _plan(w.P, w.N, w.G, comp, mode) as plan:
             assert plan.launches_per_call() == per
             plan.profile_enable(True)
@@ -264,7 +269,7 @@ def test_profile_counts_launches():
             p = plan.profile_read(reset=True)
             assert p["calls"] == 3 and p["launches"] == 3 * per
             assert p["entry_ms"] > 0 and p["reduce_ms"] > 0
-            if comp:          # uncompensated, the reduce writes the outputs: no exit pass
+            if exit_pass:
                 assert p["exit_ms"] > 0
 
 
