@@ -332,3 +332,26 @@ def test_large_1gib_per_rank(comp, calls):
         assert all(torch.equal(out[0], out[r]) for r in range(1, w.P))
         del x, out
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("comp", [True, False], ids=["comp", "off"])
+def test_message_beyond_int32_elements(comp):
+    """P=2 ranks of 2^31 + 1024 elements each (4 GiB of bf16 per rank):
+    every index of every kernel is past 32 bits somewhere; 2048 sampled
+    group columns plus the first and the last, two calls."""
+    from bench import BENCH_FIXUP
+    N = (1 << 31) + 1024
+    w = W.with_size(W.LARGE, P=2, rows=1, hidden=N, G=128)
+    cols = W.column_sample(w, 2048)
+    assert cols.max() * w.G >= (1 << 31)
+    with _plan(w.P, w.N, w.G, comp, BENCH_FIXUP) as plan:
+        chk = SequenceChecker(plan, oracle_params(plan), cols)
+        x = torch.empty((w.P, w.N), dtype=torch.bfloat16, device=DEV)
+        out = torch.empty_like(x)
+        for t in range(2):
+            W.generate(w, t, DEV, out=x)
+            chk.step(x, out=out)
+        assert torch.equal(out[0], out[1])
+        del x, out
+    torch.cuda.empty_cache()
+
