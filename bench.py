@@ -274,7 +274,7 @@ def aggregate(per_rank_ms, per_rank_bytes):
 # ------------------------------------------------------------ CPU baseline
 
 def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: int = 7,
-                      bits: int = 4):
+                      bits: int = 4, op: str = "all-reduce"):
     """Time the oracle (as it stands, one host thread) on ``ncols`` group
     columns of workload ``w``; inputs are the device inputs at those columns
     when given, else a host draw of the same distribution."""
@@ -290,8 +290,9 @@ def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: i
     prm = oracle.Params(P=w.P, N=w.N, G=w.G, compensate=comp, bits=bits)
     mf = np.zeros((w.P, idx.size), np.float32)
     ms = np.zeros_like(mf)
+    call = oracle.reduce_scatter if op == "reduce-scatter" else oracle.allreduce
     t0 = time.perf_counter()
-    oracle.allreduce(prm, xb, mf, ms, cols)
+    call(prm, xb, mf, ms, cols)
     dt = time.perf_counter() - t0
     nbytes = 2 * w.P * idx.size
     return nbytes / dt / 1e9, dt, cols.size
@@ -352,6 +353,32 @@ def oracle_parallel_run(w: W.Workload, comp: bool, ncols: int, x_dev, bits: int 
 
 
 # ------------------------------------------------------------ modes
+
+def metric_of(comp: bool, rs: bool, bits: int) -> str:
+    """The step line's metric for this mode (the headline one by default)."""
+    metric = METRIC if comp else METRIC.replace("compensated", "uncompensated")
+    if rs:
+        metric = metric.replace("reduce input", "reduce-scatter input")
+    if bits == 8:
+        metric = metric.replace("4-bit", "8-bit")
+    return metric
+
+
+def dtypes_of(bits: int) -> dict:
+    """The types the path moves and computes in (the line's dtype is the
+    arithmetic one, f32)."""
+    return {"inputs_outputs": "bf16", "transport": "int%d codes + f32 group scales" % bits,
+            "sums_states_residuals": "f32"}
+
+
+def step_config(args, w: W.Workload, comp: bool, fixup: str, ws: int) -> dict:
+    """The workload of a step line, the same for both arms."""
+    return {"workload": w.name, "op": args.op, "bits": args.bits, "P": w.P, "N_per_rank": w.N,
+            "G": w.G, "compensate": comp, "fixup": fixup, "alpha": 0.5, "beta_fast": 0.5,
+            "beta_slow": 0.95,
+            "l2": "inputs larger than L2 (%.1f GiB of x per step)" % (2 * w.P * w.N / 2**30),
+            "parallelism": "replicas" if ws > 1 else "1 GPU"}
+
 
 def run_step_mode(args, ws, rank, local):
     from bit_error_compensated_echo_b200.api import EchoPlan
@@ -456,22 +483,15 @@ def run_step_mode(args, ws, rank, local):
         bmin = (rs_min_bytes(P, N, G, comp, args.bits) if rs
                 else call_min_bytes(P, N, G, comp, args.bits))
         traffic = ncu_traffic(w.name, comp, fixup, args.bits)
-        metric = METRIC if comp else METRIC.replace("compensated", "uncompensated")
-        if rs:
-            metric = metric.replace("reduce input", "reduce-scatter input")
-        if args.bits == 8:
-            metric = metric.replace("4-bit", "8-bit")
+        metric = metric_of(comp, rs, args.bits)
         line = {
             "metric": metric,
             "value": round(value, 3), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, int4 transport, f32 sum+state",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "dtypes": dtypes_of(args.bits),
             "data": "synthetic (seeded N(0,0.5^2) bf16 draws, no dataset)",
-            "config": {"workload": w.name, "op": args.op, "bits": args.bits, "P": P,
-                       "N_per_rank": N, "G": G,
-                       "compensate": comp, "fixup": fixup, "alpha": 0.5, "beta_fast": 0.5,
-                       "beta_slow": 0.95, "l2": "inputs larger than L2 (%.1f GiB of x per step)"
-                       % (2 * P * N / 2**30), "parallelism": "replicas" if ws > 1 else "1 GPU"},
+            "config": step_config(args, w, comp, fixup, ws),
             "call_roofline": {"min_bytes": bmin, "achieved_gbs": round(bmin / (ms / 1e3) / 1e9, 1),
                               "peak": peak, "frac": round(bmin / (ms / 1e3) / 1e9 / peak, 4),
                               "time_at_peak_ms": round(bmin / peak / 1e6, 3)},
@@ -495,10 +515,11 @@ def run_reference(args, ws, rank):
     w = WORKLOADS[args.workload]
     comp = not args.uncompensated
     for i in range(args.warmup):
-        oracle_sample_run(w, comp, args.ref_cols, seed=100 + i)
+        oracle_sample_run(w, comp, args.ref_cols, seed=100 + i, bits=args.bits, op=args.op)
     times, nbytes = [], 0
     for i in range(args.steps):
-        gbs, dt, ncols = oracle_sample_run(w, comp, args.ref_cols, seed=1000 + i)
+        gbs, dt, ncols = oracle_sample_run(w, comp, args.ref_cols, seed=1000 + i,
+                                           bits=args.bits, op=args.op)
         times.append(dt)
         nbytes = 2 * w.P * ncols * w.G
     ms = 1e3 * sum(times) / len(times)
@@ -506,13 +527,12 @@ def run_reference(args, ws, rank):
     sample = ("%d of %d group columns (x %d ranks x G=%d) per step, host draw of the same "
               "distribution, one call from zero state" % (args.ref_cols + 2, w.N // w.G, w.P, w.G))
     line = {
-        "metric": METRIC if comp else METRIC.replace("compensated", "uncompensated"),
+        "metric": metric_of(comp, args.op == "reduce-scatter", args.bits),
         "value": round(value, 6), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, int4 transport, f32 sum+state",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "dtypes": dtypes_of(args.bits),
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": w.name, "P": w.P, "N_per_rank": w.N, "G": w.G,
-                   "compensate": comp},
+        "config": step_config(args, w, comp, args.fixup, ws),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
