@@ -329,8 +329,11 @@ def oracle_parallel_run(w: W.Workload, comp: bool, ncols: int, x_dev, bits: int 
     workers = workers or len(os.sched_getaffinity(0))
     cols = W.column_sample(w, ncols, seed=7)
     idx = W.column_elements(cols, w.G)
-    ti = torch.from_numpy(idx).to(x_dev.device)
-    xb = W.bf16_bits(x_dev.index_select(1, ti))
+    if x_dev is not None:
+        ti = torch.from_numpy(idx).to(x_dev.device)
+        xb = W.bf16_bits(x_dev.index_select(1, ti))
+    else:   # a host draw of the same distribution, only the sampled columns
+        xb = W.bf16_bits(W.generate(W.with_size(w, rows=1, hidden=idx.size), 0, "cpu"))
     shm = shared_memory.SharedMemory(create=True, size=xb.nbytes)
     try:
         np.ndarray(xb.shape, dtype=np.uint16, buffer=shm.buf)[:] = xb
@@ -761,6 +764,32 @@ def run_group_mode(args, ws, rank, local):
         dist.destroy_process_group()
 
 
+def run_cpu_mode(args, ws, rank, local):
+    """The oracle, as it stands, on the host cores for each configuration:
+    one call (the tiny workload whole, the others on a sample of group
+    columns), on one thread and split by group columns over all cores.
+    Prints one JSON line per configuration."""
+    if rank != 0:
+        return
+    cases = [(W.TINY, None), (W.LLAMA, 65536), (W.DEPTH, 65536), (W.LARGE, 262144)]
+    for w, ncols in cases:
+        # the tiny workload whole; the others: only the sampled columns are drawn
+        x = W.generate(w, 0, "cpu") if ncols is None else None
+        n = ncols - 2 if ncols else w.N // w.G
+        gbs1, dt1, c1 = oracle_sample_run(w, True, n, x_dev=x)
+        gbs_all, dt_all, nw = oracle_parallel_run(w, True, n, x, reps=3)
+        elems = w.P * c1 * w.G
+        print(json.dumps({
+            "mode": "cpu", "workload": w.name, "kind": "oracle", "group_columns": c1,
+            "of_columns": w.N // w.G, "rank_elements": elems,
+            "one_thread": {"seconds": round(dt1, 4), "ns_per_rank_element": round(dt1 / elems * 1e9, 2),
+                           "input_gbs": round(gbs1, 5)},
+            "all_cores": {"cores": nw, "seconds": round(dt_all, 4),
+                          "ns_per_rank_element": round(dt_all / elems * 1e9, 3),
+                          "input_gbs": round(gbs_all, 5)}}), flush=True)
+        del x
+
+
 def run_depth_chain_mode(args, ws, rank, local):
     """Deviation from the exact fp32 chain per site, forward and backward."""
     from bit_error_compensated_echo_b200 import depth_chain
@@ -789,7 +818,7 @@ def main(argv=None):
     ap.add_argument("--uncompensated", action="store_true")
     ap.add_argument("--op", choices=("all-reduce", "reduce-scatter"), default="all-reduce")
     ap.add_argument("--bits", type=int, choices=(4, 8), default=4)
-    ap.add_argument("--mode", choices=("step", "depth-chain", "sweep", "overlap", "group"),
+    ap.add_argument("--mode", choices=("step", "depth-chain", "sweep", "overlap", "group", "cpu"),
                     default="step")
     ap.add_argument("--sweep-max-mib", type=int, default=0,
                     help="sweep only points up to this many MiB per rank (0: all)")
@@ -819,6 +848,8 @@ def main(argv=None):
             run_overlap_mode(args, ws, rank, local)
         elif args.mode == "group":
             run_group_mode(args, ws, rank, local)
+        elif args.mode == "cpu":
+            run_cpu_mode(args, ws, rank, local)
         else:
             run_step_mode(args, ws, rank, local)
     finally:
