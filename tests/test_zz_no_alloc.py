@@ -35,8 +35,9 @@ def _check_same(got_bits, want_bits, what):
     assert np.array_equal(got_bits, want_bits), what
 
 
+# N above and below 2^19 per rank: the call with and without the exit pass
 @pytest.mark.parametrize("P,G,k,comp", [(8, 128, 70, True), (3, 32, 41, True),
-                                        (4, 64, 33, False)])
+                                        (4, 64, 33, False), (8, 128, 600, True)])
 def test_noalloc_matches_plan_two_calls(P, G, k, comp):
     N = P * G * k
     w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
