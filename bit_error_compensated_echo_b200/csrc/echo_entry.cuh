@@ -21,9 +21,11 @@ namespace echo {
 //   VPT   : vectors per thread.  A block covers kThreads*VPT vectors; thread t
 //           takes vectors t, t + kThreads, ... so each load instruction of a
 //           warp is contiguous, and all of a thread's input and state loads
-//           are issued before any arithmetic: the bytes in flight per SM grow
-//           with VPT, which is what bounds the uncompensated pass (2.5 bytes
-//           per element).
+//           are issued before any arithmetic.  One vector per thread (62
+//           registers, 4 blocks per SM) measured faster than two (80
+//           registers, 3 blocks) at every size from 1 MiB to 1 GiB per rank:
+//           2.4 % per call at 1 GiB, 3-4 % at 4-16 MiB (finer blocks also
+//           leave a smaller last wave).
 // x is a __grid_constant__ parameter: the block's rank selects its pointer
 // straight from the parameter bank.  Indexing a by-value array parameter
 // with a run-time index otherwise copies the whole array to every thread's
@@ -31,8 +33,8 @@ namespace echo {
 // launch), which measured 7% of the entry's time.
 template <bool COMP>
 struct EntryShape {
-    static constexpr int VPT = COMP ? 2 : 4;
-    static constexpr int MIN_BLOCKS = COMP ? 3 : 4;  // resident blocks per SM (register cap)
+    static constexpr int VPT = COMP ? 1 : 4;
+    static constexpr int MIN_BLOCKS = 4;  // resident blocks per SM (register cap)
 };
 
 template <bool COMP>
