@@ -54,6 +54,11 @@ Layout layout_of(const echo_config &c) {
     return L;
 }
 
+// Slabs of the pipelined host call: copies in, kernels and copies out of
+// successive slabs overlap, and only the first slab's copy in and the last
+// one's copy out are not hidden.
+constexpr int kHostSlabs = 32;
+
 struct ProfRecord {
     cudaEvent_t ev[6];   // entry start, entry end, reduce end, exit end, fixup start, fixup end
     bool side;
@@ -92,7 +97,7 @@ struct echo_plan {
     cudaEvent_t ev_reduced = nullptr, ev_side_done = nullptr;
     void *stage = nullptr;           // host-call staging: [P][N] in, [P][N] out
     cudaStream_t hstream[3] = {nullptr, nullptr, nullptr};  // host call: copy in, compute, copy out
-    cudaEvent_t hev[2 * 16 + 2] = {};                       // host call: per-slab and boundary events
+    cudaEvent_t hev[2 * kHostSlabs + 2] = {};               // host call: per-slab and boundary events
     bool profiling = false;
     std::vector<ProfRecord> records;
     std::vector<cudaEvent_t> pool;
@@ -438,7 +443,7 @@ echo_status echo_allreduce_host(echo_plan *p, const void *const *in_host, void *
     }
     cudaStream_t st = (cudaStream_t)stream;
     cudaStream_t s_in = p->hstream[0], s_comp = p->hstream[1], s_out = p->hstream[2];
-    cudaEvent_t ev_start = p->hev[32], ev_done = p->hev[33];
+    cudaEvent_t ev_start = p->hev[2 * kHostSlabs], ev_done = p->hev[2 * kHostSlabs + 1];
 
     InPtrs xi{};
     OutPtrs yo{};
@@ -454,7 +459,7 @@ echo_status echo_allreduce_host(echo_plan *p, const void *const *in_host, void *
     // Slab k is vectors [k*sv, (k+1)*sv) of every owner chunk: one strided
     // copy per rank moves it (P rows of sv*16 bytes, pitch chunk_vec*16).
     const int64_t align = p->cfg.G / kVec;  // slab edges on group edges (and even)
-    int64_t nslab = 16;
+    int64_t nslab = kHostSlabs;
     if (p->chunk_vec / align < nslab) nslab = p->chunk_vec / align;
     int64_t sv = (p->chunk_vec + nslab - 1) / nslab;
     sv = (sv + align - 1) / align * align;

@@ -170,7 +170,7 @@ echo_status echo_reduce_scatter(echo_plan *plan, const void *const *in_device,
                                 void *const *out_device, void *stream,
                                 void *side_stream);
 
-/* The same call on host buffers, pipelined: the call is cut into up to 16
+/* The same call on host buffers, pipelined: the call is cut into up to 32
  * slabs (the same sub-range of every owner chunk); each slab's inputs are
  * copied host -> device, its kernels run, and its outputs are copied
  * device -> host, on three internal streams, so copies in both directions
