@@ -13,7 +13,8 @@ namespace echo {
 //   COMP  : compensator on (read/write the states)
 //   DEFER : apply the previous call's pending owner fix-up first
 //           (state += (1-beta)*e_req on this rank's own chunk), which is the
-//           same fp32 operation the exit kernel would have done.
+//           same fp32 operation the reduce kernel would have done in the
+//           "exit" fix-up mode.
 // The kernel serves the P virtual ranks of one plan (grid y = P*P, rank0 = 0,
 // e_req holding every owner chunk: er_chunk_vec = chunk_vec) and one rank of
 // a group spread over processes (grid y = P, rank0 = that rank's index, e_req

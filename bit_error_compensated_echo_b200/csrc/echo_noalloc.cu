@@ -98,7 +98,7 @@ extern "C" echo_status echo_allreduce_noalloc(const echo_config *cfg, const void
                                               float *m_slow_device, void *stream) {
     if (!cfg || !in_device || !out_device) return ECHO_ERR_INVALID_ARG;
     echo_config c = *cfg;
-    c.fixup = ECHO_FIXUP_EXIT;   // the fix-up always runs in the exit kernel here
+    c.fixup = ECHO_FIXUP_EXIT;   // the fix-up always runs before the call returns here
     const echo_status v = validate_config(&c);
     if (v != ECHO_OK) return v;
     if (cfg->device >= kMaxDevices) return ECHO_ERR_INVALID_ARG;

@@ -13,7 +13,8 @@ namespace echo {
 // pack it (the reduced transport).  The dequantized sum y = bf16(k2*scale2)
 // is what every rank receives, so on one GPU the kernel can also write it to
 // the n_out outputs itself (OUT), with no second pass over the reduced
-// codes; without OUT that is the exit kernel's job.  Compensating, the output residual e_req = s - float(y) is either
+// codes; without OUT that is the exit kernel's job.  Compensating, the
+// output residual e_req = s - float(y) is either
 // written out (for a side-stream or deferred fix-up) or, with fix, folded
 // into the owner's states here (state row o, the owner's own chunk).
 // Each thread owns 16 consecutive elements: one 8-byte word pair of codes
