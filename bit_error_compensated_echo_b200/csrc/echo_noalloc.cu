@@ -1,6 +1,6 @@
 // echo_noalloc.cu -- echo_allreduce_noalloc: the same call as
-// echo_allreduce (fix-up inside the exit kernel), for callers that cannot
-// allocate device memory.  The scratch the three kernels pass between each
+// echo_allreduce (owner fix-up inside the reduce kernel), for callers that
+// cannot allocate device memory.  The scratch the kernels pass between each
 // other (entry codes and scales, the requantized codes and scales, e_req)
 // lives in one file-scope device array instead of a plan's workspace, and
 // the caller owns the compensator state.  Nothing here calls cudaMalloc,

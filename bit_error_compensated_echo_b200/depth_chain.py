@@ -1,10 +1,10 @@
 """Synthetic depth chain: how the all-reduce's error accumulates over sites.
 
-The pages claim the accumulated error stays bounded independently of depth
-when each injected rounding error is fed back into later calls, under the
-assumption that the network does not keep amplifying a perturbation along
-one direction (arXiv abstract on the fugumt mirror; ai4snews news summary,
-"Interpretation" and "Perspective").  This harness measures that on a
+The pages claim that, with every rounding error carried into the calls that
+follow, the total error has a bound that does not grow with the number of
+layers, provided the network has no direction along which it keeps
+magnifying a perturbation (arXiv abstract on the fugumt mirror; ai4snews
+news summary, "Interpretation" and "Perspective").  This harness measures that on a
 synthetic pre-norm residual chain of tensor-parallel sites, each followed
 by the all-reduce of the P ranks' partial products:
 
@@ -18,7 +18,7 @@ amplify perturbations, which is the bound's assumption.  Five chains run
 side by side: the exact chain (fp32 partials summed in fp32), the
 compensated 4-bit all-reduce, the uncompensated one, a bf16 all-reduce
 (bf16 partials summed in fp32, rounded to bf16), and "promoted": the
-compensated all-reduce under the pages' serving policy, the first half of
+compensated all-reduce under the pages' serving policy, the earlier half of
 the layers (two sites each) at 8-bit codes and the rest at 4 bits, on one
 state (ai4snews news summary, "Perspective").  Per site it reports the
 absolute RMS deviation from the exact chain and the relative Frobenius

@@ -1,6 +1,6 @@
 """Per-layer code width: which all-reduce calls run at 8 bits.
 
-The pages' serving policy for Llama-3-8B promotes the first half of the
+The pages' serving policy for Llama-3-8B promotes the earlier half of the
 layers to 8-bit codes, which recovers most of the accuracy that 4 bits
 loses there (ai4snews news summary, "Perspective").  The pages give the
 fraction and the direction (the early layers) but no other rule, so the

@@ -5,15 +5,15 @@
  * arXiv 2610.14277).
  *
  * What one call computes (sources, by page and section):
- *  - ai4snews news summary, "Interpretation", paragraph 1: the all-reduce
- *    moves 4-bit integer values and sums them in high precision.
- *  - arXiv abstract (fugumt mirror), "Abstract": each value is quantized at
- *    most twice per call for any number of ranks; the sum reveals the error
- *    it injects and the error is fed back into later calls.
+ *  - ai4snews news summary, "Interpretation", paragraph 1: the values cross
+ *    between ranks as 4-bit integers and are added at high precision.
+ *  - arXiv abstract (fugumt mirror), "Abstract": no value is rounded more
+ *    than twice in a call whatever the number of ranks; the rounding error
+ *    that the sum exposes is carried into the calls that follow.
  *  - ai4snews news summary, "Interpretation", paragraph 2: the compensator
- *    is two moving averages with different decay rates; a correction is
- *    added to the input before each all-reduce and the averages are
- *    refreshed from the output residual.
+ *    is a fast and a slow exponential moving average; a weighted mix of the
+ *    two is added to each input before quantization, and both are updated
+ *    from the residual of the output.
  *
  * Per call, for P ranks of N elements each, group size G:
  *   1. c_r  = alpha*m_fast_r + (1-alpha)*m_slow_r;  xt_r = float(x_r) + c_r
@@ -79,7 +79,7 @@ typedef enum echo_fixup_mode {
     ECHO_FIXUP_EXIT = 0,
     /* in its own kernel on the side stream given to echo_allreduce, so it
      * can run beside the caller's next matrix multiplication (the pages'
-     * "update running beside the next matmul"); the next call on the plan
+     * arrangement: the update overlaps the next matrix multiplication); the next call on the plan
      * waits for it */
     ECHO_FIXUP_SIDE = 1,
     /* kept pending in the plan and folded into the next call's entry pass,
@@ -99,7 +99,7 @@ typedef struct echo_config {
     int32_t fixup;      /* echo_fixup_mode */
     int32_t bits;       /* code width: 4 (levels -7..7, two codes per byte) or
                          * 8 (levels -127..127, one code per byte; the
-                         * pages' serving policy promotes the first half of
+                         * pages' serving policy promotes the earlier half of
                          * the layers to 8 bits, ai4snews "Perspective").
                          * The widest width of the plan's calls: the
                          * transport is sized for it, and a plan with
@@ -240,7 +240,7 @@ echo_status echo_profile_enable(echo_plan *plan, int32_t on);
 echo_status echo_profile_read(echo_plan *plan, echo_profile *out, int32_t reset);
 
 /* Code width of the plan's following calls: 4, or 8 when cfg.bits == 8
- * (per-call promotion: the pages' serving policy runs the first half of the
+ * (per-call promotion: the pages' serving policy runs the earlier half of the
  * layers at 8 bits, ai4snews news summary, "Perspective").  Every width
  * shares the plan's one compensator state and any pending fix-up: the
  * state and e_req are fp32 whatever the width.  Takes effect for calls made

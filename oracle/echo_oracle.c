@@ -17,15 +17,16 @@
  * Sources for each step (page title + section):
  *  - ai4snews news summary, "Interpretation" paragraph 1: the all-reduce is
  *    replaced by 4-bit integer transport plus a high-precision sum.
- *  - ai4snews news summary, "Interpretation" paragraph 2: two moving averages
- *    with different decay rates; a correction is added to the input before
- *    each all-reduce; the averages are refreshed from the output residual;
- *    the sum reveals the rounding error just injected.
- *  - arXiv abstract (fugumt mirror, "Abstract"): data moves in 4 bits, is
- *    summed in high precision, and each value is quantized at most twice per
- *    call for any number of GPUs (reduce-scatter, requantize, all-gather).
+ *  - ai4snews news summary, "Interpretation" paragraph 2: the compensator is
+ *    a pair of exponential moving averages, one fast and one slow; a weighted
+ *    mix of the two is added to each input before it is quantized; both are
+ *    then updated from the residual of the output, which the sum exposes.
+ *  - arXiv abstract (fugumt mirror, "Abstract"): codes travel at 4 bits and
+ *    are added at high precision, and no value is rounded more than twice in
+ *    a call whatever the number of GPUs (reduce-scatter, requantize,
+ *    all-gather).
  *  - heraldofai explainer, "How Echo keeps errors from snowballing": the
- *    same "rounded at most twice" statement.
+ *    same bound of two roundings per value.
  * The pages fix no constants, no scale format and no rounding rule; the
  * readings taken here (symmetric absmax int4 with levels -7..7, fp32 scale
  * per group of G contiguous elements, round half to even, requantization

@@ -3,8 +3,8 @@ deviation from the exact fp32 chain stays bounded over 56 sites; without it
 the deviation keeps growing (Qwen3-0.6B-like shape: P=8, 32768 tokens x
 1024 hidden, Student-t nu=3 inputs, Haar-orthogonal site maps, RMSNorm).
 
-The pages state the accumulated error stays bounded independently of depth
-under a no-persistent-amplification assumption (arXiv abstract on the
+The pages state that the total error has a bound that does not grow with
+the number of layers, if no direction is magnified again and again (arXiv abstract on the
 fugumt mirror; ai4snews news summary, "Perspective"); orthogonal maps and
 RMSNorm satisfy that assumption.  This is a property check, not a parity
 check: the all-reduce inside it is the parity-tested library.
@@ -44,7 +44,7 @@ def test_backward_deviation_smaller_with_compensation(chain):
 
 
 def test_layer_policy_promotion(chain):
-    """The serving policy (first half of the layers at 8 bits, one state;
+    """The serving policy (the earlier half of the layers at 8 bits, one state;
     ai4snews news summary, "Perspective"): forward, the 8-bit half stays far
     below the 4-bit chain and the end of the chain is well below it;
     backward runs the 4-bit layers first, so the promoted chain equals the
