@@ -173,7 +173,8 @@ class EchoPlan:
         abi.echo_reset_state(self.handle, _stream_handle(stream, self.device))
 
     def get_state(self, stream=None):
-        """(m_fast, m_slow) as new [P, N] fp32 tensors (pending fix-up applied)."""
+        """(m_fast, m_slow) as new [P, N] fp32 tensors (pending fix-up applied;
+        in deferred mode e_req is -0, a no-op, when none is pending)."""
         mf = torch.empty((self.P, self.N), dtype=torch.float32, device=self.device)
         ms = torch.empty_like(mf)
         abi.echo_get_state(self.handle, mf.data_ptr(), ms.data_ptr(),

@@ -92,7 +92,7 @@ struct echo_plan {
     float *m_fast = nullptr, *m_slow = nullptr, *scales = nullptr, *rscales = nullptr,
           *e_req = nullptr;
     uint32_t *codes = nullptr, *rcodes = nullptr;
-    bool pending = false;            // deferred fix-up not yet applied
+    bool pending = false;            // a deferred-mode call ran since the last reset (host view)
     bool side_inflight = false;      // a side-stream fix-up may still run
     cudaEvent_t ev_reduced = nullptr, ev_side_done = nullptr;
     void *stage = nullptr;           // host-call staging: [P][N] in, [P][N] out
@@ -230,7 +230,10 @@ echo_status echo_plan_create(echo_plan **out, const echo_config *cfg) {
     if (e == cudaSuccess && comp) {
         e = cudaMemset(p->m_fast, 0, (size_t)cfg->P * cfg->N * 4);
         if (e == cudaSuccess) e = cudaMemset(p->m_slow, 0, (size_t)cfg->P * cfg->N * 4);
-        if (e == cudaSuccess) e = cudaMemset(p->e_req, 0, (size_t)cfg->N * 4);
+        if (e == cudaSuccess) {
+            launch_fill(p->e_req, cfg->N, kNoFixup, nullptr);
+            e = cudaGetLastError();
+        }
     }
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
@@ -294,6 +297,11 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
     cudaStream_t side = (cudaStream_t)side_stream;
     const bool comp = p->cfg.compensate != 0;
     const int mode = p->cfg.fixup;
+    // Under stream capture: a side-stream fix-up leaves in the graph an event
+    // that the plan's next call would wait on, and profiling keeps per-call
+    // events on the host; replays would honour neither.
+    if (capturing(st) && (p->profiling || (comp && mode == ECHO_FIXUP_SIDE && side)))
+        return ECHO_ERR_UNSUPPORTED;
 
     ProfRecord rec{};
     rec.kernels = exit_pass(p) ? 3 : 2;
@@ -306,7 +314,7 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
     }
 
     ECHO_TRY(order_after_side(p, st));
-    const bool defer = comp && mode == ECHO_FIXUP_DEFERRED && p->pending;
+    const bool defer = comp && mode == ECHO_FIXUP_DEFERRED;   // e_req is -0 if none pending
 
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[0], st));
     plan_entry(p, xi, whole(p), st, defer);
@@ -373,6 +381,11 @@ echo_status echo_reduce_scatter(echo_plan *p, const void *const *in, void *const
     cudaStream_t side = (cudaStream_t)side_stream;
     const bool comp = p->cfg.compensate != 0;
     const int mode = p->cfg.fixup;
+    // Under stream capture: a side-stream fix-up leaves in the graph an event
+    // that the plan's next call would wait on, and profiling keeps per-call
+    // events on the host; replays would honour neither.
+    if (capturing(st) && (p->profiling || (comp && mode == ECHO_FIXUP_SIDE && side)))
+        return ECHO_ERR_UNSUPPORTED;
 
     ProfRecord rec{};
     rec.kernels = 2;
@@ -383,7 +396,7 @@ echo_status echo_reduce_scatter(echo_plan *p, const void *const *in, void *const
         }
     }
     ECHO_TRY(order_after_side(p, st));
-    const bool defer = comp && mode == ECHO_FIXUP_DEFERRED && p->pending;
+    const bool defer = comp && mode == ECHO_FIXUP_DEFERRED;   // e_req is -0 if none pending
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[0], st));
     plan_entry(p, xi, whole(p), st, defer);
     ECHO_TRY(cudaGetLastError());
@@ -428,6 +441,8 @@ echo_status echo_allreduce_host(echo_plan *p, const void *const *in_host, void *
         if (!in_host[r] || !out_host[r]) return ECHO_ERR_INVALID_ARG;
     DeviceGuard guard(p->cfg.device);
     if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    // host copies on internal streams, allocated on first use: not for capture
+    if (capturing((cudaStream_t)stream)) return ECHO_ERR_UNSUPPORTED;
     const size_t bytes = (size_t)p->cfg.N * 2;
     if (!p->stage) {
         cudaError_t e = cudaMalloc(&p->stage, 2 * (size_t)P * bytes);
@@ -471,7 +486,7 @@ echo_status echo_allreduce_host(echo_plan *p, const void *const *in_host, void *
     p->side_inflight = false;
     const bool comp = p->cfg.compensate != 0;
     const bool deferred = comp && p->cfg.fixup == ECHO_FIXUP_DEFERRED;
-    const bool defer = deferred && p->pending;
+    const bool defer = deferred;   // e_req is -0 if none pending
     for (int64_t k = 0; k < nslab; ++k) {
         const int64_t vb = k * sv;
         if (vb >= p->chunk_vec) break;
@@ -509,6 +524,8 @@ echo_status echo_reset_state(echo_plan *p, void *stream) {
     const size_t bytes = (size_t)p->cfg.P * p->cfg.N * 4;
     ECHO_TRY(cudaMemsetAsync(p->m_fast, 0, bytes, st));
     ECHO_TRY(cudaMemsetAsync(p->m_slow, 0, bytes, st));
+    launch_fill(p->e_req, p->cfg.N, kNoFixup, st);
+    ECHO_TRY(cudaGetLastError());
     p->pending = false;
     return ECHO_OK;
 }
@@ -520,7 +537,10 @@ echo_status echo_get_state(echo_plan *p, float *m_fast, float *m_slow, void *str
     if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     ECHO_TRY(order_after_side(p, st));
-    plan_fixup(p, p->m_fast, p->m_slow, m_fast, m_slow, p->pending, false, whole(p), st);
+    // deferred mode: e_req holds the pending fix-up, or -0 (a no-op) if none is
+    // pending; applying it unconditionally is right after graph replays too
+    const bool apply = p->cfg.fixup == ECHO_FIXUP_DEFERRED;
+    plan_fixup(p, p->m_fast, p->m_slow, m_fast, m_slow, apply, false, whole(p), st);
     ECHO_TRY(cudaGetLastError());
     return ECHO_OK;
 }
@@ -534,6 +554,8 @@ echo_status echo_set_state(echo_plan *p, const float *m_fast, const float *m_slo
     const size_t bytes = (size_t)p->cfg.P * p->cfg.N * 4;
     ECHO_TRY(cudaMemcpyAsync(p->m_fast, m_fast, bytes, cudaMemcpyDeviceToDevice, st));
     ECHO_TRY(cudaMemcpyAsync(p->m_slow, m_slow, bytes, cudaMemcpyDeviceToDevice, st));
+    launch_fill(p->e_req, p->cfg.N, kNoFixup, st);
+    ECHO_TRY(cudaGetLastError());
     p->pending = false;
     return ECHO_OK;
 }

@@ -36,6 +36,17 @@ inline echo_status from_cuda(cudaError_t e) {
 inline bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
 inline bool aligned4(const void *ptr) { return ((uintptr_t)ptr & 3u) == 0; }
 
+// Whether st is capturing into a CUDA graph (false if the query fails: the
+// launches that follow then report the error).
+inline bool capturing(cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return cs != cudaStreamCaptureStatusNone;
+}
+
 }  // namespace echo
 
 #define ECHO_TRY(expr)                                     \

@@ -184,6 +184,13 @@ void launch_rs(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix,
     else rs_b<4>(b, out, owners, sl, fix, st);
 }
 
+void launch_fill(float *p, int64_t n, float v, cudaStream_t st) {
+    int64_t blocks = (n + kThreads - 1) / kThreads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    echo_fill_kernel<<<(unsigned)blocks, kThreads, 0, st>>>(p, n, v);
+}
+
 void launch_fixup(const Bufs &b, const float *src_fast, const float *src_slow, float *dst_fast,
                   float *dst_slow, int ranks, int owners, bool apply, bool only_owner, Slab sl,
                   cudaStream_t st) {

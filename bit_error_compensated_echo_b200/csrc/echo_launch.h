@@ -47,6 +47,12 @@ inline Consts make_consts(const echo_config &c) {
     return k;
 }
 
+// The e_req value of "no fix-up pending" (see echo_fill_kernel).
+constexpr float kNoFixup = -0.0f;
+
+// p[0..n) = v on st.
+void launch_fill(float *p, int64_t n, float v, cudaStream_t st);
+
 // Entry over `rows` input rows (grid y = rows * P chunks).  rank0: index of
 // row 0 in the group (the owner test for the deferred fix-up);
 // er_chunk_vec: vectors between consecutive owners' e_req chunks (0 when

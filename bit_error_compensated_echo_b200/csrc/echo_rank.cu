@@ -35,7 +35,6 @@ struct echo_rank_plan {
     Consts k{};
     char *ws = nullptr;
     float *m_fast = nullptr, *m_slow = nullptr, *e_req = nullptr;
-    bool pending = false;        // deferred fix-up not yet folded into an entry
     bool entered = false;        // an entry ran since the last reduce
     bool side_inflight = false;  // a side-stream fix-up may still run
     cudaEvent_t ev_reduced = nullptr, ev_side_done = nullptr;
@@ -87,8 +86,7 @@ void own_chunk_fixup(echo_rank_plan *p, const float *src_f, const float *src_s, 
 echo_status after_reduce(echo_rank_plan *p, cudaStream_t st, cudaStream_t side, bool in_kernel) {
     if (!p->cfg.compensate) return ECHO_OK;
     switch (p->cfg.fixup) {
-        case ECHO_FIXUP_DEFERRED:
-            p->pending = true;
+        case ECHO_FIXUP_DEFERRED:   // e_req now holds it; the next entry applies it
             return ECHO_OK;
         case ECHO_FIXUP_EXIT:
             if (!in_kernel) {
@@ -164,6 +162,10 @@ echo_status echo_rank_plan_create(echo_rank_plan **out, const echo_config *cfg, 
         p->m_slow = (float *)(p->ws + align_up((size_t)cfg->N * 4));
         p->e_req = (float *)(p->ws + 2 * align_up((size_t)cfg->N * 4));
         e = cudaMemset(p->ws, 0, bytes);
+        if (e == cudaSuccess && p->cfg.compensate) {
+            launch_fill(p->e_req, p->C, kNoFixup, nullptr);
+            e = cudaGetLastError();
+        }
     }
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_reduced, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ev_side_done, cudaEventDisableTiming);
@@ -196,7 +198,8 @@ echo_status echo_rank_entry(echo_rank_plan *p, const void *x, void *send_codes,
     if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
     ECHO_TRY(order_after_side(p, st));
-    const bool defer = p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_DEFERRED && p->pending;
+    // e_req is -0 (a no-op) when no fix-up is pending
+    const bool defer = p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_DEFERRED;
 
     Bufs b = base_bufs(p);
     b.m_fast = p->m_fast;
@@ -209,7 +212,6 @@ echo_status echo_rank_entry(echo_rank_plan *p, const void *x, void *send_codes,
     xi.p[0] = (const uint4 *)x;
     launch_entry(b, xi, 1, p->rank, 0, chunk_slab(p), defer, st);
     ECHO_TRY(cudaGetLastError());
-    p->pending = false;
     p->entered = true;
     return ECHO_OK;
 }
@@ -225,6 +227,10 @@ echo_status echo_rank_reduce(echo_rank_plan *p, const void *recv_codes, const fl
     DeviceGuard guard(p->cfg.device);
     if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
+    // a side-stream fix-up under capture leaves in the graph an event that the
+    // plan's next call would wait on
+    if (side_stream && p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_SIDE && capturing(st))
+        return ECHO_ERR_UNSUPPORTED;
 
     Bufs b = base_bufs(p);
     b.codes = (uint32_t *)recv_codes;
@@ -274,6 +280,10 @@ echo_status echo_rank_reduce_scatter(echo_rank_plan *p, const void *recv_codes,
     DeviceGuard guard(p->cfg.device);
     if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
     cudaStream_t st = (cudaStream_t)stream;
+    // a side-stream fix-up under capture leaves in the graph an event that the
+    // plan's next call would wait on
+    if (side_stream && p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_SIDE && capturing(st))
+        return ECHO_ERR_UNSUPPORTED;
     const bool fix = p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_EXIT;
 
     Bufs b = base_bufs(p);
@@ -305,7 +315,8 @@ echo_status echo_rank_reset_state(echo_rank_plan *p, void *stream) {
     const size_t bytes = (size_t)p->cfg.N * 4;
     ECHO_TRY(cudaMemsetAsync(p->m_fast, 0, bytes, st));
     ECHO_TRY(cudaMemsetAsync(p->m_slow, 0, bytes, st));
-    p->pending = false;
+    launch_fill(p->e_req, p->C, kNoFixup, st);
+    ECHO_TRY(cudaGetLastError());
     return ECHO_OK;
 }
 
@@ -319,7 +330,7 @@ echo_status echo_rank_get_state(echo_rank_plan *p, float *m_fast, float *m_slow,
     const size_t bytes = (size_t)p->cfg.N * 4;
     ECHO_TRY(cudaMemcpyAsync(m_fast, p->m_fast, bytes, cudaMemcpyDeviceToDevice, st));
     ECHO_TRY(cudaMemcpyAsync(m_slow, p->m_slow, bytes, cudaMemcpyDeviceToDevice, st));
-    if (p->pending) {
+    if (p->cfg.fixup == ECHO_FIXUP_DEFERRED) {   // -0 in e_req when none is pending
         own_chunk_fixup(p, m_fast, m_slow, m_fast, m_slow, st);
         ECHO_TRY(cudaGetLastError());
     }
@@ -337,7 +348,8 @@ echo_status echo_rank_set_state(echo_rank_plan *p, const float *m_fast, const fl
     const size_t bytes = (size_t)p->cfg.N * 4;
     ECHO_TRY(cudaMemcpyAsync(p->m_fast, m_fast, bytes, cudaMemcpyDeviceToDevice, st));
     ECHO_TRY(cudaMemcpyAsync(p->m_slow, m_slow, bytes, cudaMemcpyDeviceToDevice, st));
-    p->pending = false;
+    launch_fill(p->e_req, p->C, kNoFixup, st);
+    ECHO_TRY(cudaGetLastError());
     p->entered = false;
     return ECHO_OK;
 }

@@ -82,8 +82,13 @@ typedef enum echo_fixup_mode {
      * arrangement: the update overlaps the next matrix multiplication); the next call on the plan
      * waits for it */
     ECHO_FIXUP_SIDE = 1,
-    /* kept pending in the plan and folded into the next call's entry pass,
-     * which reads the state anyway (fewest HBM bytes) */
+    /* kept pending in e_req and folded into the next call's entry pass,
+     * which reads the state anyway (fewest HBM bytes).  e_req holds -0.0f
+     * whenever no fix-up is pending (after plan creation, echo_reset_state
+     * and echo_set_state), and m + (1-beta)*(-0) = m exactly, so every
+     * entry applies e_req: no host-side flag selects the kernels a call
+     * launches, and a captured graph replays correctly (see "Stream
+     * capture" below) */
     ECHO_FIXUP_DEFERRED = 2
 } echo_fixup_mode;
 
@@ -152,6 +157,20 @@ echo_status echo_allreduce(echo_plan *plan, const void *const *in_device,
                            void *const *out_device, void *stream,
                            void *side_stream);
 
+/* Stream capture.  echo_allreduce and echo_reduce_scatter only launch
+ * kernels (and, with a side stream, record and wait on events); they
+ * allocate nothing and never synchronize, so they may be captured into a
+ * CUDA graph on stream.  A replay runs the captured kernels on the plan's
+ * current state and buffers, exactly as the same eager calls would, in the
+ * EXIT and DEFERRED modes, whatever calls, replays or state resets came
+ * before it, and in ECHO_FIXUP_SIDE mode without a side stream.  A capture
+ * fixes the buffers and the code width (echo_plan_set_bits).  Refused with
+ * UNSUPPORTED while stream is capturing: a call with profiling on (its
+ * events are kept per call on the host), a side-stream fix-up (it leaves in
+ * the graph an event that the plan's next call would wait on), and
+ * echo_allreduce_host (host copies on internal streams).  echo_reset_state,
+ * echo_get_state and echo_set_state capture too (copies and kernels). */
+
 /* One reduce-scatter over the P ranks: the reduce-scatter of sequence
  * parallelism, which the pages name as a next target for the same scheme
  * (ai4snews news summary, "Perspective").  Steps 1-4 as for
@@ -188,7 +207,8 @@ echo_status echo_allreduce_host(echo_plan *plan, const void *const *in_host,
                                 void *const *out_host, void *stream);
 
 /* Zero the compensator state (m_fast = m_slow = 0) and drop any pending
- * deferred fix-up, on stream.  A no-op (ECHO_OK) when compensate == 0. */
+ * deferred fix-up (e_req = -0), on stream.  A no-op (ECHO_OK) when
+ * compensate == 0. */
 echo_status echo_reset_state(echo_plan *plan, void *stream);
 
 /* Copy the current states, with any pending deferred fix-up applied, into
@@ -199,7 +219,7 @@ echo_status echo_get_state(echo_plan *plan, float *m_fast_device,
                            float *m_slow_device, void *stream);
 
 /* Overwrite the states from caller device buffers ([P][N] fp32) and drop
- * any pending fix-up, on stream (checkpoint restore, tests).
+ * any pending fix-up (e_req = -0), on stream (checkpoint restore, tests).
  * Errors: INVALID_ARG (null, or compensate == 0), CUDA. */
 echo_status echo_set_state(echo_plan *plan, const float *m_fast_device,
                            const float *m_slow_device, void *stream);
@@ -215,7 +235,9 @@ typedef struct echo_debug_view {
     uint8_t *rcodes;    /* [N*bits/8] requantized sum codes */
     float *rscales;     /* [N/G] requantization scales */
     float *e_req;       /* [N] requantization error, or NULL */
-    int32_t fixup_pending; /* 1 if a deferred fix-up is pending */
+    int32_t fixup_pending; /* 1 if a deferred-mode call ran since the last
+                              reset or restore (host view: graph replays
+                              do not change it) */
     int32_t bits;       /* code width of the calls (echo_plan_set_bits) */
 } echo_debug_view;
 

@@ -83,7 +83,9 @@ echo_status echo_rank_plan_create(echo_rank_plan **out, const echo_config *cfg, 
 echo_status echo_rank_plan_destroy(echo_rank_plan *plan);
 
 /* Steps 1-3 on this rank's input, writing the send buffers.  With
- * ECHO_FIXUP_DEFERRED the previous call's owner fix-up is folded in first.
+ * ECHO_FIXUP_DEFERRED the entry first applies the owner fix-up held in the
+ * plan's e_req: the previous reduce's, or -0.0f (an exact no-op) when none
+ * is pending (after plan creation, reset_state and set_state).
  *   x_device       : bf16, N elements of this rank (read)
  *   send_codes     : [P][cb] bytes (written)
  *   send_scales    : [P][cs] fp32 (written)
@@ -92,14 +94,14 @@ echo_status echo_rank_entry(echo_rank_plan *plan, const void *x_device, void *se
                             float *send_scales_device, void *stream);
 
 /* Steps 4-5 for this rank's chunk, from the received buffers, writing the
- * reduced codes and scales that the all-gather distributes, and keeping
- * e_req in the plan.  Step 7 by the plan's fix-up mode: EXIT runs it here on
- * stream after the reduce, SIDE on side_stream (NULL: on stream; the plan's
- * next call waits for it), DEFERRED folds it into the next entry.
+ * reduced codes and scales that the all-gather distributes.  Step 7 by the
+ * plan's fix-up mode: EXIT applies it inside the reduce kernel, SIDE keeps
+ * e_req and runs it in its own kernel on side_stream (NULL: on stream; the
+ * plan's next call waits for it), DEFERRED keeps e_req for the next entry.
  *   recv_codes, recv_scales : [P][cb] bytes, [P][cs] fp32 (read)
  *   red_codes, red_scales   : [cb] bytes, [cs] fp32 (written)
  * Must follow an echo_rank_entry on the plan (a second reduce without a new
- * entry would apply the fix-up twice).  One kernel, two with the fix-up.
+ * entry would apply the fix-up twice).  One kernel, two in SIDE mode.
  * Errors: INVALID_ARG (null, or no entry since the last reduce),
  * ALIGNMENT, CUDA. */
 echo_status echo_rank_reduce(echo_rank_plan *plan, const void *recv_codes_device,
@@ -123,8 +125,8 @@ echo_status echo_rank_reduce_scatter(echo_rank_plan *plan, const void *recv_code
                                      const float *recv_scales_device, void *out_device,
                                      void *stream, void *side_stream);
 
-/* Zero this rank's state and drop a pending fix-up, on stream (a no-op when
- * compensate == 0). */
+/* Zero this rank's state and drop a pending fix-up (e_req = -0), on stream
+ * (a no-op when compensate == 0). */
 echo_status echo_rank_reset_state(echo_rank_plan *plan, void *stream);
 
 /* Copy this rank's states ([N] fp32 each), with a pending fix-up applied,
@@ -134,7 +136,16 @@ echo_status echo_rank_get_state(echo_rank_plan *plan, float *m_fast_device,
                                 float *m_slow_device, void *stream);
 
 /* Overwrite this rank's states from caller device buffers ([N] fp32 each)
- * and drop a pending fix-up.  Errors as echo_rank_get_state. */
+ * and drop a pending fix-up (e_req = -0).  Errors as echo_rank_get_state.
+ *
+ * Stream capture: every call above only launches kernels, copies on the
+ * device and (with a side stream) records and waits on events, so a whole
+ * rank call -- stages and the caller's exchanges -- may be captured into a
+ * CUDA graph, with the same rules as echo_allreduce (include/echo.h): a
+ * reduce or reduce-scatter with a side-stream fix-up returns UNSUPPORTED
+ * while stream is capturing.  The host-side order check of
+ * echo_rank_reduce applies when the calls are captured, not when the graph
+ * is replayed. */
 echo_status echo_rank_set_state(echo_rank_plan *plan, const float *m_fast_device,
                                 const float *m_slow_device, void *stream);
 
