@@ -689,11 +689,14 @@ def run_group_mode(args, ws, rank, local):
     """The rank path over NCCL: this process is rank ``rank`` of a group of
     ws ranks; per step one EchoRankPlan.allreduce (entry, all-to-all of the
     packed chunks, reduce, all-gather, exit), timed with CUDA events between
-    barriers, max over ranks; then NCCL's bf16 all-reduce of the same input,
-    timed the same way."""
+    barriers, max over ranks; then the same call over the fused transport
+    (allreduce_peers: the entry stores into the owners' windows, the exit
+    loads from them, two one-element NCCL all-reduces as barriers), and
+    NCCL's bf16 all-reduce of the same input, timed the same way."""
     import torch.distributed as dist
 
-    from bit_error_compensated_echo_b200.rank import EchoRankPlan, TorchDistTransport
+    from bit_error_compensated_echo_b200.rank import (EchoRankPlan, PeerWindows,
+                                                      TorchDistBarrier, TorchDistTransport)
     if ws == 1 and not dist.is_initialized():
         import datetime
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
@@ -729,6 +732,9 @@ def run_group_mode(args, ws, rank, local):
         return times
 
     echo_fn = lambda: plan.allreduce(x, transport, out=out)  # noqa: E731
+    win = PeerWindows.exchange(plan)
+    barrier = TorchDistBarrier(dev)
+    peers_fn = lambda: plan.allreduce_peers(x, win, barrier, out=out)  # noqa: E731
     y = x.clone()
     nccl_fn = lambda: dist.all_reduce(y)  # noqa: E731
     timed(echo_fn, max(args.warmup, 3))
@@ -737,10 +743,18 @@ def run_group_mode(args, ws, rank, local):
         sampler.start()
     t_echo = timed(echo_fn, args.steps)
     clocks = sampler.stop() if sampler else None
+    timed(peers_fn, max(args.warmup, 3))
+    t_peers = timed(peers_fn, args.steps)
     timed(nccl_fn, max(args.warmup, 3))
     t_nccl = timed(nccl_fn, args.steps)
     ms_echo = max_over_ranks(statistics.median(t_echo), ws, dev)
+    ms_peers = max_over_ranks(statistics.median(t_peers), ws, dev)
     ms_nccl = max_over_ranks(statistics.median(t_nccl), ws, dev)
+    # no rank unmaps, and no owner frees, a window a peer may still read
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    win.close()
+    dist.barrier()
     wire = plan.bufs.wire_bytes()
     if rank == 0:
         line = {
@@ -757,6 +771,12 @@ def run_group_mode(args, ws, rank, local):
                        "transport": "torch.distributed NCCL all_to_all_single + "
                        "all_gather_into_tensor"},
             "gpu_launches_per_call": plan.launches_per_call(), "clocks": clocks,
+            "fused_transport": {
+                "ms_per_call": round(ms_peers, 4),
+                "value": round(2.0 * P * N / (ms_peers / 1e3) / 1e9, 3),
+                "speedup_vs_nccl_bf16": round(ms_nccl / ms_peers, 3),
+                "transport": "entry stores into the owners' windows, exit loads from them "
+                "(CUDA IPC), two one-element NCCL all-reduces as barriers"},
         }
         print(json.dumps(line), flush=True)
     plan.close()

@@ -54,6 +54,16 @@ class echo_debug_view(ctypes.Structure):
                 ("bits", ctypes.c_int32)]
 
 
+class echo_rank_window_layout(ctypes.Structure):
+    _fields_ = [("base", ctypes.c_void_p), ("bytes", ctypes.c_size_t),
+                ("recv_codes", ctypes.c_size_t), ("recv_scales", ctypes.c_size_t),
+                ("red_codes", ctypes.c_size_t), ("red_scales", ctypes.c_size_t)]
+
+
+class echo_ipc_handle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_uint8 * 64)]
+
+
 class echo_profile(ctypes.Structure):
     _fields_ = [("calls", ctypes.c_int64), ("entry_ms", ctypes.c_double),
                 ("reduce_ms", ctypes.c_double), ("exit_ms", ctypes.c_double),
@@ -105,6 +115,13 @@ def _load():
         "echo_rank_set_state": (st, [vp, vp, vp, vp]),
         "echo_rank_launches_per_call": (ctypes.c_int32, [vp]),
         "echo_rank_plan_set_bits": (st, [vp, ctypes.c_int32]),
+        "echo_rank_window": (st, [vp, ctypes.POINTER(echo_rank_window_layout)]),
+        "echo_rank_entry_peers": (st, [vp, vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp]),
+        "echo_rank_exit_peers": (st, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, vp]),
+        "echo_ipc_handle_get": (st, [vp, ctypes.POINTER(echo_ipc_handle)]),
+        "echo_ipc_open": (st, [ctypes.POINTER(echo_ipc_handle), ctypes.c_int32,
+                               ctypes.POINTER(vp)]),
+        "echo_ipc_close": (st, [vp, ctypes.c_int32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -269,6 +286,52 @@ def echo_rank_exit(plan: int, all_codes_device: int, all_scales_device: int, out
                    stream: int = 0) -> None:
     _check(lib.echo_rank_exit(plan, all_codes_device, all_scales_device, out_device,
                               stream or None), "echo_rank_exit")
+
+
+def echo_rank_window(plan: int) -> dict:
+    """The plan's window (allocated on first use): base, bytes and the byte
+    offsets recv_codes, recv_scales, red_codes, red_scales."""
+    L = echo_rank_window_layout()
+    _check(lib.echo_rank_window(plan, ctypes.byref(L)), "echo_rank_window")
+    return {"base": int(L.base or 0), "bytes": int(L.bytes), "recv_codes": int(L.recv_codes),
+            "recv_scales": int(L.recv_scales), "red_codes": int(L.red_codes),
+            "red_scales": int(L.red_scales)}
+
+
+def echo_rank_entry_peers(plan: int, x_device: int, recv_codes_peers: Sequence[int],
+                          recv_scales_peers: Sequence[int], stream: int = 0) -> None:
+    _check(lib.echo_rank_entry_peers(plan, x_device, _ptr_array(recv_codes_peers),
+                                     _ptr_array(recv_scales_peers), stream or None),
+           "echo_rank_entry_peers")
+
+
+def echo_rank_exit_peers(plan: int, red_codes_peers: Sequence[int],
+                         red_scales_peers: Sequence[int], out_device: int,
+                         stream: int = 0) -> None:
+    _check(lib.echo_rank_exit_peers(plan, _ptr_array(red_codes_peers),
+                                    _ptr_array(red_scales_peers), out_device, stream or None),
+           "echo_rank_exit_peers")
+
+
+def echo_ipc_handle_get(device_ptr: int) -> bytes:
+    """The 64-byte CUDA IPC handle of the allocation holding device_ptr."""
+    h = echo_ipc_handle()
+    _check(lib.echo_ipc_handle_get(device_ptr, ctypes.byref(h)), "echo_ipc_handle_get")
+    return bytes(h.bytes)
+
+
+def echo_ipc_open(handle: bytes, device: int) -> int:
+    """Map another process's allocation (its handle) into this one; returns
+    the base address."""
+    h = echo_ipc_handle()
+    ctypes.memmove(h.bytes, handle, 64)
+    out = ctypes.c_void_p()
+    _check(lib.echo_ipc_open(ctypes.byref(h), device, ctypes.byref(out)), "echo_ipc_open")
+    return int(out.value)
+
+
+def echo_ipc_close(ptr: int, device: int) -> None:
+    _check(lib.echo_ipc_close(ptr, device), "echo_ipc_close")
 
 
 def echo_rank_reduce_scatter(plan: int, recv_codes_device: int, recv_scales_device: int,

@@ -34,6 +34,24 @@ struct OutPtrs {
     uint4 *p[kMaxRanks];
 };
 
+// Where the entry puts owner chunk o's packed codes and scales: codes[o]
+// and scales[o] hold the chunk's first vector and first group of row 0
+// (row r follows at r rows of n_vec vectors).  One buffer of every chunk
+// back to back is the case codes[o] = base + o chunk sizes; the rank path
+// may instead point codes[o] into rank o's receive buffer, in another
+// GPU's memory.
+struct ChunkDst {
+    uint8_t *codes[kMaxRanks];
+    float *scales[kMaxRanks];
+};
+
+// Where the exit reads owner o's reduced chunk (codes[o], scales[o]: its
+// first vector and group), in this GPU's memory or in owner o's.
+struct ChunkSrc {
+    const uint8_t *codes[kMaxRanks];
+    const float *scales[kMaxRanks];
+};
+
 // A slab: the vectors [v_begin, v_begin + v_count) of every owner chunk
 // (a vector is 8 elements; owner chunk o is vectors [o*chunk_vec,
 // (o+1)*chunk_vec) of every rank).  A whole call is the slab (0, chunk_vec);

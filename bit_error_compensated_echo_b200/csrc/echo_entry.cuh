@@ -18,7 +18,10 @@ namespace echo {
 // The kernel serves the P virtual ranks of one plan (grid y = P*P, rank0 = 0,
 // e_req holding every owner chunk: er_chunk_vec = chunk_vec) and one rank of
 // a group spread over processes (grid y = P, rank0 = that rank's index, e_req
-// holding its own chunk only: er_chunk_vec = 0).
+// holding its own chunk only: er_chunk_vec = 0).  Chunk o's codes and scales
+// go to dst.codes[o] / dst.scales[o] (ChunkDst): one local buffer, or, on the
+// rank path, rank o's receive buffer on its GPU, so that the quantized chunk
+// crosses NVLink as the kernel writes it.
 //   VPT   : vectors per thread.  A block covers kThreads*VPT vectors; thread t
 //           takes vectors t, t + kThreads, ... so each load instruction of a
 //           warp is contiguous, and all of a thread's input and state loads
@@ -47,7 +50,7 @@ inline unsigned entry_blocks(int64_t v_count) {
 template <int G, bool COMP, bool DEFER, int BITS>
 __global__ void __launch_bounds__(kThreads, EntryShape<COMP>::MIN_BLOCKS)
 echo_entry_kernel(const __grid_constant__ InPtrs x, float *__restrict__ m_fast, float *__restrict__ m_slow,
-                  uint32_t *__restrict__ codes, float *__restrict__ scales,
+                  const __grid_constant__ ChunkDst dst,
                   const float *__restrict__ e_req, int64_t n_vec, int64_t chunk_vec,
                   Slab sl, int P, Consts k, int rank0, int64_t er_chunk_vec) {
     constexpr int LANES = G / kVec;
@@ -128,9 +131,10 @@ echo_entry_kernel(const __grid_constant__ InPtrs x, float *__restrict__ m_fast, 
         }
         if (!valid[v]) continue;
 
-        store_packed8<BITS>(codes, (int64_t)r * n_vec + j[v], w);
+        const int64_t vc = sl.v_begin + base + (int64_t)v * kThreads;   // vector in chunk o
+        store_packed8<BITS>(reinterpret_cast<uint32_t *>(dst.codes[o]), (int64_t)r * n_vec + vc, w);
         if ((threadIdx.x & (LANES - 1)) == 0)
-            scales[(int64_t)r * (n_vec / LANES) + j[v] / LANES] = scale;
+            dst.scales[o][(int64_t)r * (n_vec / LANES) + vc / LANES] = scale;
 
         if (COMP) {
             const float2 s2 = splat2(scale);

@@ -16,6 +16,8 @@ namespace echo {
 // threads (G = 32: one thread, no exchange), and the thread's 4 code words
 // (8 for 8-bit codes) leave in one (two) 16-byte store.  The 4 loads of a
 // warp are 64 bytes apart per lane; together they read whole lines.
+// Chunk o's codes and scales go to dst.codes[o] / dst.scales[o], as in the
+// compensated entry.
 // Grid: x over the slab's vectors / (4 * kThreads), y = rank * P + chunk.
 constexpr int kRawVPT = 4;
 
@@ -26,15 +28,15 @@ inline unsigned entry_raw_blocks(int64_t v_count) {
 
 template <int G, int BITS>
 __global__ void __launch_bounds__(kThreads)
-echo_entry_raw_kernel(const __grid_constant__ InPtrs x, uint32_t *__restrict__ codes,
-                      float *__restrict__ scales, int64_t n_vec, int64_t chunk_vec, Slab sl,
-                      int P, Consts k) {
+echo_entry_raw_kernel(const __grid_constant__ InPtrs x, const __grid_constant__ ChunkDst dst,
+                      int64_t n_vec, int64_t chunk_vec, Slab sl, int P, Consts k) {
     constexpr int VPG = G / kVec;            // vectors per group: 4, 8 or 16
     constexpr int TPG = VPG / kRawVPT;       // threads per group: 1, 2 or 4
     const int r = blockIdx.y / P, o = blockIdx.y % P;
     const int64_t t = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     const bool valid = t < sl.v_count / kRawVPT;
-    const int64_t j0 = (int64_t)o * chunk_vec + sl.v_begin + t * kRawVPT;  // first vector
+    const int64_t vc = sl.v_begin + t * kRawVPT;          // first vector, in chunk o
+    const int64_t j0 = (int64_t)o * chunk_vec + vc;         // first vector, in rank r
     const float2 z = splat2(k.neg_zero);
 
     float v[kRawVPT][8];
@@ -60,15 +62,16 @@ echo_entry_raw_kernel(const __grid_constant__ InPtrs x, uint32_t *__restrict__ c
     for (int q = 0; q < kRawVPT; ++q) w[q] = quantize8_q<BITS>(v[q], gs, kf, z);
     if (!valid) return;
 
-    uint4 *dst = reinterpret_cast<uint4 *>(codes + ((int64_t)r * n_vec + j0) * (BITS / 4));
+    uint4 *cd = reinterpret_cast<uint4 *>(reinterpret_cast<uint32_t *>(dst.codes[o]) +
+                                          ((int64_t)r * n_vec + vc) * (BITS / 4));
     if (BITS == 4) {
-        dst[0] = make_uint4(w[0].w[0], w[1].w[0], w[2].w[0], w[3].w[0]);
+        cd[0] = make_uint4(w[0].w[0], w[1].w[0], w[2].w[0], w[3].w[0]);
     } else {
-        dst[0] = make_uint4(w[0].w[0], w[0].w[BITS / 4 - 1], w[1].w[0], w[1].w[BITS / 4 - 1]);
-        dst[1] = make_uint4(w[2].w[0], w[2].w[BITS / 4 - 1], w[3].w[0], w[3].w[BITS / 4 - 1]);
+        cd[0] = make_uint4(w[0].w[0], w[0].w[BITS / 4 - 1], w[1].w[0], w[1].w[BITS / 4 - 1]);
+        cd[1] = make_uint4(w[2].w[0], w[2].w[BITS / 4 - 1], w[3].w[0], w[3].w[BITS / 4 - 1]);
     }
     if ((threadIdx.x & (TPG - 1)) == 0)
-        scales[(int64_t)r * (n_vec / VPG) + j0 / VPG] = gs.scale;
+        dst.scales[o][(int64_t)r * (n_vec / VPG) + vc / VPG] = gs.scale;
 }
 
 }  // namespace echo

@@ -10,22 +10,25 @@ namespace echo {
 //
 // All-gather half: dequantize the reduced codes once to bf16 and write them
 // to n_out outputs (all P ranks' on one GPU, this process's one across
-// GPUs).  Uncompensated calls on one GPU skip it: their reduce kernel writes
-// the outputs itself.
+// GPUs).  Owner o's reduced chunk is read from src.codes[o] / src.scales[o]
+// (ChunkSrc): one local buffer, or, on the rank path, owner o's own buffer
+// on its GPU, so that the all-gather is these loads.  Uncompensated calls
+// on one GPU skip the kernel: their reduce writes the outputs itself.
 // Grid: x over the vectors of the slab, y = owner.
 template <int G, int BITS>
 __global__ void __launch_bounds__(kThreads)
-echo_exit_kernel(const uint32_t *__restrict__ rcodes, const float *__restrict__ rscales,
-                 const __grid_constant__ OutPtrs out, int n_out, int64_t chunk_vec, Slab sl) {
+echo_exit_kernel(const __grid_constant__ ChunkSrc src, const __grid_constant__ OutPtrs out,
+                 int n_out, int64_t chunk_vec, Slab sl) {
     constexpr int LANES = G / kVec;
     const int o = blockIdx.y;
     const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (local >= sl.v_count) return;
-    const int64_t j = (int64_t)o * chunk_vec + sl.v_begin + local;
+    const int64_t vc = sl.v_begin + local;                  // vector in chunk o
+    const int64_t j = (int64_t)o * chunk_vec + vc;          // vector in the output
 
     uint32_t w[BITS / 4];
-    load_packed8<BITS>(rcodes, j, w);
-    const float2 sc2 = splat2(__ldg(rscales + j / LANES));
+    load_packed8<BITS>(reinterpret_cast<const uint32_t *>(src.codes[o]), vc, w);
+    const float2 sc2 = splat2(__ldg(src.scales[o] + vc / LANES));
     float2 kp[4];
     decode_pairs<BITS, 4>(w, kp);
     uint32_t yw[4];

@@ -13,35 +13,36 @@ namespace {
 // ---- entry
 template <int G, bool COMP, bool DEFER, int BITS>
 void entry_t(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chunk_vec, Slab sl,
-             cudaStream_t st) {
+             cudaStream_t st, const ChunkDst &dst) {
     dim3 grid(entry_blocks<COMP>(sl.v_count), (unsigned)(rows * b.P));
     echo_entry_kernel<G, COMP, DEFER, BITS><<<grid, kThreads, 0, st>>>(
-        x, b.m_fast, b.m_slow, b.codes, b.scales, b.e_req, b.n_vec, b.chunk_vec, sl, b.P, b.k,
-        rank0, er_chunk_vec);
+        x, b.m_fast, b.m_slow, dst, b.e_req, b.n_vec, b.chunk_vec, sl, b.P, b.k, rank0,
+        er_chunk_vec);
 }
 
 template <int G, int BITS>
-void entry_raw_t(const Bufs &b, const InPtrs &x, int rows, Slab sl, cudaStream_t st) {
+void entry_raw_t(const Bufs &b, const InPtrs &x, int rows, Slab sl, cudaStream_t st,
+                 const ChunkDst &dst) {
     dim3 grid(entry_raw_blocks(sl.v_count), (unsigned)(rows * b.P));
-    echo_entry_raw_kernel<G, BITS><<<grid, kThreads, 0, st>>>(x, b.codes, b.scales, b.n_vec,
-                                                               b.chunk_vec, sl, b.P, b.k);
+    echo_entry_raw_kernel<G, BITS><<<grid, kThreads, 0, st>>>(x, dst, b.n_vec, b.chunk_vec, sl,
+                                                               b.P, b.k);
 }
 
 template <int G, int BITS>
 void entry_g(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er, Slab sl, bool defer,
-             cudaStream_t st) {
-    if (!b.comp) entry_raw_t<G, BITS>(b, x, rows, sl, st);
-    else if (defer) entry_t<G, true, true, BITS>(b, x, rows, rank0, er, sl, st);
-    else entry_t<G, true, false, BITS>(b, x, rows, rank0, er, sl, st);
+             cudaStream_t st, const ChunkDst &dst) {
+    if (!b.comp) entry_raw_t<G, BITS>(b, x, rows, sl, st, dst);
+    else if (defer) entry_t<G, true, true, BITS>(b, x, rows, rank0, er, sl, st, dst);
+    else entry_t<G, true, false, BITS>(b, x, rows, rank0, er, sl, st, dst);
 }
 
 template <int BITS>
 void entry_b(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er, Slab sl, bool defer,
-             cudaStream_t st) {
+             cudaStream_t st, const ChunkDst &dst) {
     switch (b.G) {
-        case 32: entry_g<32, BITS>(b, x, rows, rank0, er, sl, defer, st); break;
-        case 64: entry_g<64, BITS>(b, x, rows, rank0, er, sl, defer, st); break;
-        default: entry_g<128, BITS>(b, x, rows, rank0, er, sl, defer, st); break;
+        case 32: entry_g<32, BITS>(b, x, rows, rank0, er, sl, defer, st, dst); break;
+        case 64: entry_g<64, BITS>(b, x, rows, rank0, er, sl, defer, st, dst); break;
+        default: entry_g<128, BITS>(b, x, rows, rank0, er, sl, defer, st, dst); break;
     }
 }
 
@@ -99,18 +100,19 @@ void reduce_b(const Bufs &b, int owners, Slab sl, cudaStream_t st, const ReduceO
 
 // ---- exit
 template <int G, int BITS>
-void exit_g(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, cudaStream_t st) {
+void exit_g(const ChunkSrc &src, int64_t chunk_vec, const OutPtrs &out, int n_out, int owners,
+            Slab sl, cudaStream_t st) {
     dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)owners);
-    echo_exit_kernel<G, BITS><<<grid, kThreads, 0, st>>>(b.rcodes, b.rscales, out, n_out,
-                                                          b.chunk_vec, sl);
+    echo_exit_kernel<G, BITS><<<grid, kThreads, 0, st>>>(src, out, n_out, chunk_vec, sl);
 }
 
 template <int BITS>
-void exit_b(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl, cudaStream_t st) {
+void exit_b(const Bufs &b, const ChunkSrc &src, const OutPtrs &out, int n_out, int owners,
+            Slab sl, cudaStream_t st) {
     switch (b.G) {
-        case 32: exit_g<32, BITS>(b, out, n_out, owners, sl, st); break;
-        case 64: exit_g<64, BITS>(b, out, n_out, owners, sl, st); break;
-        default: exit_g<128, BITS>(b, out, n_out, owners, sl, st); break;
+        case 32: exit_g<32, BITS>(src, b.chunk_vec, out, n_out, owners, sl, st); break;
+        case 64: exit_g<64, BITS>(src, b.chunk_vec, out, n_out, owners, sl, st); break;
+        default: exit_g<128, BITS>(src, b.chunk_vec, out, n_out, owners, sl, st); break;
     }
 }
 
@@ -154,10 +156,33 @@ void rs_b(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix, cuda
 
 }  // namespace
 
+ChunkDst chunks_of(const Bufs &b) {
+    ChunkDst d{};
+    const int64_t cbytes = b.chunk_vec * b.bits;          // 8 codes of bits/8 bytes per vector
+    const int64_t cgroups = b.chunk_vec * kVec / b.G;
+    for (int o = 0; o < b.P; ++o) {
+        d.codes[o] = reinterpret_cast<uint8_t *>(b.codes) + o * cbytes;
+        d.scales[o] = b.scales + o * cgroups;
+    }
+    return d;
+}
+
+ChunkSrc reduced_chunks_of(const Bufs &b) {
+    ChunkSrc s{};
+    const int64_t cbytes = b.chunk_vec * b.bits;
+    const int64_t cgroups = b.chunk_vec * kVec / b.G;
+    for (int o = 0; o < b.P; ++o) {
+        s.codes[o] = reinterpret_cast<const uint8_t *>(b.rcodes) + o * cbytes;
+        s.scales[o] = b.rscales + o * cgroups;
+    }
+    return s;
+}
+
 void launch_entry(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chunk_vec,
-                  Slab sl, bool defer, cudaStream_t st) {
-    if (b.bits == 8) entry_b<8>(b, x, rows, rank0, er_chunk_vec, sl, defer, st);
-    else entry_b<4>(b, x, rows, rank0, er_chunk_vec, sl, defer, st);
+                  Slab sl, bool defer, cudaStream_t st, const ChunkDst *dst) {
+    const ChunkDst d = dst ? *dst : chunks_of(b);
+    if (b.bits == 8) entry_b<8>(b, x, rows, rank0, er_chunk_vec, sl, defer, st, d);
+    else entry_b<4>(b, x, rows, rank0, er_chunk_vec, sl, defer, st, d);
 }
 
 void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st, const OutPtrs *out,
@@ -173,9 +198,10 @@ void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st, const Ou
 }
 
 void launch_exit(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl,
-                 cudaStream_t st) {
-    if (b.bits == 8) exit_b<8>(b, out, n_out, owners, sl, st);
-    else exit_b<4>(b, out, n_out, owners, sl, st);
+                 cudaStream_t st, const ChunkSrc *src) {
+    const ChunkSrc s = src ? *src : reduced_chunks_of(b);
+    if (b.bits == 8) exit_b<8>(b, s, out, n_out, owners, sl, st);
+    else exit_b<4>(b, s, out, n_out, owners, sl, st);
 }
 
 void launch_rs(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix,

@@ -56,9 +56,15 @@ void launch_fill(float *p, int64_t n, float v, cudaStream_t st);
 // Entry over `rows` input rows (grid y = rows * P chunks).  rank0: index of
 // row 0 in the group (the owner test for the deferred fix-up);
 // er_chunk_vec: vectors between consecutive owners' e_req chunks (0 when
-// e_req holds one chunk).
+// e_req holds one chunk).  dst: where each chunk's codes and scales go;
+// nullptr: b.codes / b.scales, chunk after chunk.
 void launch_entry(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chunk_vec,
-                  Slab sl, bool defer, cudaStream_t st);
+                  Slab sl, bool defer, cudaStream_t st, const ChunkDst *dst = nullptr);
+
+// b.codes / b.scales seen as consecutive chunks of b.chunk_vec vectors, and
+// b.rcodes / b.rscales the same way.
+ChunkDst chunks_of(const Bufs &b);
+ChunkSrc reduced_chunks_of(const Bufs &b);
 
 // Compensated calls of at most this many elements per rank (1 MiB of bf16)
 // let the reduce write the outputs too, as uncompensated calls always do:
@@ -75,9 +81,10 @@ void launch_reduce(const Bufs &b, int owners, Slab sl, cudaStream_t st,
                    const OutPtrs *out = nullptr, int n_out = 0, bool fix = false);
 
 // Exit over `owners` chunks (grid y): dequantize the reduced transport into
-// n_out outputs.
+// n_out outputs.  src: where each owner's reduced chunk is read; nullptr:
+// b.rcodes / b.rscales, chunk after chunk.
 void launch_exit(const Bufs &b, const OutPtrs &out, int n_out, int owners, Slab sl,
-                 cudaStream_t st);
+                 cudaStream_t st, const ChunkSrc *src = nullptr);
 
 // Reduce-scatter second kernel over `owners` chunks (grid y): out.p[o]
 // receives bf16(s) of chunk o; fix: owner residual folded into state row o.

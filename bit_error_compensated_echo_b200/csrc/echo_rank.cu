@@ -13,6 +13,12 @@
 // The owner fix-up of the EXIT mode runs in the reduce kernel, and that of
 // the SIDE mode in its own kernel; both work on this rank's chunk of the
 // state through pointers offset by rank*C.
+//
+// The fused transport replaces both exchanges by the kernels' own accesses
+// to peer memory: entry_peers stores chunk o into rank o's receive buffer,
+// exit_peers loads owner o's reduced chunk from owner o's buffer.  The
+// buffers peers reach live in the plan's window, one cudaMalloc (so that one
+// IPC handle maps all of it), created on first use.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -36,6 +42,8 @@ struct echo_rank_plan {
     char *ws = nullptr;
     float *m_fast = nullptr, *m_slow = nullptr, *e_req = nullptr;
     bool entered = false;        // an entry ran since the last reduce
+    char *win = nullptr;         // the window: recv codes, recv scales, red codes, red scales
+    echo_rank_window_layout wl{};
     bool side_inflight = false;  // a side-stream fix-up may still run
     cudaEvent_t ev_reduced = nullptr, ev_side_done = nullptr;
 };
@@ -183,6 +191,7 @@ echo_status echo_rank_plan_destroy(echo_rank_plan *p) {
     DeviceGuard guard(p->cfg.device);
     cudaError_t e = cudaDeviceSynchronize();
     if (p->ev_reduced) cudaEventDestroy(p->ev_reduced);
+    if (p->win) cudaFree(p->win);
     if (p->ev_side_done) cudaEventDestroy(p->ev_side_done);
     if (p->ws) cudaFree(p->ws);
     delete p;
@@ -365,6 +374,142 @@ int32_t echo_rank_launches_per_call(const echo_rank_plan *p) {
     if (!p) return 0;
     const bool own_kernel = p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_SIDE;
     return own_kernel ? 4 : 3;
+}
+
+// ------------------------------------------------------------ fused transport
+
+echo_status echo_rank_window(echo_rank_plan *p, echo_rank_window_layout *out) {
+    if (!p || !out) return ECHO_ERR_INVALID_ARG;
+    if (!p->win) {
+        const size_t P = (size_t)p->cfg.P, C = (size_t)p->C;
+        const size_t cb = C * (size_t)p->cfg.bits / 8, cs = C / (size_t)p->cfg.G * 4;
+        echo_rank_window_layout L{};
+        size_t off = 0;
+        auto take = [&](size_t bytes) {
+            const size_t at = off;
+            off += align_up(bytes);
+            return at;
+        };
+        L.recv_codes = take(P * cb);
+        L.recv_scales = take(P * cs);
+        L.red_codes = take(cb);
+        L.red_scales = take(cs);
+        L.bytes = off;
+        DeviceGuard guard(p->cfg.device);
+        if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+        cudaError_t e = cudaMalloc((void **)&p->win, L.bytes);
+        if (e == cudaSuccess) e = cudaMemset(p->win, 0, L.bytes);
+        if (e != cudaSuccess) {
+            if (p->win) cudaFree(p->win);
+            p->win = nullptr;
+            cudaGetLastError();
+            return from_cuda(e);
+        }
+        L.base = p->win;
+        p->wl = L;
+    }
+    *out = p->wl;
+    return ECHO_OK;
+}
+
+echo_status echo_rank_entry_peers(echo_rank_plan *p, const void *x, void *const *recv_codes_peers,
+                                  float *const *recv_scales_peers, void *stream) {
+    if (!p || !x || !recv_codes_peers || !recv_scales_peers) return ECHO_ERR_INVALID_ARG;
+    const int P = p->cfg.P;
+    for (int o = 0; o < P; ++o) {
+        if (!recv_codes_peers[o] || !recv_scales_peers[o]) return ECHO_ERR_INVALID_ARG;
+        if (!aligned16(recv_codes_peers[o]) || !aligned4(recv_scales_peers[o]))
+            return ECHO_ERR_ALIGNMENT;
+    }
+    if (!aligned16(x)) return ECHO_ERR_ALIGNMENT;
+    DeviceGuard guard(p->cfg.device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    ECHO_TRY(order_after_side(p, st));
+    // e_req is -0 (a no-op) when no fix-up is pending
+    const bool defer = p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_DEFERRED;
+
+    Bufs b = base_bufs(p);
+    b.m_fast = p->m_fast;
+    b.m_slow = p->m_slow;
+    b.n_vec = p->n_vec;
+    b.chunk_vec = p->chunk_vec;
+    // this rank's slot in rank o's receive buffer: part `rank` of [P][cb]
+    const int64_t cb = p->C * p->bits / 8, cs = p->C / p->cfg.G;
+    ChunkDst d{};
+    for (int o = 0; o < P; ++o) {
+        d.codes[o] = static_cast<uint8_t *>(recv_codes_peers[o]) + (int64_t)p->rank * cb;
+        d.scales[o] = recv_scales_peers[o] + (int64_t)p->rank * cs;
+    }
+    InPtrs xi{};
+    xi.p[0] = (const uint4 *)x;
+    launch_entry(b, xi, 1, p->rank, 0, chunk_slab(p), defer, st, &d);
+    ECHO_TRY(cudaGetLastError());
+    p->entered = true;
+    return ECHO_OK;
+}
+
+echo_status echo_rank_exit_peers(echo_rank_plan *p, const void *const *red_codes_peers,
+                                 const float *const *red_scales_peers, void *out, void *stream) {
+    if (!p || !red_codes_peers || !red_scales_peers || !out) return ECHO_ERR_INVALID_ARG;
+    const int P = p->cfg.P;
+    ChunkSrc s{};
+    for (int o = 0; o < P; ++o) {
+        if (!red_codes_peers[o] || !red_scales_peers[o]) return ECHO_ERR_INVALID_ARG;
+        if (!aligned16(red_codes_peers[o]) || !aligned4(red_scales_peers[o]))
+            return ECHO_ERR_ALIGNMENT;
+        s.codes[o] = static_cast<const uint8_t *>(red_codes_peers[o]);
+        s.scales[o] = red_scales_peers[o];
+    }
+    if (!aligned16(out)) return ECHO_ERR_ALIGNMENT;
+    DeviceGuard guard(p->cfg.device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    Bufs b = base_bufs(p);
+    b.n_vec = p->n_vec;
+    b.chunk_vec = p->chunk_vec;
+    OutPtrs yo{};
+    yo.p[0] = (uint4 *)out;
+    launch_exit(b, yo, 1, P, chunk_slab(p), (cudaStream_t)stream, &s);
+    ECHO_TRY(cudaGetLastError());
+    return ECHO_OK;
+}
+
+echo_status echo_ipc_handle_get(const void *device_ptr, echo_ipc_handle *out) {
+    if (!device_ptr || !out) return ECHO_ERR_INVALID_ARG;
+    static_assert(sizeof(cudaIpcMemHandle_t) == sizeof(out->bytes), "IPC handle size");
+    cudaIpcMemHandle_t h;
+    const cudaError_t e = cudaIpcGetMemHandle(&h, const_cast<void *>(device_ptr));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return from_cuda(e);
+    }
+    std::memcpy(out->bytes, &h, sizeof(h));
+    return ECHO_OK;
+}
+
+echo_status echo_ipc_open(const echo_ipc_handle *handle, int32_t device, void **out) {
+    if (!handle || !out || device < 0) return ECHO_ERR_INVALID_ARG;
+    *out = nullptr;
+    DeviceGuard guard(device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle->bytes, sizeof(h));
+    const cudaError_t e = cudaIpcOpenMemHandle(out, h, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        *out = nullptr;
+        return from_cuda(e);
+    }
+    return ECHO_OK;
+}
+
+echo_status echo_ipc_close(void *ptr, int32_t device) {
+    if (!ptr || device < 0) return ECHO_ERR_INVALID_ARG;
+    DeviceGuard guard(device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    const cudaError_t e = cudaIpcCloseMemHandle(ptr);
+    if (e != cudaSuccess) cudaGetLastError();
+    return from_cuda(e);
 }
 
 }  // extern "C"

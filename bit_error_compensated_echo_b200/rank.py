@@ -16,7 +16,7 @@ GPU, and leaves each rank the state of its virtual counterpart, bit for bit.
 """
 from __future__ import annotations
 
-from typing import Optional
+from typing import List, Optional, Sequence
 
 import torch
 import torch.distributed as dist
@@ -85,6 +85,101 @@ class ExchangeBuffers:
         all-to-all and its reduced chunk to P-1 ranks in the all-gather."""
         chunk = self.cb + 4 * self.cs
         return 2 * (self.P - 1) * chunk
+
+
+class TorchDistBarrier:
+    """The stream-ordered barrier of the fused transport: a one-element
+    all-reduce on the current stream, which completes on a rank only after
+    every rank's earlier work on its stream."""
+
+    def __init__(self, device, group=None):
+        self.group = group
+        self.flag = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def __call__(self) -> None:
+        dist.all_reduce(self.flag, group=self.group)
+
+
+def _offsets(layout: dict) -> dict:
+    return {k: v for k, v in layout.items() if k != "base"}
+
+
+class PeerWindows:
+    """Every rank's window as mapped in this process (include/echo_rank.h,
+    "Fused transport over peer memory").
+
+    bases[o] is the base address of rank o's window here (this rank's own
+    allocation for o == rank); the byte offsets of the four buffers are the
+    same on every rank of a group (same config).  The pointer tables of the
+    fused stage calls follow from the two."""
+
+    def __init__(self, plan: "EchoRankPlan", bases: Sequence[int], layout: dict,
+                 opened: Sequence[int] = ()):
+        if len(bases) != plan.P:
+            raise ValueError("one window base per rank")
+        self.rank, self.P, self.device = plan.rank, plan.P, plan.device
+        self.bases = [int(b) for b in bases]
+        self.layout = dict(layout)
+        self._opened = list(opened)
+
+    def _at(self, key: str) -> List[int]:
+        off = self.layout[key]
+        return [b + off for b in self.bases]
+
+    # tables over the P ranks, and this rank's own buffers
+    def recv_codes_peers(self) -> List[int]:
+        return self._at("recv_codes")
+
+    def recv_scales_peers(self) -> List[int]:
+        return self._at("recv_scales")
+
+    def red_codes_peers(self) -> List[int]:
+        return self._at("red_codes")
+
+    def red_scales_peers(self) -> List[int]:
+        return self._at("red_scales")
+
+    def own(self, key: str) -> int:
+        return self.bases[self.rank] + self.layout[key]
+
+    @classmethod
+    def exchange(cls, plan: "EchoRankPlan", group=None) -> "PeerWindows":
+        """Run by every rank of the group: share the windows' CUDA IPC
+        handles and map the other ranks' windows into this process."""
+        layout = abi.echo_rank_window(plan.handle)
+        mine = (plan.rank, abi.echo_ipc_handle_get(layout["base"]), layout)
+        got = [None] * plan.P
+        dist.all_gather_object(got, mine, group=group)
+        bases, opened = [], []
+        try:
+            for o, (r, handle, lay) in enumerate(got):
+                if r != o or _offsets(lay) != _offsets(layout):
+                    raise RuntimeError("rank %d: window layouts differ across the group" % o)
+                if o == plan.rank:
+                    bases.append(layout["base"])
+                else:
+                    b = abi.echo_ipc_open(handle, plan.device.index)
+                    opened.append(b)
+                    bases.append(b)
+        except Exception:
+            for b in opened:
+                abi.echo_ipc_close(b, plan.device.index)
+            raise
+        return cls(plan, bases, layout, opened)
+
+    @classmethod
+    def in_process(cls, plans: Sequence["EchoRankPlan"]) -> List["PeerWindows"]:
+        """Every rank's plan in this one process (one device): each rank's
+        tables point straight at the other plans' windows, no IPC."""
+        layouts = [abi.echo_rank_window(p.handle) for p in plans]
+        bases = [lay["base"] for lay in layouts]
+        return [cls(p, bases, layouts[0]) for p in plans]
+
+    def close(self) -> None:
+        """Unmap the peers' windows (this rank's own stays with its plan)."""
+        opened, self._opened = self._opened, []
+        for b in opened:
+            abi.echo_ipc_close(b, self.device.index)
 
 
 def exchange(bufs: ExchangeBuffers, transport) -> None:
@@ -225,6 +320,66 @@ class EchoRankPlan:
         exchange(self.bufs, transport)
         self.reduce_scatter_finish(out, side_stream=side_stream)
         return out
+
+    # ------------------------------------------------------------ fused transport
+    def entry_peers(self, x: torch.Tensor, win: PeerWindows, stream=None) -> None:
+        """Steps 1-3, chunk o stored straight into rank o's receive buffers."""
+        self._check_bf16(x, self.N, "input")
+        abi.echo_rank_entry_peers(self.handle, x.data_ptr(), win.recv_codes_peers(),
+                                  win.recv_scales_peers(), self._st(stream))
+
+    def reduce_window(self, win: PeerWindows, stream=None, side_stream=None) -> None:
+        """Steps 4-5 from this rank's receive buffers into its reduced
+        buffers (both in its window)."""
+        side = int(side_stream.cuda_stream) if side_stream is not None else 0
+        abi.echo_rank_reduce(self.handle, win.own("recv_codes"), win.own("recv_scales"),
+                             win.own("red_codes"), win.own("red_scales"), self._st(stream), side)
+
+    def exit_peers(self, win: PeerWindows, out: torch.Tensor, stream=None) -> None:
+        """Step 6, owner o's reduced chunk loaded straight from owner o."""
+        self._check_bf16(out, self.N, "output")
+        abi.echo_rank_exit_peers(self.handle, win.red_codes_peers(), win.red_scales_peers(),
+                                 out.data_ptr(), self._st(stream))
+
+    def allreduce_peers(self, x: torch.Tensor, win: PeerWindows, barrier,
+                        out: Optional[torch.Tensor] = None, side_stream=None,
+                        bits: Optional[int] = None) -> torch.Tensor:
+        """The all-reduce over the fused transport: entry_peers, barrier,
+        reduce, barrier, exit_peers (include/echo_rank.h).  barrier: a
+        stream-ordered barrier of the group (TorchDistBarrier)."""
+        if bits is not None and int(bits) != self.bits:
+            self.set_bits(bits)
+        if out is None:
+            out = torch.empty(self.N, dtype=torch.bfloat16, device=self.device)
+        self.entry_peers(x, win)
+        barrier()
+        self.reduce_window(win, side_stream=side_stream)
+        barrier()
+        self.exit_peers(win, out)
+        return out
+
+    def reduce_scatter_peers(self, x: torch.Tensor, win: PeerWindows, barrier,
+                             out: Optional[torch.Tensor] = None, side_stream=None,
+                             bits: Optional[int] = None) -> torch.Tensor:
+        """The reduce-scatter over the fused transport: entry_peers, barrier,
+        the owner's bf16 sum from its receive buffers, barrier."""
+        if bits is not None and int(bits) != self.bits:
+            self.set_bits(bits)
+        if out is None:
+            out = torch.empty(self.N // self.P, dtype=torch.bfloat16, device=self.device)
+        self.entry_peers(x, win)
+        barrier()
+        self.reduce_scatter_peers_finish(win, out, side_stream=side_stream)
+        barrier()
+        return out
+
+    def reduce_scatter_peers_finish(self, win: PeerWindows, out: torch.Tensor, stream=None,
+                                    side_stream=None) -> None:
+        """bf16 sum of this rank's chunk from its receive buffers into out."""
+        self._check_bf16(out, self.N // self.P, "output")
+        side = int(side_stream.cuda_stream) if side_stream is not None else 0
+        abi.echo_rank_reduce_scatter(self.handle, win.own("recv_codes"), win.own("recv_scales"),
+                                     out.data_ptr(), self._st(stream), side)
 
     # ------------------------------------------------------------ state
     def reset_state(self, stream=None) -> None:

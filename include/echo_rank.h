@@ -157,8 +157,95 @@ echo_status echo_rank_set_state(echo_rank_plan *plan, const float *m_fast_device
 echo_status echo_rank_plan_set_bits(echo_rank_plan *plan, int32_t bits);
 
 /* Kernels one all-reduce (entry + reduce + exit) launches with this plan:
- * 3, or 4 when the fix-up runs as its own kernel (EXIT and SIDE modes). */
+ * 3, or 4 in SIDE mode (the fix-up as its own kernel). */
 int32_t echo_rank_launches_per_call(const echo_rank_plan *plan);
+
+/* ---------------------------------------------------------------------------
+ * Fused transport over peer memory.
+ *
+ * The two exchanges become accesses of the stage kernels themselves to the
+ * other ranks' memory (NVLink on a B200 node), so that the bytes cross while
+ * the kernel quantizes or dequantizes:
+ *
+ *   echo_rank_entry_peers  steps 1-3, storing chunk o of the codes and
+ *                          scales straight into part `rank` of rank o's
+ *                          receive buffers (the all-to-all)
+ *   (caller)               barrier: every rank's entry has completed
+ *   echo_rank_reduce       unchanged, from this rank's receive buffers into
+ *                          its reduced buffers
+ *   (caller)               barrier: every rank's reduce has completed
+ *   echo_rank_exit_peers   step 6, loading owner o's reduced chunk straight
+ *                          from owner o's reduced buffers (the all-gather)
+ *
+ * The barrier is any stream-ordered operation that completes on a rank only
+ * after the preceding work of every rank has completed, for example a
+ * one-element all-reduce of the collective library on the same stream.  No
+ * kernel waits on another rank.  Two barriers per call also order the next
+ * call: a rank's next entry_peers writes receive buffers that every owner
+ * has finished reading (its reduce came before the second barrier), and an
+ * owner's next reduce writes reduced buffers that every rank has finished
+ * reading (each rank's exit came before its next entry, hence before the
+ * next call's first barrier).  For the reduce-scatter: entry_peers, a
+ * barrier, echo_rank_reduce_scatter from this rank's receive buffers, and a
+ * barrier (the next entry_peers must not write receive buffers an owner is
+ * still reading).
+ *
+ * The receive and reduced buffers peers reach are this plan's window: one
+ * device allocation (so that a single CUDA IPC handle maps it into another
+ * process) with the layouts above, viewed at the code width in force.  Every
+ * rank of a group must use the same width for a call.  Plain loads and
+ * stores only: no TMA, no multicast.
+ * ------------------------------------------------------------------------- */
+
+typedef struct echo_rank_window_layout {
+    void *base;          /* the allocation, on the plan's device */
+    size_t bytes;        /* its size */
+    size_t recv_codes;   /* byte offsets of the four buffers from base, */
+    size_t recv_scales;  /* each 256-byte aligned: recv codes [P][cb_max], */
+    size_t red_codes;    /* recv scales [P][cs] fp32, red codes [cb_max], */
+    size_t red_scales;   /* red scales [cs] fp32; cb_max = C*cfg.bits/8 */
+} echo_rank_window_layout;
+
+/* The plan's window, allocated (and zeroed) on the first call; the plan
+ * owns it and frees it in echo_rank_plan_destroy.
+ * Errors: INVALID_ARG, OOM, CUDA. */
+echo_status echo_rank_window(echo_rank_plan *plan, echo_rank_window_layout *out);
+
+/* Steps 1-3 as echo_rank_entry, with chunk o's codes and scales stored to
+ * recv_codes_peers[o] + rank*cb and recv_scales_peers[o] + rank*cs:
+ *   recv_codes_peers[o]  : rank o's receive codes buffer ([P][cb] bytes),
+ *                          as mapped in this process (16-byte aligned);
+ *                          entry o == rank may be this plan's own
+ *   recv_scales_peers[o] : rank o's receive scales ([P][cs] fp32, 4-byte
+ *                          aligned)
+ * Both are host arrays of P pointers.  One kernel.
+ * Errors: INVALID_ARG (null), ALIGNMENT, CUDA. */
+echo_status echo_rank_entry_peers(echo_rank_plan *plan, const void *x_device,
+                                  void *const *recv_codes_peers, float *const *recv_scales_peers,
+                                  void *stream);
+
+/* Step 6 as echo_rank_exit, with owner o's reduced chunk loaded from
+ * red_codes_peers[o] ([cb] bytes, 16-byte aligned) and red_scales_peers[o]
+ * ([cs] fp32): owner o's reduced buffers as mapped in this process.
+ * One kernel.  Reads no plan state.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+echo_status echo_rank_exit_peers(echo_rank_plan *plan, const void *const *red_codes_peers,
+                                 const float *const *red_scales_peers, void *out_device,
+                                 void *stream);
+
+/* CUDA IPC of a window between the processes of a group (a thin layer over
+ * cudaIpcGetMemHandle / cudaIpcOpenMemHandle / cudaIpcCloseMemHandle).
+ * echo_ipc_handle_get: the handle of the allocation that holds device_ptr
+ * (pass a window base).  echo_ipc_open: map another process's allocation
+ * into this one on `device` (peer access enabled as needed); *out is its
+ * base.  A process cannot open its own handles.  echo_ipc_close: unmap.
+ * Errors: INVALID_ARG, CUDA. */
+typedef struct echo_ipc_handle {
+    uint8_t bytes[64];
+} echo_ipc_handle;
+
+echo_status echo_ipc_handle_get(const void *device_ptr, echo_ipc_handle *out);
+echo_status echo_ipc_open(const echo_ipc_handle *handle, int32_t device, void **out);
+echo_status echo_ipc_close(void *ptr, int32_t device);
 
 #ifdef __cplusplus
 }

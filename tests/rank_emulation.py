@@ -12,7 +12,7 @@ from typing import List, Optional
 
 import torch
 
-from bit_error_compensated_echo_b200.rank import EchoRankPlan
+from bit_error_compensated_echo_b200.rank import EchoRankPlan, PeerWindows
 
 
 def _part(t: torch.Tensor, i: int, size: int) -> torch.Tensor:
@@ -81,3 +81,33 @@ class EmulatedGroup:
         """(m_fast, m_slow) as [P, N] fp32, row r = rank r's state."""
         mf, ms = zip(*(p.get_state() for p in self.plans))
         return torch.stack(mf), torch.stack(ms)
+
+
+class EmulatedPeerGroup(EmulatedGroup):
+    """The same P rank plans on the fused transport: each rank's entry
+    stores into the other plans' windows and its exit loads from them
+    (PeerWindows.in_process).  The stages still run rank by rank, each stage
+    for every rank before the next, so the barrier of a real group is the
+    stream order here and no kernel waits on another."""
+
+    def __init__(self, P: int, N: int, G: int, device: int = 0, **kw):
+        super().__init__(P, N, G, device=device, **kw)
+        self.wins = PeerWindows.in_process(self.plans)
+
+    def allreduce(self, xs: torch.Tensor, side_stream: Optional[torch.cuda.Stream] = None):
+        out = torch.empty_like(xs)
+        for r, (p, w) in enumerate(zip(self.plans, self.wins)):
+            p.entry_peers(xs[r], w)
+        for p, w in zip(self.plans, self.wins):
+            p.reduce_window(w, side_stream=side_stream)
+        for r, (p, w) in enumerate(zip(self.plans, self.wins)):
+            p.exit_peers(w, out[r])
+        return out
+
+    def reduce_scatter(self, xs: torch.Tensor, side_stream: Optional[torch.cuda.Stream] = None):
+        out = torch.empty((self.P, self.N // self.P), dtype=xs.dtype, device=xs.device)
+        for r, (p, w) in enumerate(zip(self.plans, self.wins)):
+            p.entry_peers(xs[r], w)
+        for r, (p, w) in enumerate(zip(self.plans, self.wins)):
+            p.reduce_scatter_peers_finish(w, out[r], side_stream=side_stream)
+        return out
