@@ -111,7 +111,12 @@ class PeerWindows:
     bases[o] is the base address of rank o's window here (this rank's own
     allocation for o == rank); the byte offsets of the four buffers are the
     same on every rank of a group (same config).  The pointer tables of the
-    fused stage calls follow from the two."""
+    fused stage calls follow from the two.
+
+    Teardown, on every rank: synchronize the stream, barrier the group,
+    ``close()`` (unmaps the peers' windows), barrier again, and only then
+    destroy the plan (which frees this rank's window): no rank may still
+    read a window that is unmapped or freed."""
 
     def __init__(self, plan: "EchoRankPlan", bases: Sequence[int], layout: dict,
                  opened: Sequence[int] = ()):
