@@ -184,3 +184,22 @@ def test_refused_captures():
         xh = x.cpu().pin_memory()
         yh = torch.empty_like(xh).pin_memory()
         _refused_under_capture(lambda: pp.allreduce_host(xh, yh))
+
+
+@pytest.mark.filterwarnings("ignore:The CUDA Graph is empty")   # the refused calls queue nothing
+def test_rank_side_fixup_refused_under_capture():
+    """The rank path's reduce and reduce-scatter with a side-stream fix-up
+    return UNSUPPORTED while the stream is capturing; the plan then runs
+    eagerly as if the refused calls had not been made."""
+    from bit_error_compensated_echo_b200.rank import EchoRankPlan
+    P, G, N = 2, 32, 2 * 32 * 4
+    side = torch.cuda.Stream()
+    x = torch.zeros(N, dtype=torch.bfloat16, device=DEV)
+    with EchoRankPlan(P, 0, N, G, device=0, fixup="side") as p:
+        p.entry(x)
+        _refused_under_capture(lambda: p.reduce(side_stream=side))
+        _refused_under_capture(
+            lambda: p.reduce_scatter_finish(torch.empty(N // P, dtype=torch.bfloat16,
+                                                        device=DEV), side_stream=side))
+        p.reduce(side_stream=side)          # the entry is still waiting for its reduce
+        torch.cuda.synchronize()
