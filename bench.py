@@ -497,7 +497,10 @@ def run_step_mode(args, ws, rank, local):
             "config": step_config(args, w, comp, fixup, ws),
             "call_roofline": {"min_bytes": bmin, "achieved_gbs": round(bmin / (ms / 1e3) / 1e9, 1),
                               "peak": peak, "frac": round(bmin / (ms / 1e3) / 1e9 / peak, 4),
-                              "time_at_peak_ms": round(bmin / peak / 1e6, 3)},
+                              "time_at_peak_ms": round(bmin / peak / 1e6, 3),
+                              "frac_of_nominal_8tbs": round(bmin / (ms / 1e3) / 8e12, 4)},
+            # NCCL's algorithm bandwidth: one rank's message over the call time
+            "algbw_gbs": round(2.0 * N / (ms / 1e3) / 1e9, 3),
             "roofline": {"kernel": "echo_entry", "bound": "hbm", "achieved": round(achieved, 1),
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -505,7 +508,8 @@ def run_step_mode(args, ws, rank, local):
             "kernels_ms": {k: round(prof[k] / max(calls, 1), 4)
                            for k in ("entry_ms", "reduce_ms", "exit_ms", "fixup_ms")},
             "gpu_launches": int(prof["launches"]),
-            "e2e": e2e, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_par, "clocks": clk,
+            "e2e": e2e, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_par,
+            "host": host_info() if cpu else None, "clocks": clk,
         }
         print(json.dumps(line), flush=True)
     plan.close()
@@ -540,6 +544,7 @@ def run_reference(args, ws, rank):
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
+        "host": host_info(),
     }
     print(json.dumps(line), flush=True)
 
@@ -784,6 +789,20 @@ def run_group_mode(args, ws, rank, local):
         dist.destroy_process_group()
 
 
+def host_info() -> dict:
+    """The host the CPU legs ran on: CPU model and logical CPUs."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "logical_cpus": os.cpu_count()}
+
+
 def run_cpu_mode(args, ws, rank, local):
     """The oracle, as it stands, on the host cores for each configuration:
     one call (the tiny workload whole, the others on a sample of group
@@ -800,7 +819,8 @@ def run_cpu_mode(args, ws, rank, local):
         gbs_all, dt_all, nw = oracle_parallel_run(w, True, n, x, reps=3)
         elems = w.P * c1 * w.G
         print(json.dumps({
-            "mode": "cpu", "workload": w.name, "kind": "oracle", "group_columns": c1,
+            "mode": "cpu", "workload": w.name, "kind": "oracle", "host": host_info(),
+            "group_columns": c1,
             "of_columns": w.N // w.G, "rank_elements": elems,
             "one_thread": {"seconds": round(dt1, 4), "ns_per_rank_element": round(dt1 / elems * 1e9, 2),
                            "input_gbs": round(gbs1, 5)},
