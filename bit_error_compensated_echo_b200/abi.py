@@ -51,7 +51,8 @@ class echo_debug_view(ctypes.Structure):
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("rcodes", ctypes.c_void_p), ("rscales", ctypes.c_void_p),
                 ("e_req", ctypes.c_void_p), ("fixup_pending", ctypes.c_int32),
-                ("bits", ctypes.c_int32)]
+                ("bits", ctypes.c_int32), ("guard", ctypes.c_void_p),
+                ("guard_bytes", ctypes.c_int64)]
 
 
 class echo_rank_window_layout(ctypes.Structure):

@@ -207,6 +207,7 @@ class EchoPlan:
             "rcodes": t(v.rcodes, (N * bits // 8,), "|u1"),
             "rscales": t(v.rscales, (N // G,), "<f4"),
             "e_req": t(v.e_req, (N,), "<f4"), "fixup_pending": bool(v.fixup_pending),
+            "guard": t(v.guard, (int(v.guard_bytes),), "|u1"),
         }
 
     def profile_enable(self, on: bool = True) -> None:

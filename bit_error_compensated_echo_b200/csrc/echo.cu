@@ -25,6 +25,11 @@ using namespace echo;
 namespace {
 
 constexpr size_t kAlign = 256;
+// After the workspace's sub-buffers: a guard zone of this many bytes filled
+// with kGuardByte at plan creation, which no kernel writes (tests read it
+// through echo_debug_view_get to catch an overrun of the last sub-buffer).
+constexpr size_t kGuardBytes = 4096;
+constexpr int kGuardByte = 0xA5;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -177,7 +182,7 @@ void echo_config_default(echo_config *cfg) {
 
 size_t echo_workspace_bytes(const echo_config *cfg) {
     if (validate_config(cfg) != ECHO_OK) return 0;
-    return layout_of(*cfg).total;
+    return layout_of(*cfg).total + kGuardBytes;
 }
 
 echo_status echo_plan_create(echo_plan **out, const echo_config *cfg) {
@@ -197,9 +202,16 @@ echo_status echo_plan_create(echo_plan **out, const echo_config *cfg) {
     p->chunk_vec = p->n_vec / cfg->P;
     p->b.k = make_consts(*cfg);
 
-    cudaError_t e = cudaMalloc((void **)&p->ws, p->L.total);
+    cudaError_t e = cudaMalloc((void **)&p->ws, p->L.total + kGuardBytes);
     if (e != cudaSuccess) {
         cudaGetLastError();
+        delete p;
+        return from_cuda(e);
+    }
+    e = cudaMemset(p->ws + p->L.total, kGuardByte, kGuardBytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(p->ws);
         delete p;
         return from_cuda(e);
     }
@@ -571,6 +583,8 @@ echo_status echo_debug_view_get(echo_plan *p, echo_debug_view *v) {
     v->e_req = p->e_req;
     v->fixup_pending = p->pending ? 1 : 0;
     v->bits = p->b.bits;
+    v->guard = (uint8_t *)(p->ws + p->L.total);
+    v->guard_bytes = (int64_t)kGuardBytes;
     return ECHO_OK;
 }
 

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define ECHO_ABI_VERSION 2
+#define ECHO_ABI_VERSION 3
 #define ECHO_MAX_RANKS 8
 
 typedef enum echo_status {
@@ -123,7 +123,8 @@ void echo_config_default(echo_config *cfg);
  * (2*P*N fp32 when compensating), the entry transport (P*N*bits/8 code
  * bytes + P*N/G fp32 scales), the reduced transport (N*bits/8 + 4*N/G
  * bytes), e_req (N fp32 when compensating), each sub-buffer 256-byte
- * aligned.
+ * aligned, and a 4 KiB guard zone after them (filled with 0xA5 at plan
+ * creation and written by no kernel; see echo_debug_view).
  * Returns 0 for an invalid config. */
 size_t echo_workspace_bytes(const echo_config *cfg);
 
@@ -239,6 +240,8 @@ typedef struct echo_debug_view {
                               reset or restore (host view: graph replays
                               do not change it) */
     int32_t bits;       /* code width of the calls (echo_plan_set_bits) */
+    uint8_t *guard;     /* the guard zone after the workspace: guard_bytes */
+    int64_t guard_bytes;/* bytes, each 0xA5 unless something overran */
 } echo_debug_view;
 
 echo_status echo_debug_view_get(echo_plan *plan, echo_debug_view *view);

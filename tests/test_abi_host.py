@@ -95,6 +95,7 @@ def test_workspace_bytes_closed_form(abi):
                 + al((N // G) * 4))
         if comp:
             want += 2 * al(P * N * 4) + al(N * 4)
+        want += 4096                        # the guard zone after the sub-buffers
         assert abi.echo_workspace_bytes(c) == want
 
 

@@ -1,5 +1,5 @@
-"""Guard canaries around every caller buffer (the stand-in for a memory
-checker, which is closed here).
+"""Guard canaries around every caller buffer, and after the plan's own
+workspace (the stand-in for a memory checker, which is closed here).
 
 Each buffer the library reads or writes on the caller's side -- inputs,
 outputs, the caller-owned state of the allocation-free call, host buffers of
@@ -58,6 +58,14 @@ def _bits(t):
     return t.contiguous().view(torch.uint8)
 
 
+def _plan_guard_intact(plan: EchoPlan, what: str):
+    """The guard zone after the plan's own workspace (include/echo.h)."""
+    torch.cuda.synchronize()
+    g = plan.debug_view()["guard"]
+    assert g.numel() == 4096
+    assert bool((g == PATTERN).all()), "%s: the plan's workspace guard changed" % what
+
+
 CASES = [(2, 32, 37, 4), (3, 64, 5, 4), (8, 128, 3, 4), (4, 32, 11, 8), (8, 128, 2, 8)]
 
 
@@ -89,6 +97,7 @@ def test_device_calls_keep_guards(P, G, k, bits, comp, fixup):
                 gp.allreduce(xs, out=xs, side_stream=side)
                 want, got = ref.allreduce(x, side_stream=side), torch.stack(xs)
             g.check("call %d (%s)" % (t, op))
+            _plan_guard_intact(gp, "call %d (%s)" % (t, op))
             assert torch.equal(_bits(got), _bits(want)), t
             if op != "I":
                 assert torch.equal(_bits(torch.stack(xs)), _bits(x)), "input changed"
@@ -113,6 +122,7 @@ def test_host_call_keeps_guards(fixup):
             want = ref.allreduce(x).cpu()
             torch.cuda.synchronize()
             g.check("host call %d" % t)
+            _plan_guard_intact(gp, "host call %d" % t)
             assert torch.equal(_bits(torch.stack(ys)), _bits(want)), t
             assert torch.equal(_bits(torch.stack(xs)), _bits(xc)), "input changed"
 
