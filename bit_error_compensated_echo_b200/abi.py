@@ -16,6 +16,7 @@ from typing import Sequence
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libecho_b200.so")
+ABI_VERSION = 3            # ECHO_ABI_VERSION of the headers these bindings follow
 
 ECHO_MAX_RANKS = 8
 
@@ -128,6 +129,11 @@ def _load():
         fn = getattr(L, name)
         fn.restype = res
         fn.argtypes = args
+    if L.echo_abi_version() != ABI_VERSION:
+        raise ImportError(
+            "%s has ABI version %d, these bindings expect %d; rebuild it with "
+            "`python -m bit_error_compensated_echo_b200.build`"
+            % (LIB_PATH, L.echo_abi_version(), ABI_VERSION))
     return L
 
 
