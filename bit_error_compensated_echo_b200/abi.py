@@ -16,7 +16,7 @@ from typing import Sequence
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libecho_b200.so")
-ABI_VERSION = 3            # ECHO_ABI_VERSION of the headers these bindings follow
+ABI_VERSION = 4            # ECHO_ABI_VERSION of the headers these bindings follow
 
 ECHO_MAX_RANKS = 8
 
@@ -59,7 +59,8 @@ class echo_debug_view(ctypes.Structure):
 class echo_rank_window_layout(ctypes.Structure):
     _fields_ = [("base", ctypes.c_void_p), ("bytes", ctypes.c_size_t),
                 ("recv_codes", ctypes.c_size_t), ("recv_scales", ctypes.c_size_t),
-                ("red_codes", ctypes.c_size_t), ("red_scales", ctypes.c_size_t)]
+                ("red_codes", ctypes.c_size_t), ("red_scales", ctypes.c_size_t),
+                ("guard", ctypes.c_size_t), ("guard_bytes", ctypes.c_size_t)]
 
 
 class echo_ipc_handle(ctypes.Structure):
@@ -302,7 +303,8 @@ def echo_rank_window(plan: int) -> dict:
     _check(lib.echo_rank_window(plan, ctypes.byref(L)), "echo_rank_window")
     return {"base": int(L.base or 0), "bytes": int(L.bytes), "recv_codes": int(L.recv_codes),
             "recv_scales": int(L.recv_scales), "red_codes": int(L.red_codes),
-            "red_scales": int(L.red_scales)}
+            "red_scales": int(L.red_scales), "guard": int(L.guard),
+            "guard_bytes": int(L.guard_bytes)}
 
 
 def echo_rank_entry_peers(plan: int, x_device: int, recv_codes_peers: Sequence[int],

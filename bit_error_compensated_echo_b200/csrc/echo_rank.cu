@@ -54,6 +54,10 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
+// The window ends in a guard zone of this many kWindowGuardByte bytes.
+constexpr size_t kWindowGuardBytes = 4096;
+constexpr int kWindowGuardByte = 0xA5;
+
 size_t rank_ws_bytes(const echo_config &c) {
     if (!c.compensate) return 0;
     return 2 * align_up((size_t)c.N * 4) + align_up((size_t)(c.N / c.P) * 4);
@@ -394,11 +398,14 @@ echo_status echo_rank_window(echo_rank_plan *p, echo_rank_window_layout *out) {
         L.recv_scales = take(P * cs);
         L.red_codes = take(cb);
         L.red_scales = take(cs);
-        L.bytes = off;
+        L.guard = off;                       // written by no kernel: overrun checks
+        L.guard_bytes = kWindowGuardBytes;
+        L.bytes = off + kWindowGuardBytes;
         DeviceGuard guard(p->cfg.device);
         if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
         cudaError_t e = cudaMalloc((void **)&p->win, L.bytes);
-        if (e == cudaSuccess) e = cudaMemset(p->win, 0, L.bytes);
+        if (e == cudaSuccess) e = cudaMemset(p->win, 0, L.guard);
+        if (e == cudaSuccess) e = cudaMemset(p->win + L.guard, kWindowGuardByte, L.guard_bytes);
         if (e != cudaSuccess) {
             if (p->win) cudaFree(p->win);
             p->win = nullptr;

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define ECHO_ABI_VERSION 3
+#define ECHO_ABI_VERSION 4
 #define ECHO_MAX_RANKS 8
 
 typedef enum echo_status {

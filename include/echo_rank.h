@@ -199,11 +199,13 @@ int32_t echo_rank_launches_per_call(const echo_rank_plan *plan);
 
 typedef struct echo_rank_window_layout {
     void *base;          /* the allocation, on the plan's device */
-    size_t bytes;        /* its size */
+    size_t bytes;        /* its size, guard zone included */
     size_t recv_codes;   /* byte offsets of the four buffers from base, */
     size_t recv_scales;  /* each 256-byte aligned: recv codes [P][cb_max], */
     size_t red_codes;    /* recv scales [P][cs] fp32, red codes [cb_max], */
     size_t red_scales;   /* red scales [cs] fp32; cb_max = C*cfg.bits/8 */
+    size_t guard;        /* offset of a guard zone after them: guard_bytes */
+    size_t guard_bytes;  /* bytes of 0xA5 that no kernel writes */
 } echo_rank_window_layout;
 
 /* The plan's window, allocated (and zeroed) on the first call; the plan

@@ -49,6 +49,8 @@ def _compare_windows(grp: EmulatedPeerGroup, plan: EchoPlan, call: int):
     rcodes = dv["rcodes"].reshape(P, cb)
     rscales = dv["rscales"].reshape(P, cs)
     for o, w in enumerate(grp.wins):
+        guard = _window_bytes(w, "guard", w.layout["guard_bytes"], torch.uint8)
+        assert bool((guard == 0xA5).all()), "call %d: window guard of rank %d changed" % (call, o)
         rc = _window_bytes(w, "recv_codes", P * cb, torch.uint8).reshape(P, cb)
         rs = _window_bytes(w, "recv_scales", P * cs, torch.float32).reshape(P, cs)
         _same("recv codes of rank %d" % o, rc, codes[:, o], call)
@@ -138,7 +140,8 @@ def test_peer_calls_arguments():
         assert lay == abi.echo_rank_window(p.handle)          # allocated once
         C = N // P
         assert lay["red_codes"] >= lay["recv_scales"] + P * (C // G) * 4
-        assert lay["bytes"] >= lay["red_scales"] + (C // G) * 4
+        assert lay["guard"] >= lay["red_scales"] + (C // G) * 4
+        assert lay["guard_bytes"] == 4096 and lay["bytes"] == lay["guard"] + 4096
         x = torch.zeros(N, dtype=torch.bfloat16, device=DEV)
         codes = [lay["base"] + lay["recv_codes"]] * P
         scales = [lay["base"] + lay["recv_scales"]] * P
