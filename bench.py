@@ -274,10 +274,13 @@ def aggregate(per_rank_ms, per_rank_bytes):
 # ------------------------------------------------------------ CPU baseline
 
 def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: int = 7,
-                      bits: int = 4, op: str = "all-reduce"):
+                      bits: int = 4, op: str = "all-reduce", calls: int = 1):
     """Time the oracle (as it stands, one host thread) on ``ncols`` group
-    columns of workload ``w``; inputs are the device inputs at those columns
-    when given, else a host draw of the same distribution."""
+    columns of workload ``w``: ``calls`` consecutive calls on the same inputs
+    from zero state, as the benchmark's steps repeat the call on its resident
+    inputs; inputs are the device inputs at those columns when given, else a
+    host draw of the same distribution.  Returns (input GB/s, seconds,
+    columns)."""
     import oracle
     cols = W.column_sample(w, ncols, seed=seed)
     idx = W.column_elements(cols, w.G)
@@ -292,9 +295,10 @@ def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: i
     ms = np.zeros_like(mf)
     call = oracle.reduce_scatter if op == "reduce-scatter" else oracle.allreduce
     t0 = time.perf_counter()
-    call(prm, xb, mf, ms, cols)
+    for _ in range(calls):
+        call(prm, xb, mf, ms, cols)
     dt = time.perf_counter() - t0
-    nbytes = 2 * w.P * idx.size
+    nbytes = 2 * w.P * idx.size * calls
     return nbytes / dt / 1e9, dt, cols.size
 
 
@@ -466,11 +470,12 @@ def run_step_mode(args, ws, rank, local):
 
     cpu = cpu_par = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        gbs, dt, ncols = oracle_sample_run(w, comp, args.cpu_cols, x_dev=x, bits=args.bits)
+        gbs, dt, ncols = oracle_sample_run(w, comp, args.cpu_cols, x_dev=x, bits=args.bits,
+                                           calls=args.cpu_calls)
         cpu = {"value": round(gbs, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": "%d of %d group columns (x %d ranks x G=%d) of the same inputs, one "
-                         "call from zero state, %.1f s on one host thread" %
-                         (ncols, N // G, P, G, dt)}
+               "sample": "%d of %d group columns (x %d ranks x G=%d) of the same inputs, %d "
+                         "consecutive calls from zero state, %.1f s on one host thread" %
+                         (ncols, N // G, P, G, args.cpu_calls, dt)}
         if not args.no_cpu_parallel:
             pg, pdt, nw = oracle_parallel_run(w, comp, args.cpu_cols, x, bits=args.bits)
             cpu_par = {"value": round(pg, 5), "unit": UNIT, "cores": nw, "kind": "oracle",
@@ -870,6 +875,9 @@ def main(argv=None):
                     help="skip the all-cores run of the oracle beside the CPU baseline")
     ap.add_argument("--cpu-cols", type=int, default=655360,
                     help="group columns of the CPU-baseline sample")
+    ap.add_argument("--cpu-calls", type=int, default=2,
+                    help="consecutive oracle calls on that sample (about 7-8 s each on one "
+                         "core of the GPU hosts)")
     ap.add_argument("--ref-cols", type=int, default=131072,
                     help="group columns per step of the reference arm")
     args = ap.parse_args(argv)
