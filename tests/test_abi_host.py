@@ -5,6 +5,7 @@ and rejects invalid configurations on the host before any CUDA call.  The
 benchmark's byte counts and cross-rank aggregation are checked here too,
 the latter with two gloo ranks on the CPU.
 """
+import ctypes
 import os
 import re
 import socket
@@ -129,6 +130,16 @@ def test_rank_plan_sizes_and_host_checks(abi):
     assert L.echo_rank_exit(None, None, None, None, None) == abi.ECHO_ERR_INVALID_ARG
     assert L.echo_rank_plan_destroy(None) == abi.ECHO_OK
     assert L.echo_rank_launches_per_call(None) == 0
+    # the fused transport and the IPC layer (include/echo_rank.h)
+    assert L.echo_rank_window(None, None) == abi.ECHO_ERR_INVALID_ARG
+    assert L.echo_rank_entry_peers(None, None, None, None, None) == abi.ECHO_ERR_INVALID_ARG
+    assert L.echo_rank_exit_peers(None, None, None, None, None) == abi.ECHO_ERR_INVALID_ARG
+    assert L.echo_ipc_handle_get(None, None) == abi.ECHO_ERR_INVALID_ARG
+    assert L.echo_ipc_open(None, 0, None) == abi.ECHO_ERR_INVALID_ARG
+    assert L.echo_ipc_close(None, 0) == abi.ECHO_ERR_INVALID_ARG
+    h = abi.echo_ipc_handle()
+    out = ctypes.c_void_p()
+    assert L.echo_ipc_open(ctypes.byref(h), -1, ctypes.byref(out)) == abi.ECHO_ERR_INVALID_ARG
 
 
 def test_bench_byte_counts():
