@@ -104,8 +104,9 @@ typedef struct echo_config {
     int32_t fixup;      /* echo_fixup_mode */
     int32_t bits;       /* code width: 4 (levels -7..7, two codes per byte) or
                          * 8 (levels -127..127, one code per byte; the
-                         * pages' serving policy promotes the earlier half of
-                         * the layers to 8 bits, ai4snews "Perspective").
+                         * pages' serving policy gives 8-bit codes to the
+                         * earlier layers, half of them, ai4snews
+                         * "Perspective").
                          * The widest width of the plan's calls: the
                          * transport is sized for it, and a plan with
                          * bits = 8 can run any call at 4 bits

@@ -1,7 +1,7 @@
 """8-bit codes (levels -127..127, one byte per code) against the oracle:
 whole sequences, ragged shapes, the reduce-scatter, the pipelined host
 call, grid-exact inputs and the Llama-shaped workload on sampled columns.
-The pages' serving policy promotes the earlier half of the layers to 8 bits
+The pages' serving policy gives 8-bit codes to the earlier layers, half of them
 (ai4snews news summary, "Perspective"): a plan made with bits=8 runs each
 call at 4 or 8 bits on one compensator state, which the mixed-width
 sequences below check call by call, following the layer policy."""
