@@ -274,13 +274,14 @@ def aggregate(per_rank_ms, per_rank_bytes):
 # ------------------------------------------------------------ CPU baseline
 
 def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: int = 7,
-                      bits: int = 4, op: str = "all-reduce", calls: int = 1):
+                      bits: int = 4, op: str = "all-reduce", calls: int = 1, keep=None):
     """Time the oracle (as it stands, one host thread) on ``ncols`` group
     columns of workload ``w``: ``calls`` consecutive calls on the same inputs
     from zero state, as the benchmark's steps repeat the call on its resident
     inputs; inputs are the device inputs at those columns when given, else a
     host draw of the same distribution.  Returns (input GB/s, seconds,
-    columns)."""
+    columns); a dict given as ``keep`` receives the element indices, the
+    last call's outputs and the states after it."""
     import oracle
     cols = W.column_sample(w, ncols, seed=seed)
     idx = W.column_elements(cols, w.G)
@@ -296,10 +297,37 @@ def oracle_sample_run(w: W.Workload, comp: bool, ncols: int, x_dev=None, seed: i
     call = oracle.reduce_scatter if op == "reduce-scatter" else oracle.allreduce
     t0 = time.perf_counter()
     for _ in range(calls):
-        call(prm, xb, mf, ms, cols)
+        res = call(prm, xb, mf, ms, cols)
     dt = time.perf_counter() - t0
+    if keep is not None:
+        keep.update(idx=idx, y=res.y, m_fast=mf, m_slow=ms)
+    del res
     nbytes = 2 * w.P * idx.size * calls
     return nbytes / dt / 1e9, dt, cols.size
+
+
+def sampled_parity(plan, x, out, ref: dict, comp: bool, calls: int, side) -> dict:
+    """The benchmark's own configuration against the oracle: after the
+    timed region, the plan's state is reset and the oracle's calls (the same
+    inputs, from zero state) are made again on the GPU; the outputs of the
+    last call and the two states after it are compared, bit for bit, at the
+    oracle's sampled group columns."""
+    plan.reset_state()
+    for _ in range(calls):
+        plan.allreduce(x, out=out, side_stream=side)
+    torch.cuda.synchronize()
+    ti = torch.from_numpy(ref["idx"]).to(x.device)
+    y = out.index_select(1, ti).view(torch.int16).cpu().numpy().view(np.uint16)
+    res = {"calls_from_zero_state": calls,
+           "outputs_bit_exact": bool((y == ref["y"][None, :]).all())}
+    if comp:
+        states_equal = True
+        for m_gpu, m_ref in zip(plan.get_state(), (ref["m_fast"], ref["m_slow"])):
+            m = m_gpu.index_select(1, ti).view(torch.int32).cpu().numpy()
+            states_equal &= bool(np.array_equal(m, m_ref.view(np.int32)))
+            del m_gpu
+        res["states_bit_exact"] = states_equal
+    return res
 
 
 def _oracle_part(job):
@@ -468,10 +496,15 @@ def run_step_mode(args, ws, rank, local):
                "d2h_bytes_per_step": 2 * P * N}
         del xh, yh
 
-    cpu = cpu_par = None
+    cpu = cpu_par = parity = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        ref = {}
         gbs, dt, ncols = oracle_sample_run(w, comp, args.cpu_cols, x_dev=x, bits=args.bits,
-                                           calls=args.cpu_calls)
+                                           calls=args.cpu_calls, keep=ref)
+        if not rs:
+            parity = sampled_parity(plan, x, out, ref, comp, args.cpu_calls, side)
+            parity["group_columns"] = ncols
+        del ref
         cpu = {"value": round(gbs, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "%d of %d group columns (x %d ranks x G=%d) of the same inputs, %d "
                          "consecutive calls from zero state, %.1f s on one host thread" %
@@ -514,7 +547,7 @@ def run_step_mode(args, ws, rank, local):
                            for k in ("entry_ms", "reduce_ms", "exit_ms", "fixup_ms")},
             "gpu_launches": int(prof["launches"]),
             "e2e": e2e, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_par,
-            "host": host_info() if cpu else None, "clocks": clk,
+            "host": host_info() if cpu else None, "parity": parity, "clocks": clk,
         }
         print(json.dumps(line), flush=True)
     plan.close()
