@@ -315,7 +315,8 @@ def sampled_parity(plan, x, out, ref: dict, comp: bool, calls: int, side) -> dic
     plan.reset_state()
     for _ in range(calls):
         plan.allreduce(x, out=out, side_stream=side)
-    torch.cuda.synchronize()
+    if x.is_cuda:
+        torch.cuda.synchronize(x.device)
     ti = torch.from_numpy(ref["idx"]).to(x.device)
     y = out.index_select(1, ti).view(torch.int16).cpu().numpy().view(np.uint16)
     res = {"calls_from_zero_state": calls,
