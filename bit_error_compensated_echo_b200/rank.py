@@ -327,8 +327,15 @@ class EchoRankPlan:
         return out
 
     # ------------------------------------------------------------ fused transport
+    def _check_win(self, win: PeerWindows) -> None:
+        if win.rank != self.rank or win.P != self.P or win.device != self.device:
+            raise ValueError("the windows were mapped for rank %d of %d on %s, not for this "
+                             "plan (rank %d of %d on %s)" % (win.rank, win.P, win.device,
+                                                             self.rank, self.P, self.device))
+
     def entry_peers(self, x: torch.Tensor, win: PeerWindows, stream=None) -> None:
         """Steps 1-3, chunk o stored straight into rank o's receive buffers."""
+        self._check_win(win)
         self._check_bf16(x, self.N, "input")
         abi.echo_rank_entry_peers(self.handle, x.data_ptr(), win.recv_codes_peers(),
                                   win.recv_scales_peers(), self._st(stream))
@@ -336,12 +343,14 @@ class EchoRankPlan:
     def reduce_window(self, win: PeerWindows, stream=None, side_stream=None) -> None:
         """Steps 4-5 from this rank's receive buffers into its reduced
         buffers (both in its window)."""
+        self._check_win(win)
         side = int(side_stream.cuda_stream) if side_stream is not None else 0
         abi.echo_rank_reduce(self.handle, win.own("recv_codes"), win.own("recv_scales"),
                              win.own("red_codes"), win.own("red_scales"), self._st(stream), side)
 
     def exit_peers(self, win: PeerWindows, out: torch.Tensor, stream=None) -> None:
         """Step 6, owner o's reduced chunk loaded straight from owner o."""
+        self._check_win(win)
         self._check_bf16(out, self.N, "output")
         abi.echo_rank_exit_peers(self.handle, win.red_codes_peers(), win.red_scales_peers(),
                                  out.data_ptr(), self._st(stream))
@@ -381,6 +390,7 @@ class EchoRankPlan:
     def reduce_scatter_peers_finish(self, win: PeerWindows, out: torch.Tensor, stream=None,
                                     side_stream=None) -> None:
         """bf16 sum of this rank's chunk from its receive buffers into out."""
+        self._check_win(win)
         self._check_bf16(out, self.N // self.P, "output")
         side = int(side_stream.cuda_stream) if side_stream is not None else 0
         abi.echo_rank_reduce_scatter(self.handle, win.own("recv_codes"), win.own("recv_scales"),

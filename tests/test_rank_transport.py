@@ -53,8 +53,10 @@ def _transport_main(rank, ws, port, q):
         t = TorchDistTransport()
         exchange(b, t)
         gather(b, t)
-        q.put((rank, b.recv_codes.clone(), b.recv_scales.clone(), b.all_codes.clone(),
-               b.all_scales.clone()))
+        # numpy copies travel by value: a tensor would be fetched from this
+        # process, which may have exited by the time the parent reads it
+        q.put((rank, b.recv_codes.numpy().copy(), b.recv_scales.numpy().copy(),
+               b.all_codes.numpy().copy(), b.all_scales.numpy().copy()))
     finally:
         dist.destroy_process_group()
 
@@ -81,7 +83,7 @@ def test_transport_matches_the_buffer_layout(ws):
     got = {}
     for _ in range(ws):
         r, *bufs = q.get(timeout=120)
-        got[r] = bufs
+        got[r] = [torch.from_numpy(a) for a in bufs]
     for p in procs:
         p.join(60)
         assert p.exitcode == 0
@@ -152,7 +154,7 @@ def _orchestration_main(rank, ws, port, q):
         y = plan.allreduce(x, TorchDistTransport(), out=torch.empty(ws * C, dtype=torch.uint8))
         scales = plan.bufs.all_scales.clone()
         z = plan.reduce_scatter(x, TorchDistTransport(), out=torch.empty(C, dtype=torch.uint8))
-        q.put((rank, y, scales, z))
+        q.put((rank, y.numpy().copy(), scales.numpy().copy(), z.numpy().copy()))
     finally:
         dist.destroy_process_group()
 
@@ -169,7 +171,7 @@ def test_allreduce_orchestration_with_byte_stages(ws):
     got = {}
     for _ in range(ws):
         r, y, scales, z = q.get(timeout=120)
-        got[r] = (y, scales, z)
+        got[r] = (torch.from_numpy(y), torch.from_numpy(scales), torch.from_numpy(z))
     for p in procs:
         p.join(60)
         assert p.exitcode == 0
