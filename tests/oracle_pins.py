@@ -220,6 +220,43 @@ def pin_golden_call(o):
     assert r.rcodes.tolist() == [int(t, 16) for t in spec["rcodes"].split()]
 
 
+def pin_golden_sequence(o):
+    """Two hand-worked calls on one state (tests/golden/sequence_worked.txt):
+    the second starts from the first one's states, so the corrections, the
+    partial update of a nonzero state and the owner fix-up are pinned by
+    exact values."""
+    spec = {}
+    for row in _read_golden("sequence_worked.txt"):
+        key, val = [p.strip() for p in row.split("=", 1)]
+        spec[key] = val
+
+    def vec(key, conv=float):
+        return [conv(t) for t in spec[key].split()]
+
+    P, N, G = int(spec["P"]), int(spec["N"]), int(spec["G"])
+    prm = _params(o, P, N, G, True, alpha=float(spec["alpha"]),
+                  beta_fast=float(spec["beta_fast"]), beta_slow=float(spec["beta_slow"]))
+    mf = np.zeros((P, N), np.float32)
+    ms = np.zeros((P, N), np.float32)
+    hexbytes = lambda t: int(t, 16)    # noqa: E731
+    for call in (1, 2):
+        x = np.array([vec("x%d.%d" % (r, call)) for r in range(P)], np.float32)
+        r = o.allreduce(prm, bf16_bits(x), mf, ms)
+        assert bits_to_f64(r.y).tolist() == vec("y.%d" % call), call
+        assert r.rcodes.tolist() == vec("rcodes.%d" % call, hexbytes), call
+        for rr in range(P):
+            assert r.codes[rr].tolist() == vec("codes%d.%d" % (rr, call), hexbytes), (call, rr)
+            assert mf[rr].tolist() == vec("m_fast%d.%d" % (rr, call)), (call, rr)
+            assert ms[rr].tolist() == vec("m_slow%d.%d" % (rr, call)), (call, rr)
+        if call == 2:
+            assert r.rscales.tolist() == vec("rscales.2")
+            assert r.e_req.tolist() == vec("e_req.2")
+            for rr in range(P):
+                assert r.xt[rr].tolist() == vec("xt%d.2" % rr), rr
+                assert r.scales[rr].tolist() == vec("scales%d.2" % rr), rr
+                assert r.e_in[rr].tolist() == vec("e_in%d.2" % rr), rr
+
+
 # ---------------------------------------------------------------- invariants
 
 def grid_exact_inputs(rng, P, N, G, L=7):
