@@ -6,7 +6,8 @@ libecho_b200.so and raises ``EchoError`` (carrying the status code) when it
 returns anything but ECHO_OK.  Pointers are passed as Python ints (device
 or host addresses), streams as cudaStream_t handles (ints; 0 is the legacy
 default stream).  Importing this module loads the library and fails loudly
-if it has not been built: there is no other implementation to fall back on.
+if it has not been built, or was built from headers of another ABI version
+(ABI_VERSION): there is no other implementation to fall back on.
 """
 from __future__ import annotations
 
