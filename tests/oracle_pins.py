@@ -257,6 +257,35 @@ def pin_golden_sequence(o):
                 assert r.e_in[rr].tolist() == vec("e_in%d.2" % rr), rr
 
 
+def pin_golden_reduce_scatter(o):
+    """A hand-worked reduce-scatter call with a sum that is not a bf16
+    value, so the owner's residual is not zero
+    (tests/golden/reduce_scatter_worked.txt)."""
+    spec = {}
+    for row in _read_golden("reduce_scatter_worked.txt"):
+        key, val = [p.strip() for p in row.split("=", 1)]
+        spec[key] = val
+
+    def vec(key, conv=float):
+        return [conv(t) for t in spec[key].split()]
+
+    P, N, G = int(spec["P"]), int(spec["N"]), int(spec["G"])
+    prm = _params(o, P, N, G, True, alpha=float(spec["alpha"]),
+                  beta_fast=float(spec["beta_fast"]), beta_slow=float(spec["beta_slow"]))
+    mf = np.zeros((P, N), np.float32)
+    ms = np.zeros((P, N), np.float32)
+    x = np.array([vec("x%d" % r) for r in range(P)], np.float32)
+    r = o.reduce_scatter(prm, bf16_bits(x), mf, ms)
+    assert r.s.tolist() == vec("s")
+    assert bits_to_f64(r.y).tolist() == vec("y")
+    assert r.e_req.tolist() == vec("e_req")
+    for rr in range(P):
+        assert r.codes[rr].tolist() == vec("codes%d" % rr, lambda t: int(t, 16)), rr
+        assert r.scales[rr].tolist() == vec("scales%d" % rr), rr
+        assert mf[rr].tolist() == vec("m_fast%d" % rr), rr
+        assert ms[rr].tolist() == vec("m_slow%d" % rr), rr
+
+
 # ---------------------------------------------------------------- invariants
 
 def grid_exact_inputs(rng, P, N, G, L=7):
