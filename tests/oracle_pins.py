@@ -257,6 +257,49 @@ def pin_golden_sequence(o):
                 assert r.e_in[rr].tolist() == vec("e_in%d.2" % rr), rr
 
 
+def pin_golden_sequence_padded(o):
+    """The premise of the GPU's check against the hand-worked sequence: the
+    fixture's 4-element groups, each padded with zeros to 32 elements, give
+    the fixture's values at its elements and +0 (code 0) everywhere else."""
+    spec = {}
+    for row in _read_golden("sequence_worked.txt"):
+        key, val = [p.strip() for p in row.split("=", 1)]
+        spec[key] = val
+    P, g, G = int(spec["P"]), int(spec["G"]), 32
+    groups = int(spec["N"]) // g
+    N = groups * G
+
+    def spread(key):
+        v = [float(t) for t in spec[key].split()]
+        out = np.zeros(N)
+        for c in range(groups):
+            out[c * G:c * G + g] = v[c * g:(c + 1) * g]
+        return out
+
+    def spread_bytes(key):
+        v = [int(t, 16) for t in spec[key].split()]
+        out = np.zeros(N // 2, np.uint8)
+        for c in range(groups):
+            out[c * G // 2:c * G // 2 + g // 2] = v[c * g // 2:(c + 1) * g // 2]
+        return out
+
+    prm = _params(o, P, N, G, True, alpha=float(spec["alpha"]),
+                  beta_fast=float(spec["beta_fast"]), beta_slow=float(spec["beta_slow"]))
+    mf = np.zeros((P, N), np.float32)
+    ms = np.zeros((P, N), np.float32)
+    for call in (1, 2):
+        x = np.stack([spread("x%d.%d" % (r, call)) for r in range(P)]).astype(np.float32)
+        r = o.allreduce(prm, bf16_bits(x), mf, ms)
+        assert np.array_equal(bits_to_f64(r.y), spread("y.%d" % call)), call
+        assert np.array_equal(r.rcodes, spread_bytes("rcodes.%d" % call)), call
+        for rr in range(P):
+            assert np.array_equal(r.codes[rr], spread_bytes("codes%d.%d" % (rr, call)))
+            for m, name in ((mf, "m_fast"), (ms, "m_slow")):
+                want = spread("%s%d.%d" % (name, rr, call))
+                assert np.array_equal(m[rr].astype(np.float64), want), (call, name, rr)
+                assert not np.signbit(m[rr][want == 0]).any(), (call, name, rr)
+
+
 def pin_golden_reduce_scatter(o):
     """A hand-worked reduce-scatter call with a sum that is not a bf16
     value, so the owner's residual is not zero
