@@ -31,7 +31,7 @@ state), separate for the forward and the backward pass.
 """
 from __future__ import annotations
 
-from typing import Dict, List
+from typing import Callable, Dict, List, Optional
 
 import torch
 
@@ -78,15 +78,21 @@ class _Chain:
         self.name, self.h, self.plan = name, h0.clone(), plan
 
 
-def _ar(kind: str, parts32: torch.Tensor, plan, buf_bf16, out_bf16, bits=None) -> torch.Tensor:
-    """The site's all-reduce of the P partials ([P, T, D] fp32) -> [T, D] fp32."""
+def _ar(kind: str, parts32: torch.Tensor, plan, buf_bf16, out_bf16, bits=None,
+        seen=None) -> torch.Tensor:
+    """The site's all-reduce of the P partials ([P, T, D] fp32) -> [T, D] fp32.
+    seen(plan, x, y) is called after a library call with its [P, N] bf16
+    inputs and outputs."""
     if kind == "exact":
         return parts32.sum(dim=0)
     buf_bf16.copy_(parts32)
     if kind == "bf16":
         return buf_bf16.float().sum(dim=0).to(torch.bfloat16).float()
     P = parts32.shape[0]
-    plan.allreduce(buf_bf16.view(P, -1), out=out_bf16.view(P, -1), bits=bits)
+    x, y = buf_bf16.view(P, -1), out_bf16.view(P, -1)
+    plan.allreduce(x, out=y, bits=bits)
+    if seen is not None:
+        seen(plan, x, y)
     return out_bf16[0].float()
 
 
@@ -97,8 +103,16 @@ def _dev(h, ref):
 
 
 def run(P: int = 8, tokens: int = 32768, hidden: int = 1024, sites: int = 56, G: int = 128,
-        seed: int = 3, device: str = "cuda", backward: bool = True) -> Dict[str, Dict[str, List[float]]]:
-    """Run the four chains; returns {pass: {chain: [rms per site]}, ...}."""
+        seed: int = 3, device: str = "cuda", backward: bool = True,
+        observer: Optional[Callable] = None) -> Dict[str, Dict[str, List[float]]]:
+    """Run the five chains; returns {pass: {chain: [rms per site]}, ...}.
+
+    observer, if given, is called as observer(direction, site, chain, plan,
+    x, y) right after every call of the library's all-reduce (chains comp,
+    off and promoted), with the call's plan and its [P, N] bf16 inputs and
+    outputs, before anything else touches them; the plan of a chain is the
+    same object from its first site to its last within one direction.  It
+    lets a caller inspect each call (e.g. check it against a reference)."""
     dev = torch.device(device)
     wl = W.Workload("depth", P=1, rows=tokens, hidden=hidden, G=G, seed=seed, dist="student_t")
     h0 = W.generate(wl, 0, dev)[0].view(tokens, hidden).float()
@@ -126,12 +140,16 @@ def run(P: int = 8, tokens: int = 32768, hidden: int = 1024, sites: int = 56, G:
                 site = step if direction == "forward" else len(ws) - 1 - step
                 for c in chains:
                     bits = policy.bits_for_site(site) if c.name == "promoted" else None
+                    seen = None
+                    if observer is not None:
+                        def seen(plan, x, y, _name=c.name, _site=site):
+                            observer(direction, _site, _name, plan, x, y)
                     if direction == "forward":
                         partials(rmsnorm(c.h), wmat, P, parts)
-                        c.h = c.h + _ar(c.name, parts, c.plan, buf, out, bits)
+                        c.h = c.h + _ar(c.name, parts, c.plan, buf, out, bits, seen)
                     else:
                         partials(c.h, wmat.t().contiguous(), P, parts)
-                        u = _ar(c.name, parts, c.plan, buf, out, bits)
+                        u = _ar(c.name, parts, c.plan, buf, out, bits, seen)
                         c.h = c.h + rmsnorm_jt(h_exact_fwd[len(ws) - 1 - step], u)
                 ref = chains[0].h
                 for c in chains[1:]:

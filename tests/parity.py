@@ -107,8 +107,15 @@ class SequenceChecker:
              check_states: bool = True, bits: int | None = None):
         """One call on x ([P, N] bf16 on the plan's device) and its check
         (bits: the call's code width, None for the plan's current one)."""
+        out = self.plan.allreduce(x, out=out, side_stream=side_stream, bits=bits)
+        return out, self.verify(x, out, check_states=check_states)
+
+    def verify(self, x: torch.Tensor, out: torch.Tensor, check_states: bool = True):
+        """Check an all-reduce call that was already made on the plan, on
+        inputs x and outputs out ([P, N] bf16 on the plan's device), at the
+        plan's current code width; the oracle's carried states advance by
+        this call.  Returns the oracle's CallResult."""
         plan = self.plan
-        out = plan.allreduce(x, out=out, side_stream=side_stream, bits=bits)
         prm = self._prm()
         torch.cuda.synchronize()
         call = self.calls
@@ -134,7 +141,7 @@ class SequenceChecker:
                 assert_same("m_fast", _f32(self.gather(mf, "e")), self.mf, "f32", call)
                 assert_same("m_slow", _f32(self.gather(ms, "e")), self.ms, "f32", call)
                 del mf, ms
-        return out, ref
+        return ref
 
 
 def oracle_params(plan: EchoPlan) -> oracle.Params:

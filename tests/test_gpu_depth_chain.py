@@ -6,22 +6,76 @@ the deviation keeps growing (Qwen3-0.6B-like shape: P=8, 32768 tokens x
 The pages state that the total error has a bound that does not grow with
 the number of layers, if no direction is magnified again and again (arXiv abstract on the
 fugumt mirror; ai4snews news summary, "Perspective"); orthogonal maps and
-RMSNorm satisfy that assumption.  This is a property check, not a parity
-check: the all-reduce inside it is the parity-tested library.
+RMSNorm satisfy that assumption.  The deviation tests are property checks;
+in the same run every one of the library's calls (56 forward and 56
+backward sites of the compensated, uncompensated and promoted chains, the
+promoted one across its 8-bit to 4-bit switch) is also checked against the
+oracle, bit for bit, on a sample of group columns: entry and reduced codes
+and scales, outputs, e_req and both states.  The inputs of these calls are
+post-RMSNorm partial products of rotated heavy-tailed activations, and the
+states carry across all 56 sites.
 """
+import collections
+
 import pytest
 
 from bit_error_compensated_echo_b200 import depth_chain
 from bit_error_compensated_echo_b200 import workloads as W
+from parity import SequenceChecker, oracle_params
 
 pytestmark = pytest.mark.gpu
 
+# 256 random group columns plus the first and the last, of 262,144
+COLS = W.column_sample(W.DEPTH, 256, seed=4242)
+
+
+class OracleWatch:
+    """Depth-chain observer: checks each call against the oracle on COLS.
+    A chain's first mismatch is recorded and ends the checks of that chain
+    (its states have left the oracle's from there on)."""
+
+    def __init__(self, cols):
+        self.cols = cols
+        self.checkers = {}
+        self.checked = collections.Counter()
+        self.failures = {}
+
+    def __call__(self, direction, site, chain, plan, x, y):
+        key = (direction, chain)
+        if key in self.failures:
+            return
+        chk = self.checkers.get(key)
+        if chk is None or chk.plan is not plan:
+            chk = self.checkers[key] = SequenceChecker(plan, oracle_params(plan), self.cols)
+        try:
+            chk.verify(x, y)
+        except AssertionError as e:
+            self.failures[key] = "site %d, %d-bit: %s" % (site, plan.bits, e)
+        self.checked[key] += 1
+
 
 @pytest.fixture(scope="module")
-def chain():
-    return depth_chain.run(P=8, tokens=W.DEPTH.rows, hidden=W.DEPTH.hidden,
-                           sites=W.DEPTH.calls, G=W.DEPTH.G, seed=W.DEPTH.seed,
-                           device="cuda:0")
+def run_with_watch():
+    watch = OracleWatch(COLS)
+    res = depth_chain.run(P=8, tokens=W.DEPTH.rows, hidden=W.DEPTH.hidden,
+                          sites=W.DEPTH.calls, G=W.DEPTH.G, seed=W.DEPTH.seed,
+                          device="cuda:0", observer=watch)
+    return res, watch
+
+
+@pytest.fixture(scope="module")
+def chain(run_with_watch):
+    return run_with_watch[0]
+
+
+def test_every_call_matches_the_oracle(run_with_watch):
+    """Config 4 at full size (P=8, 32768 x 1024, G=128): all 336 calls of
+    the three library chains against the oracle on 258 group columns."""
+    _, watch = run_with_watch
+    assert not watch.failures, watch.failures
+    for direction in ("forward", "backward"):
+        for name in ("comp", "off", "promoted"):
+            assert watch.checked[(direction, name)] == W.DEPTH.calls, (direction, name)
 
 
 def test_forward_deviation_bounded_with_compensation(chain):
