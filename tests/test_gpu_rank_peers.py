@@ -1,12 +1,17 @@
 """The fused transport of the rank path (include/echo_rank.h, "Fused
 transport over peer memory"): P rank plans on one GPU whose entries store
 each chunk straight into the owner's window and whose exits load the owners'
-reduced chunks straight from theirs, against the plan of P virtual ranks,
-call by call, bit for bit -- outputs, the bytes in every window (each
-rank's receive buffers and each owner's reduced chunk) and every rank's two
-EMA states."""
+reduced chunks straight from theirs, against the oracle and against the plan
+of P virtual ranks, call by call, bit for bit -- outputs, the bytes in every
+window (each rank's receive buffers and each owner's reduced chunk) and
+every rank's two EMA states."""
+import dataclasses
+
+import numpy as np
 import pytest
 import torch
+
+import oracle
 
 from bit_error_compensated_echo_b200 import abi
 from bit_error_compensated_echo_b200 import workloads as W
@@ -59,6 +64,117 @@ def _compare_windows(grp: EmulatedPeerGroup, plan: EchoPlan, call: int):
               rcodes[o], call)
         _same("red scales of owner %d" % o, _window_bytes(w, "red_scales", cs, torch.float32),
               rscales[o], call)
+
+
+def _windows_against_oracle(grp: EmulatedPeerGroup, ref, bits: int, call: int,
+                            reduced: bool = True):
+    """Rank o's receive part r holds rank r's chunk o of the oracle's entry
+    codes and scales; owner o's reduced chunk is chunk o of the oracle's
+    requantized codes and scales (all-reduce calls only)."""
+    P, N, G = grp.P, grp.N, grp.G
+    C = N // P
+    cb, cs = C * bits // 8, C // G
+    for o, w in enumerate(grp.wins):
+        rc = _window_bytes(w, "recv_codes", P * cb, torch.uint8).reshape(P, cb)
+        rs = _window_bytes(w, "recv_scales", P * cs, torch.float32).reshape(P, cs)
+        assert_same("recv codes of rank %d" % o, rc.numpy(), ref.codes[:, o * cb:(o + 1) * cb],
+                    "u8", call)
+        assert_same("recv scales of rank %d" % o, rs.numpy(),
+                    ref.scales[:, o * cs:(o + 1) * cs], "f32", call)
+        if reduced:
+            assert_same("red codes of owner %d" % o,
+                        _window_bytes(w, "red_codes", cb, torch.uint8).numpy(),
+                        ref.rcodes[o * cb:(o + 1) * cb], "u8", call)
+            assert_same("red scales of owner %d" % o,
+                        _window_bytes(w, "red_scales", cs, torch.float32).numpy(),
+                        ref.rscales[o * cs:(o + 1) * cs], "f32", call)
+
+
+@pytest.mark.parametrize("comp,fixup", [(True, "exit"), (True, "side"), (True, "deferred"),
+                                        (False, "deferred")])
+def test_peer_group_against_oracle(comp, fixup):
+    """The tiny workload's 16-call sequence on the fused transport, every
+    rank against the oracle: outputs, every window, both states."""
+    w = W.TINY
+    side = torch.cuda.Stream() if fixup == "side" else None
+    prm = oracle.Params(P=w.P, N=w.N, G=w.G, compensate=comp)
+    mf = np.zeros((w.P, w.N), np.float32)
+    ms = np.zeros((w.P, w.N), np.float32)
+    with EmulatedPeerGroup(w.P, w.N, w.G, compensate=comp, fixup=fixup) as grp:
+        for t in range(w.calls):
+            x = W.generate(w, t, DEV)
+            y = grp.allreduce(x, side_stream=side)
+            torch.cuda.synchronize()
+            ref = oracle.allreduce(prm, _bits_u16(x), mf, ms)
+            yb = _bits_u16(y)
+            assert_same("outputs", yb, np.broadcast_to(ref.y, yb.shape), "bf16", t)
+            _windows_against_oracle(grp, ref, 4, t)
+            if comp:
+                gmf, gms = grp.get_state()
+                assert_same("m_fast", _f32(gmf), mf, "f32", t)
+                assert_same("m_slow", _f32(gms), ms, "f32", t)
+
+
+@pytest.mark.parametrize("P,G,k", [(3, 64, 7), (8, 128, 5), (8, 32, 3), (5, 32, 11)],
+                         ids=lambda v: str(v))
+@pytest.mark.parametrize("fixup", ["exit", "side", "deferred"])
+def test_peer_group_mixed_ops_against_oracle(P, G, k, fixup):
+    """All-reduces and reduce-scatters at 8 and 4 bits on one state of a
+    bits=8 group, on the fused transport, against the oracle call by call
+    (ragged chunks: k groups per owner)."""
+    N = P * G * k
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    side = torch.cuda.Stream() if fixup == "side" else None
+    prm = oracle.Params(P=P, N=N, G=G, compensate=True)
+    mf = np.zeros((P, N), np.float32)
+    ms = np.zeros((P, N), np.float32)
+    C = N // P
+    with EmulatedPeerGroup(P, N, G, fixup=fixup, bits=8) as grp:
+        for t, (op, bits) in enumerate([("A", 8), ("R", 8), ("A", 4), ("R", 4), ("A", 4),
+                                        ("A", 8), ("R", 4), ("A", 4)]):
+            for p in grp.plans:
+                p.set_bits(bits)
+            x = W.generate(w, t, DEV)
+            cp = dataclasses.replace(prm, bits=bits)
+            if op == "A":
+                y = grp.allreduce(x, side)
+                torch.cuda.synchronize()
+                ref = oracle.allreduce(cp, _bits_u16(x), mf, ms)
+                yb = _bits_u16(y)
+                assert_same("outputs", yb, np.broadcast_to(ref.y, yb.shape), "bf16", t)
+            else:
+                y = grp.reduce_scatter(x, side)
+                torch.cuda.synchronize()
+                ref = oracle.reduce_scatter(cp, _bits_u16(x), mf, ms)
+                assert_same("owner outputs", _bits_u16(y), ref.y.reshape(P, C), "bf16", t)
+            _windows_against_oracle(grp, ref, bits, t, reduced=(op == "A"))
+            gmf, gms = grp.get_state()
+            assert_same("m_fast", _f32(gmf), mf, "f32", t)
+            assert_same("m_slow", _f32(gms), ms, "f32", t)
+
+
+def test_peer_group_llama_shape_against_oracle():
+    """P=8, 2048 x 4096 bf16 per rank, G=128, deferred fix-up, 4 calls on
+    the fused transport: outputs and both states against the oracle on 258
+    sampled group columns."""
+    wl = W.LLAMA
+    cols = W.column_sample(wl, 256, seed=99)
+    idx = torch.from_numpy(W.column_elements(cols, wl.G)).to(DEV)
+    prm = oracle.Params(P=wl.P, N=wl.N, G=wl.G, compensate=True)
+    mf = np.zeros((wl.P, idx.numel()), np.float32)
+    ms = np.zeros_like(mf)
+    with EmulatedPeerGroup(wl.P, wl.N, wl.G, fixup="deferred") as grp:
+        for t in range(4):
+            x = W.generate(wl, t, DEV)
+            y = grp.allreduce(x)
+            torch.cuda.synchronize()
+            ref = oracle.allreduce(prm, _bits_u16(x.index_select(1, idx)), mf, ms, cols)
+            yb = _bits_u16(y.index_select(1, idx))
+            assert_same("outputs", yb, np.broadcast_to(ref.y, yb.shape), "bf16", t)
+            gmf, gms = grp.get_state()
+            assert_same("m_fast", _f32(gmf.index_select(1, idx)), mf, "f32", t)
+            assert_same("m_slow", _f32(gms.index_select(1, idx)), ms, "f32", t)
+            del gmf, gms
 
 
 CASES = [  # P, G, groups per chunk, bits
