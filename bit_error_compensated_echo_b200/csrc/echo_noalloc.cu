@@ -5,6 +5,7 @@
 // lives in one file-scope device array instead of a plan's workspace, and
 // the caller owns the compensator state.  Nothing here calls cudaMalloc,
 // cudaFree or a host allocator.
+#include <cuda.h>   // CUcontext and CUresult only; the two driver calls are fetched at run time
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -23,8 +24,50 @@ static __device__ __align__(256) unsigned char echo_noalloc_scratch[ECHO_NOALLOC
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// The array's device address belongs to the CUDA context it was looked up
+// in.  A device reset, or a caller that makes another context current on
+// the device (driver-API users), loads the module anew, at an address the
+// old lookup does not know.  So the cache of each device slot is keyed by
+// the unique id of the context that was current at the lookup (cuCtxGetId:
+// the driver never gives two contexts of one process the same id), and a
+// call in any other context looks the address up again.
+struct ScratchSlot {
+    bool valid = false;
+    unsigned long long ctx_id = 0;
+    void *addr = nullptr;
+};
 std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices];  // device address of the array, per device
+ScratchSlot g_scratch[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+bool g_ctx_fns_tried = false;
+
+// The id of the calling thread's current context; false if there is none
+// yet or the driver cannot say.  Called with g_scratch_mu held.
+bool current_context_id(unsigned long long *id) {
+    if (!g_ctx_fns_tried) {
+        g_ctx_fns_tried = true;
+        void *f = nullptr, *g = nullptr;
+        cudaDriverEntryPointQueryResult qf{}, qg{};
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault,
+                                             &qf) == cudaSuccess &&
+            cudaGetDriverEntryPointByVersion("cuCtxGetId", &g, 12000, cudaEnableDefault, &qg) ==
+                cudaSuccess &&
+            qf == cudaDriverEntryPointSuccess && qg == cudaDriverEntryPointSuccess) {
+            g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+            g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(g);
+        }
+        cudaGetLastError();
+    }
+    if (!g_ctx_get_current || !g_ctx_get_id) return false;
+    CUcontext ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return g_ctx_get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
@@ -49,18 +92,33 @@ ScratchLayout scratch_layout(int P, int64_t N, int G, bool comp) {
     return L;
 }
 
-// Looks up the array's device address once per device, with that device
-// current, and caches it.
-cudaError_t scratch_address(int dev, unsigned char **out) {
+// The array's device address in the current context of device dev (which
+// is current): cached per device and context; the set-up (the lookup with
+// cudaGetSymbolAddress, which may load the module into the context) runs
+// on the first call in a context, and is refused on a capturing stream,
+// where loading a module could break the capture.  Without a context id
+// (a driver that cannot give one) every call looks the address up.
+echo_status scratch_address(int dev, cudaStream_t st, unsigned char **out) {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, echo_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
+    const bool cap = capturing(st);
+    if (cap && !g_ctx_fns_tried) return ECHO_ERR_UNSUPPORTED;   // no set-up has run yet
+    ScratchSlot &slot = g_scratch[dev];
+    unsigned long long id = 0;
+    bool have_id = current_context_id(&id);
+    if (have_id && slot.valid && slot.ctx_id == id) {
+        *out = (unsigned char *)slot.addr;
+        return ECHO_OK;
     }
-    *out = (unsigned char *)g_scratch_addr[dev];
-    return cudaSuccess;
+    if (cap) return ECHO_ERR_UNSUPPORTED;
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, echo_noalloc_scratch);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (!have_id) have_id = current_context_id(&id);   // the lookup bound a context
+    slot.valid = have_id;
+    slot.ctx_id = id;
+    slot.addr = p;
+    *out = (unsigned char *)p;
+    return ECHO_OK;
 }
 
 // The launches of one call, on the array's carved sub-buffers.
@@ -133,11 +191,11 @@ extern "C" echo_status echo_allreduce_noalloc(const echo_config *cfg, const void
     if (cudaGetDevice(&prev) != cudaSuccess) return ECHO_ERR_CUDA;
     if (prev != cfg->device && cudaSetDevice(cfg->device) != cudaSuccess) return ECHO_ERR_CUDA;
     unsigned char *scratch = nullptr;
-    cudaError_t e = scratch_address(cfg->device, &scratch);
-    if (e == cudaSuccess) {
+    echo_status st = scratch_address(cfg->device, (cudaStream_t)stream, &scratch);
+    if (st == ECHO_OK) {
         launch_all(x, y, m_fast_device, m_slow_device, scratch, L, *cfg, (cudaStream_t)stream);
-        e = cudaGetLastError();
+        if (cudaGetLastError() != cudaSuccess) st = ECHO_ERR_CUDA;
     }
     if (prev != cfg->device) cudaSetDevice(prev);
-    return e == cudaSuccess ? ECHO_OK : ECHO_ERR_CUDA;
+    return st;
 }

@@ -304,9 +304,15 @@ int32_t echo_launches_per_call(const echo_plan *plan);
  * bytes, each part rounded up to 256; a call that needs more returns
  * ECHO_ERR_UNSUPPORTED before launching anything (80 MiB holds, e.g., 8
  * ranks of 2048 x 4096 bf16 activations with the compensator on).
- * The first call on a device looks up the array's address with
- * cudaGetSymbolAddress while that device is current; make that first call
- * before any stream capture.  All calls on a device share the one array and
+ * Set-up: the first call in a CUDA context on a device looks up the
+ * array's address with cudaGetSymbolAddress while that device is current
+ * (this may load the library's device code into the context), and later
+ * calls in the same context reuse it.  The address belongs to that context:
+ * after cudaDeviceReset, or when the caller makes another context current
+ * (driver-API users), the next call sees a context it has not seen and does
+ * the set-up again.  Make the first call in each context before any stream
+ * capture: a call whose set-up is still due returns ECHO_ERR_UNSUPPORTED,
+ * launching nothing, while its stream is capturing.  All calls on a device share the one array and
  * it keeps the last call's contents: nothing in it needs to start at zero
  * (every byte a call reads was written earlier in the same call), but calls
  * that overlap on the GPU -- on streams not ordered with each other, or
