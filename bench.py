@@ -230,12 +230,8 @@ def dist_setup():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
-        if backend == "nccl":
-            torch.cuda.set_device(local)
-        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+        from bit_error_compensated_echo_b200.rank import init_process_group
+        init_process_group(timeout_s=120.0)
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return ws, rank, local
@@ -740,13 +736,12 @@ def run_group_mode(args, ws, rank, local):
     import torch.distributed as dist
 
     from bit_error_compensated_echo_b200.rank import (EchoRankPlan, PeerWindows,
-                                                      TorchDistBarrier, TorchDistTransport)
+                                                      TorchDistBarrier, TorchDistTransport,
+                                                      init_process_group)
     if ws == 1 and not dist.is_initialized():
-        import datetime
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
         os.environ.setdefault("MASTER_PORT", str(29500 + (os.getpid() % 1000)))
-        dist.init_process_group("nccl", rank=0, world_size=1,
-                                timeout=datetime.timedelta(seconds=120))
+        init_process_group("nccl", timeout_s=120.0, rank=0, world_size=1)
     dev = torch.device("cuda", local)
     w = WORKLOADS[args.workload]
     comp = not args.uncompensated

@@ -16,6 +16,8 @@ GPU, and leaves each rank the state of its virtual counterpart, bit for bit.
 """
 from __future__ import annotations
 
+import datetime
+import os
 from typing import List, Optional, Sequence
 
 import torch
@@ -23,6 +25,32 @@ import torch.distributed as dist
 
 from . import abi
 from .api import _stream_handle, make_config
+
+
+def process_group_options(backend: str, local_rank: int) -> dict:
+    """Extra keyword arguments of torch.distributed.init_process_group for a
+    process driving GPU ``local_rank``: an NCCL group is bound to that GPU
+    (device_id), so that NCCL never guesses the device from the global rank
+    -- a guess that is wrong whenever ranks and GPUs are numbered
+    differently, and then hangs the group's first collective."""
+    if backend == "nccl":
+        return {"device_id": torch.device("cuda", int(local_rank))}
+    return {}
+
+
+def init_process_group(backend: Optional[str] = None, timeout_s: float = 120.0, **kw) -> int:
+    """Join the process group of the launch (RANK, WORLD_SIZE, MASTER_* and
+    LOCAL_RANK from the environment, or rank/world_size in kw) with a short
+    timeout; with NCCL the process first makes its GPU, LOCAL_RANK, current
+    and binds the group to it.  Returns the local rank."""
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s),
+                            **process_group_options(backend, local), **kw)
+    return local
 
 
 class TorchDistTransport:

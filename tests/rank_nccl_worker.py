@@ -5,7 +5,6 @@ mapped with CUDA IPC, a one-element NCCL all-reduce as the barrier), against
 the plan of P virtual ranks that every rank also runs on the whole group's
 input.  Exits non-zero on the first difference.  Usable with any number of
 GPUs, one rank each; the single-GPU test suite runs it with one rank."""
-import datetime
 import os
 import sys
 
@@ -17,7 +16,8 @@ sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 from bit_error_compensated_echo_b200 import workloads as W  # noqa: E402
 from bit_error_compensated_echo_b200.api import EchoPlan  # noqa: E402
 from bit_error_compensated_echo_b200.rank import (EchoRankPlan, PeerWindows,  # noqa: E402
-                                                  TorchDistBarrier, TorchDistTransport)
+                                                  TorchDistBarrier, TorchDistTransport,
+                                                  init_process_group)
 
 
 def bits_equal(a, b):
@@ -65,9 +65,7 @@ def run_case(transport, P, rank, local, dev, G, k, fixup, bits, bad):
 
 
 def main():
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    local = init_process_group("nccl", timeout_s=120.0)
     rank, P = dist.get_rank(), dist.get_world_size()
     dev = torch.device("cuda", local)
     bad = []

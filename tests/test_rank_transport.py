@@ -183,3 +183,68 @@ def test_allreduce_orchestration_with_byte_stages(ws):
         assert torch.equal(y.to(torch.int64), total), r
         assert torch.equal(scales, torch.full((ws,), rank_sum)), r
         assert torch.equal(z.to(torch.int64), total[r * C:(r + 1) * C]), r
+
+
+def _bind_main(rank, ws, port, q):
+    import torch.distributed as dist
+
+    import bench
+    from bit_error_compensated_echo_b200 import rank as rank_mod
+    # ranks and local ranks numbered differently: rank r drives GPU ws-1-r
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(ws), LOCAL_RANK=str(ws - 1 - rank))
+    got_ws, got_rank, local = bench.dist_setup()
+    try:
+        opts = rank_mod.process_group_options("nccl", local)
+        locals_ = [None] * ws
+        dist.all_gather_object(locals_, local)
+        q.put((rank, got_ws, got_rank, local, str(opts["device_id"]), locals_,
+               dist.get_backend()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_process_group_binds_each_rank_to_its_local_device():
+    """World size 2 over gloo, launched as the bench's ranks are (RANK,
+    WORLD_SIZE, LOCAL_RANK from the environment), with ranks and GPUs
+    numbered differently: each rank joins as its RANK, keeps its LOCAL_RANK,
+    and an NCCL group would be bound to cuda:LOCAL_RANK, not cuda:RANK."""
+    import torch.multiprocessing as mp
+    ws = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bind_main, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(ws):
+        item = q.get(timeout=120)
+        got[item[0]] = item[1:]
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    for r in range(ws):
+        got_ws, got_rank, local, dev, locals_, backend = got[r]
+        assert (got_ws, got_rank, local) == (ws, r, ws - 1 - r)
+        assert dev == "cuda:%d" % (ws - 1 - r)
+        assert locals_ == [ws - 1 - q_ for q_ in range(ws)]
+        assert backend == "gloo"
+
+
+def test_nccl_group_is_bound_to_the_local_gpu(monkeypatch):
+    """The NCCL path of init_process_group, with fakes for the two calls it
+    makes: the process's GPU (LOCAL_RANK) is made current and passed as
+    device_id."""
+    from bit_error_compensated_echo_b200 import rank as rank_mod
+    seen = {}
+    monkeypatch.setenv("LOCAL_RANK", "3")
+    monkeypatch.setattr(rank_mod.torch.cuda, "set_device", lambda d: seen.setdefault("dev", d))
+    monkeypatch.setattr(rank_mod.dist, "init_process_group",
+                        lambda **kw: seen.setdefault("kw", kw))
+    assert rank_mod.init_process_group("nccl", timeout_s=5.0) == 3
+    assert seen["dev"] == 3
+    assert seen["kw"]["backend"] == "nccl"
+    assert seen["kw"]["device_id"] == torch.device("cuda", 3)
+    assert seen["kw"]["timeout"].total_seconds() == 5.0
+    assert rank_mod.process_group_options("gloo", 3) == {}
