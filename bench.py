@@ -127,6 +127,28 @@ def exit_bytes(P: int, N: int, G: int, bits: int = 4) -> float:
     return N * transport_bytes_per_elem(G, bits) + P * N * 2
 
 
+def kernel_rooflines(prof: dict, P: int, N: int, G: int, comp: bool, fixup: str, bits: int,
+                     peak: float) -> dict:
+    """Each kernel's algorithmic bytes per launch over its average launch
+    time (the plan's CUDA events on the launch stream), against the HBM peak.
+    When the reduce writes the outputs (no exit launch) its bytes include
+    them."""
+    calls = max(int(prof["calls"]), 1)
+    merged = prof["exit_ms"] == 0.0
+    rb = reduce_bytes(P, N, G, comp, fixup, bits) + (P * N * 2 if comp and merged else 0)
+    out = {}
+    for name, b, key in (("echo_entry", entry_bytes(P, N, G, comp, fixup, bits), "entry_ms"),
+                         ("echo_reduce", rb, "reduce_ms"),
+                         ("echo_exit", exit_bytes(P, N, G, bits), "exit_ms")):
+        ms = prof[key] / calls
+        if ms <= 0.0:
+            continue
+        gbs = b / (ms / 1e3) / 1e9
+        out[name] = {"bytes": b, "avg_launch_ms": round(ms, 4), "achieved": round(gbs, 1),
+                     "frac": round(gbs / peak, 4)}
+    return out
+
+
 # ------------------------------------------------------------ environment
 
 def load_peaks():
@@ -542,6 +564,8 @@ def run_step_mode(args, ws, rank, local):
                          "algorithmic_bytes": eb, "avg_launch_ms": round(entry_ms, 4)},
             "kernels_ms": {k: round(prof[k] / max(calls, 1), 4)
                            for k in ("entry_ms", "reduce_ms", "exit_ms", "fixup_ms")},
+            "kernels_roofline": (None if rs else
+                                 kernel_rooflines(prof, P, N, G, comp, fixup, args.bits, peak)),
             "gpu_launches": int(prof["launches"]),
             "e2e": e2e, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_par,
             "host": host_info() if cpu else None, "parity": parity, "clocks": clk,

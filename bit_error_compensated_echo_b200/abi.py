@@ -17,7 +17,7 @@ from typing import Sequence
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libecho_b200.so")
-ABI_VERSION = 4            # ECHO_ABI_VERSION of the headers these bindings follow
+ABI_VERSION = 5            # ECHO_ABI_VERSION of the headers these bindings follow
 
 ECHO_MAX_RANKS = 8
 
@@ -100,6 +100,9 @@ def _load():
         "echo_plan_set_bits": (st, [vp, ctypes.c_int32]),
         "echo_status_string": (ctypes.c_char_p, [st]),
         "echo_abi_version": (ctypes.c_int32, []),
+        "echo_device_error_get": (st, [ctypes.c_int32, ctypes.POINTER(ctypes.c_int32),
+                                       ctypes.c_int32]),
+        "echo_selftest_wait_limit": (st, [ctypes.c_int32]),
         "echo_allreduce_noalloc": (st, [ctypes.POINTER(echo_config), ctypes.POINTER(vp),
                                         ctypes.POINTER(vp), vp, vp, vp]),
         # include/echo_rank.h
@@ -232,6 +235,23 @@ def echo_launches_per_call(plan: int) -> int:
 
 def echo_status_string(status: int) -> str:
     return lib.echo_status_string(status).decode()
+
+
+ECHO_DEVERR_WAIT_TIMEOUT = 1
+
+
+def echo_device_error_get(device: int, clear: bool = False) -> int:
+    """The library's device error word on `device` (ECHO_DEVERR_* bits),
+    cleared afterwards if `clear`."""
+    flags = ctypes.c_int32()
+    _check(lib.echo_device_error_get(device, ctypes.byref(flags), int(bool(clear))),
+           "echo_device_error_get")
+    return int(flags.value)
+
+
+def echo_selftest_wait_limit(device: int) -> None:
+    """Run the bounded-wait self-test on `device` (about one second)."""
+    _check(lib.echo_selftest_wait_limit(device), "echo_selftest_wait_limit")
 
 
 def echo_abi_version() -> int:

@@ -645,6 +645,27 @@ const char *echo_status_string(echo_status s) {
     return "ECHO_ERR_UNKNOWN";
 }
 
+echo_status echo_device_error_get(int32_t device, int32_t *flags, int32_t clear) {
+    if (!flags || device < 0) return ECHO_ERR_INVALID_ARG;
+    DeviceGuard guard(device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    ECHO_TRY(device_error_read(flags, clear != 0));
+    return ECHO_OK;
+}
+
+echo_status echo_selftest_wait_limit(int32_t device) {
+    if (device < 0) return ECHO_ERR_INVALID_ARG;
+    DeviceGuard guard(device);
+    if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
+    cudaStream_t st = nullptr;
+    ECHO_TRY(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
+    launch_wait_selftest(st);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    cudaStreamDestroy(st);
+    return from_cuda(e);
+}
+
 int32_t echo_abi_version(void) { return ECHO_ABI_VERSION; }
 
 }  // extern "C"

@@ -20,6 +20,12 @@ namespace echo {
 // compensated entry.
 // Grid: x over the slab's vectors / (4 * kThreads), y = rank * P + chunk.
 constexpr int kRawVPT = 4;
+// Resident blocks per SM the register allocation must allow.  The kernel's
+// loads are all issued before its arithmetic, so the bytes in flight grow
+// with the resident warps: 6 blocks (40 registers, a few spilled to local
+// memory) measured 1.83 ms per 1 GiB-per-rank launch against 1.95 ms at 4
+// blocks (56 registers, no spill) and 1.90 ms at 5.
+constexpr int kRawMinBlocks = 6;
 
 inline unsigned entry_raw_blocks(int64_t v_count) {
     constexpr int64_t per = (int64_t)kThreads * kRawVPT;
@@ -27,7 +33,7 @@ inline unsigned entry_raw_blocks(int64_t v_count) {
 }
 
 template <int G, int BITS>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kRawMinBlocks)
 echo_entry_raw_kernel(const __grid_constant__ InPtrs x, const __grid_constant__ ChunkDst dst,
                       int64_t n_vec, int64_t chunk_vec, Slab sl, int P, Consts k) {
     constexpr int VPG = G / kVec;            // vectors per group: 4, 8 or 16

@@ -10,6 +10,19 @@
 namespace echo {
 namespace {
 
+// the bounded wait on a barrier that nothing completes (see
+// launch_wait_selftest): its limit must run out
+__global__ void echo_wait_selftest_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(b, 0);
+}
+
 // ---- entry
 template <int G, bool COMP, bool DEFER, int BITS>
 void entry_t(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t er_chunk_vec, Slab sl,
@@ -209,6 +222,19 @@ void launch_rs(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix,
     if (b.bits == 8) rs_b<8>(b, out, owners, sl, fix, st);
     else rs_b<4>(b, out, owners, sl, fix, st);
 }
+
+cudaError_t device_error_read(int32_t *flags, bool clear) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, echo_device_error, sizeof v);
+    if (e == cudaSuccess && clear && v != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(echo_device_error, &zero, sizeof zero);
+    }
+    *flags = v;
+    return e;
+}
+
+void launch_wait_selftest(cudaStream_t st) { echo_wait_selftest_kernel<<<1, 32, 0, st>>>(); }
 
 void launch_fill(float *p, int64_t n, float v, cudaStream_t st) {
     int64_t blocks = (n + kThreads - 1) / kThreads;

@@ -97,4 +97,13 @@ void launch_fixup(const Bufs &b, const float *src_fast, const float *src_slow, f
                   float *dst_slow, int ranks, int owners, bool apply, bool only_owner, Slab sl,
                   cudaStream_t st);
 
+// The library's device error word on the current device (kernels set the
+// kDevErr* bits of echo_stage.cuh in it): *flags = its value, then cleared
+// if clear.  A synchronous copy.
+cudaError_t device_error_read(int32_t *flags, bool clear);
+
+// One block of 32 threads that waits, bounded, on a barrier nothing
+// completes, so that the wait runs out and sets kDevErrWaitTimeout.
+void launch_wait_selftest(cudaStream_t st);
+
 }  // namespace echo

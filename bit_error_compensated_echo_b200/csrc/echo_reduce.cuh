@@ -3,6 +3,7 @@
 #pragma once
 
 #include "echo_common.cuh"
+#include "echo_stage.cuh"
 
 namespace echo {
 
@@ -17,10 +18,12 @@ namespace echo {
 // output residual e_req = s - float(y) is either
 // written out (for a side-stream or deferred fix-up) or, with fix, folded
 // into the owner's states here (state row o, the owner's own chunk).
-// Each thread owns 16 consecutive elements: one 8-byte word pair of codes
-// per rank, all P loads issued before any arithmetic so that every thread
-// keeps P*8 bytes of the transport in flight.
-// Grid: x over the 16-element runs of the slab, y = owner.
+// Each thread owns 16 consecutive elements (a run): one 8-byte word pair of
+// codes per rank (16 bytes at 8 bits), all P loads issued before any
+// arithmetic (sum_run), or, for the configuration where that measured
+// faster, the block's 256 runs of every rank staged in shared memory by bulk
+// copies (stage_sum, see ReduceShape).
+// Grid: x over the slab's runs in blocks of 256, y = owner.
 constexpr int kRedVec = 16;
 
 // blocks along x for a slab of v_count 8-element vectors
@@ -78,6 +81,113 @@ __device__ __forceinline__ void sum_run(const uint32_t *__restrict__ codes,
     }
 }
 
+// The sums of a block's runs: the P ranks' codes of the
+// block's runs [run0, run0 + nrun) (run indices within a rank row) arrive in
+// shared memory by one bulk copy per rank, issued by thread 0 and completing
+// on one mbarrier, and the block's scales by plain loads of all threads (a
+// rank's row of scales need not start on 16 bytes).  Each thread then reads
+// its run's P code words and P scales at fixed offsets from one shared
+// address -- no per-rank address arithmetic -- dequantizes them and adds
+// them in fp32 in ascending rank order from +0.  Threads past the slab
+// (threadIdx.x >= nrun: whole groups, since nrun is a multiple of the lanes
+// of a group) read run 0's codes; their results are not stored.  Returns
+// false in every thread if the copies did not complete within the wait
+// limit (the device error word is then set).
+//
+// Bulk-copy alignment (16 bytes for both addresses and the size): a run is
+// 2*BITS bytes of codes; a rank row is N*BITS/8 bytes and N is a multiple
+// of P*G >= 32; run0 = owner*C/16 + v_begin/2 + 256*blockIdx.x with C = N/P
+// a multiple of G and v_begin a multiple of G/8 >= 4; nrun is even (the
+// slab's run count is a multiple of G/16 >= 2); the code buffer itself is
+// 16-byte aligned (every caller checks or allocates so).
+template <int G, int P, int BITS>
+__device__ __forceinline__ bool stage_sum(const uint32_t *__restrict__ codes,
+                                          const float *__restrict__ scales, int64_t n_vec,
+                                          int64_t run0, int nrun, float2 z, float s[16]) {
+    constexpr int LANES = G / kRedVec;
+    constexpr int WB = 2 * BITS;                    // code bytes of one run
+    constexpr int WORDS = BITS / 2;                 // words holding 16 codes
+    constexpr int GPB = kThreads / LANES;           // groups per block
+    __shared__ __align__(128) uint8_t s_codes[P][kThreads * WB];
+    __shared__ float s_scales[P][GPB];
+    __shared__ __align__(8) uint64_t s_bar;
+    const int t = threadIdx.x;
+    const int64_t n_run = n_vec / 2;
+    const int64_t n_groups = n_run / LANES;
+    const uint32_t bar = smem_u32(&s_bar);
+    if (t == 0) {
+        mbar_init(bar, 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    if (t == 0) {
+        const uint32_t bytes = (uint32_t)nrun * WB;
+        mbar_arrive_expect_tx(bar, (uint32_t)P * bytes);
+#pragma unroll
+        for (int r = 0; r < P; ++r)
+            bulk_copy_g2s(smem_u32(s_codes[r]),
+                          reinterpret_cast<const uint8_t *>(codes) + (r * n_run + run0) * WB,
+                          bytes, bar);
+    }
+    const int ngrp = nrun / LANES;
+    const int64_t g0 = run0 / LANES;
+    for (int i = t; i < P * GPB; i += kThreads) {
+        const int r = i / GPB, g = i - r * GPB;
+        if (g < ngrp) s_scales[r][g] = __ldg(scales + r * n_groups + g0 + g);
+    }
+    const bool arrived = mbar_wait_bounded(bar, 0);
+    if (!__syncthreads_and(arrived)) {
+        // the copies may still be writing this block's shared memory: wait
+        // for them once more (bounded) before the block ends
+        if (t == 0) mbar_wait_bounded(bar, 0);
+        return false;
+    }
+    const int tt = t < nrun ? t : 0;
+    float2 s2[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s2[i] = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int r = 0; r < P; ++r) {
+        uint32_t w[WORDS];
+        if (BITS == 4) {
+            const uint2 v = reinterpret_cast<const uint2 *>(s_codes[r])[tt];
+            w[0] = v.x;
+            w[WORDS - 1] = v.y;
+        } else {
+            const uint4 v = reinterpret_cast<const uint4 *>(s_codes[r])[tt];
+            w[0] = v.x;
+            w[1 % WORDS] = v.y;
+            w[2 % WORDS] = v.z;
+            w[WORDS - 1] = v.w;
+        }
+        const float2 sc2 = splat2(s_scales[r][tt / LANES]);
+        float2 k[8];
+        decode_pairs<BITS, 8>(w, k);
+#pragma unroll
+        for (int p = 0; p < 8; ++p) s2[p] = add2(s2[p], prod2(k[p], sc2, z));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        s[2 * i] = s2[i].x;
+        s[2 * i + 1] = s2[i].y;
+    }
+    return true;
+}
+
+// Which way the reduce reads the transport.  Staging the block's tiles in
+// shared memory (stage_sum) measured faster only for the uncompensated
+// reduce that also writes the P outputs, at G = 128 with 4-bit codes (1 GiB
+// per rank, P=8: 1.87 -> 1.76 ms; its loads then leave the load/store
+// queues to the stores).  Elsewhere the direct loads of sum_run are faster (compensated,
+// 1 GiB per rank: 1.00 ms direct, 1.07 ms staged; uncompensated at G = 32
+// or 64: 1.9 ms direct, 2.3 ms staged): the block-wide wait for its tiles
+// exposes latency that the direct form hides warp by warp, and the address
+// arithmetic that staging removes reappears as uniform instructions.
+template <int G, bool COMP, bool OUT, int BITS>
+struct ReduceShape {
+    static constexpr bool STAGE = !COMP && OUT && G == 128 && BITS == 4;
+};
+
 template <int G, int P, bool COMP, bool OUT, int BITS>
 __global__ void __launch_bounds__(kThreads)
 echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
@@ -93,7 +203,13 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
     const int64_t j = (int64_t)o * chunk_run + sl.v_begin / 2 + local;  // run index in a rank
     const float2 z = splat2(k.neg_zero);
     float s[16];
-    sum_run<G, P, BITS>(codes, scales, n_vec, j, valid, z, s);
+    if (ReduceShape<G, COMP, OUT, BITS>::STAGE) {
+        const int64_t left = sl.v_count / 2 - (local - threadIdx.x);   // runs from the block's first
+        const int nrun = (int)(left < kThreads ? left : kThreads);
+        if (!stage_sum<G, P, BITS>(codes, scales, n_vec, j - threadIdx.x, nrun, z, s)) return;
+    } else {
+        sum_run<G, P, BITS>(codes, scales, n_vec, j, valid, z, s);
+    }
 
     float a = 0.0f;
 #pragma unroll

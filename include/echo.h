@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define ECHO_ABI_VERSION 4
+#define ECHO_ABI_VERSION 5
 #define ECHO_MAX_RANKS 8
 
 typedef enum echo_status {
@@ -68,7 +68,8 @@ typedef enum echo_status {
     ECHO_ERR_UNSUPPORTED = 4, /* P, G or bits outside the supported set */
     ECHO_ERR_OOM = 5,         /* device allocation failed */
     ECHO_ERR_CUDA = 6,        /* a CUDA runtime call failed */
-    ECHO_ERR_TIMEOUT = 7      /* reserved: no kernel here waits on a flag or barrier */
+    ECHO_ERR_TIMEOUT = 7      /* reserved: a kernel whose bounded wait runs out reports
+                               * it in the device error word (echo_device_error_get) */
 } echo_status;
 
 /* Where the owner's requantization error enters its EMA states (step 7).
@@ -326,6 +327,27 @@ int32_t echo_launches_per_call(const echo_plan *plan);
 echo_status echo_allreduce_noalloc(const echo_config *cfg, const void *const *in_device,
                                    void *const *out_device, float *m_fast_device,
                                    float *m_slow_device, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Device error word.  The one kernel here that waits -- the reduce that
+ * stages its blocks' tiles in shared memory with bulk copies (uncompensated
+ * calls at G = 128 with 4-bit codes) waits for those copies -- gives up after 1 s, sets
+ * ECHO_DEVERR_WAIT_TIMEOUT in this library's device error word on its
+ * device and writes none of its outputs; the call that launched it has
+ * already returned ECHO_OK.  echo_device_error_get copies the word of
+ * `device` into *flags (a synchronous copy: read it once the work to check
+ * has finished) and clears it when clear != 0.
+ * Errors: INVALID_ARG (null flags, device < 0), CUDA. */
+#define ECHO_DEVERR_WAIT_TIMEOUT 1
+
+echo_status echo_device_error_get(int32_t device, int32_t *flags, int32_t clear);
+
+/* Self-test of the bounded wait on `device`: one block of 32 threads waits
+ * on a barrier that nothing completes; the wait gives up after its limit
+ * (1 s) and sets ECHO_DEVERR_WAIT_TIMEOUT in the device error word.  Runs on
+ * a stream of its own and blocks the host until the kernel has ended (about
+ * one second).  Errors: INVALID_ARG (device < 0), CUDA. */
+echo_status echo_selftest_wait_limit(int32_t device);
 
 /* Static name of a status code. */
 const char *echo_status_string(echo_status s);

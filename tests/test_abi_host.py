@@ -198,3 +198,26 @@ def test_cross_rank_aggregation_gloo():
     import bench
     v, t = bench.aggregate([3.0, 5.0], [100.0, 300.0])
     assert t == 5.0 and abs(v - 400.0 / 5e-3 / 1e9) < 1e-12
+
+
+def test_bench_kernel_rooflines():
+    """Per-kernel roofline fractions of the bench line: the algorithmic bytes
+    of each kernel over its average launch time; a reduce that writes the
+    outputs (no exit launch) counts them."""
+    import bench
+    P, N, G = 8, 1 << 29, 128
+    prof = {"calls": 10, "entry_ms": 117.0, "reduce_ms": 10.0, "exit_ms": 13.8, "fixup_ms": 0.0}
+    r = bench.kernel_rooflines(prof, P, N, G, True, "deferred", 4, 6543.4)
+    q = 0.5 + 4 / 128
+    assert r["echo_entry"]["bytes"] == P * N * (18 + q) + 4 * N
+    assert r["echo_reduce"]["bytes"] == P * N * q + N * q + 4 * N
+    assert r["echo_exit"]["bytes"] == N * q + 2 * P * N
+    for k in r.values():
+        assert abs(k["achieved"] - k["bytes"] / (k["avg_launch_ms"] / 1e3) / 1e9) < 0.1
+        assert abs(k["frac"] - k["achieved"] / 6543.4) < 1e-3
+    off = dict(prof, exit_ms=0.0)
+    r = bench.kernel_rooflines(off, P, N, G, False, "deferred", 4, 6543.4)
+    assert "echo_exit" not in r
+    assert r["echo_reduce"]["bytes"] == P * N * q + N * q + 2 * P * N
+    small = bench.kernel_rooflines(off, P, 1 << 19, G, True, "exit", 4, 6543.4)
+    assert small["echo_reduce"]["bytes"] == P * (1 << 19) * (q + 2) + (1 << 19) * (q + 16)

@@ -55,3 +55,19 @@ def test_many_plans_created_and_destroyed():
     torch.cuda.synchronize()
     free1, _ = torch.cuda.mem_get_info()
     assert free1 >= free0 - (8 << 20), (free0, free1)
+
+
+def test_bounded_wait_runs_out_and_reports():
+    """A wait that nothing completes gives up after its limit (about one
+    second, not forever), sets ECHO_DEVERR_WAIT_TIMEOUT in the device error
+    word, and leaves the context usable."""
+    import time
+    abi.echo_device_error_get(0, clear=True)
+    assert abi.echo_device_error_get(0) == 0
+    t0 = time.monotonic()
+    abi.echo_selftest_wait_limit(0)
+    took = time.monotonic() - t0
+    assert 0.9 <= took < 30.0, took
+    assert abi.echo_device_error_get(0, clear=True) == abi.ECHO_DEVERR_WAIT_TIMEOUT
+    assert abi.echo_device_error_get(0) == 0
+    _small_call_works()
