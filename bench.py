@@ -127,6 +127,11 @@ def exit_bytes(P: int, N: int, G: int, bits: int = 4) -> float:
     return N * transport_bytes_per_elem(G, bits) + P * N * 2
 
 
+# compensated calls of at most this many elements per rank have no exit
+# launch: their reduce writes the outputs (as every uncompensated call's does)
+MERGE_MAX_N = 1 << 19
+
+
 def kernel_rooflines(prof: dict, P: int, N: int, G: int, comp: bool, fixup: str, bits: int,
                      peak: float) -> dict:
     """Each kernel's algorithmic bytes per launch over its average launch
@@ -134,12 +139,14 @@ def kernel_rooflines(prof: dict, P: int, N: int, G: int, comp: bool, fixup: str,
     When the reduce writes the outputs (no exit launch) its bytes include
     them."""
     calls = max(int(prof["calls"]), 1)
-    merged = prof["exit_ms"] == 0.0
+    merged = not comp or N <= MERGE_MAX_N
     rb = reduce_bytes(P, N, G, comp, fixup, bits) + (P * N * 2 if comp and merged else 0)
+    kernels = [("echo_entry", entry_bytes(P, N, G, comp, fixup, bits), "entry_ms"),
+               ("echo_reduce", rb, "reduce_ms")]
+    if not merged:
+        kernels.append(("echo_exit", exit_bytes(P, N, G, bits), "exit_ms"))
     out = {}
-    for name, b, key in (("echo_entry", entry_bytes(P, N, G, comp, fixup, bits), "entry_ms"),
-                         ("echo_reduce", rb, "reduce_ms"),
-                         ("echo_exit", exit_bytes(P, N, G, bits), "exit_ms")):
+    for name, b, key in kernels:
         ms = prof[key] / calls
         if ms <= 0.0:
             continue
