@@ -242,10 +242,12 @@ ECHO_DEVERR_WAIT_TIMEOUT = 1
 
 def echo_device_error_get(device: int, clear: bool = False) -> int:
     """The library's device error word on `device` (ECHO_DEVERR_* bits),
-    cleared afterwards if `clear`."""
+    cleared afterwards if `clear`.  The C call returns ECHO_ERR_TIMEOUT when
+    a wait ran out; here that is the returned flags, not an exception."""
     flags = ctypes.c_int32()
-    _check(lib.echo_device_error_get(device, ctypes.byref(flags), int(bool(clear))),
-           "echo_device_error_get")
+    rc = lib.echo_device_error_get(device, ctypes.byref(flags), int(bool(clear)))
+    if rc != ECHO_ERR_TIMEOUT:
+        _check(rc, "echo_device_error_get")
     return int(flags.value)
 
 

@@ -650,7 +650,7 @@ echo_status echo_device_error_get(int32_t device, int32_t *flags, int32_t clear)
     DeviceGuard guard(device);
     if (guard.err != cudaSuccess) return ECHO_ERR_CUDA;
     ECHO_TRY(device_error_read(flags, clear != 0));
-    return ECHO_OK;
+    return (*flags & ECHO_DEVERR_WAIT_TIMEOUT) ? ECHO_ERR_TIMEOUT : ECHO_OK;
 }
 
 echo_status echo_selftest_wait_limit(int32_t device) {

@@ -70,20 +70,25 @@ struct ReduceOut {
 template <int G, int P, int BITS>
 void reduce_t(const Bufs &b, int owners, Slab sl, cudaStream_t st, const ReduceOut &ro) {
     dim3 grid(reduce_blocks(sl.v_count), (unsigned)owners);
+    constexpr bool stage_ok = ReduceShape<G, P, false, true, BITS>::STAGE_OK;
     if (b.comp && ro.n_out > 0)
-        echo_reduce_kernel<G, P, true, true, BITS><<<grid, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, true, true, BITS, false><<<grid, kThreads, 0, st>>>(
             b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
             ro.out, ro.n_out, b.m_fast, b.m_slow, ro.fix);
     else if (b.comp)
-        echo_reduce_kernel<G, P, true, false, BITS><<<grid, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, true, false, BITS, false><<<grid, kThreads, 0, st>>>(
             b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
             ro.out, 0, b.m_fast, b.m_slow, ro.fix);
+    else if (ro.n_out > 0 && stage_ok && sl.v_count / 2 >= kStageMinRuns)
+        echo_reduce_kernel<G, P, false, true, BITS, stage_ok><<<grid, kThreads, 0, st>>>(
+            b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
+            ro.out, ro.n_out, nullptr, nullptr, 0);
     else if (ro.n_out > 0)
-        echo_reduce_kernel<G, P, false, true, BITS><<<grid, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, false, true, BITS, false><<<grid, kThreads, 0, st>>>(
             b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
             ro.out, ro.n_out, nullptr, nullptr, 0);
     else
-        echo_reduce_kernel<G, P, false, false, BITS><<<grid, kThreads, 0, st>>>(
+        echo_reduce_kernel<G, P, false, false, BITS, false><<<grid, kThreads, 0, st>>>(
             b.codes, b.scales, b.rcodes, b.rscales, b.e_req, b.n_vec, b.chunk_vec, sl, b.k,
             ro.out, 0, nullptr, nullptr, 0);
 }

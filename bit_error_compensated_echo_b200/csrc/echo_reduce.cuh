@@ -22,7 +22,7 @@ namespace echo {
 // codes per rank (16 bytes at 8 bits), all P loads issued before any
 // arithmetic (sum_run), or, for the configuration where that measured
 // faster, the block's 256 runs of every rank staged in shared memory by bulk
-// copies (stage_sum, see ReduceShape).
+// copies (stage_sum; STAGE, see ReduceShape).
 // Grid: x over the slab's runs in blocks of 256, y = owner.
 constexpr int kRedVec = 16;
 
@@ -176,19 +176,26 @@ __device__ __forceinline__ bool stage_sum(const uint32_t *__restrict__ codes,
 
 // Which way the reduce reads the transport.  Staging the block's tiles in
 // shared memory (stage_sum) measured faster only for the uncompensated
-// reduce that also writes the P outputs, at G = 128 with 4-bit codes (1 GiB
-// per rank, P=8: 1.87 -> 1.76 ms; its loads then leave the load/store
-// queues to the stores).  Elsewhere the direct loads of sum_run are faster (compensated,
-// 1 GiB per rank: 1.00 ms direct, 1.07 ms staged; uncompensated at G = 32
-// or 64: 1.9 ms direct, 2.3 ms staged): the block-wide wait for its tiles
-// exposes latency that the direct form hides warp by warp, and the address
-// arithmetic that staging removes reappears as uniform instructions.
-template <int G, bool COMP, bool OUT, int BITS>
-struct ReduceShape {
-    static constexpr bool STAGE = !COMP && OUT && G == 128 && BITS == 4;
-};
-
+// reduce that also writes the P outputs, at P = 8, G = 128, 4-bit codes and
+// owner chunks of at least 2^20 elements (16 MiB of bf16 per rank; 1 GiB
+// per rank: 1.87 -> 1.76 ms, call 0.89 -> 0.93 of its roofline in the
+// sweep; its loads then leave the load/store queues to the stores).
+// Elsewhere the direct loads of sum_run are faster: compensated (1 GiB per
+// rank: 1.00 ms direct, 1.07 ms staged), uncompensated at G = 32 or 64 (1.9
+// against 2.3 ms), at P = 2 and 4 (the call 1-3 points of its roofline
+// lower), and below 16 MiB per rank (4 MiB, P = 8: 29.7 against 31.7 us).
+// The block-wide wait for the tiles exposes latency that the direct form
+// hides warp by warp, and the address arithmetic that staging removes
+// reappears as uniform instructions.  STAGE_OK says which instances may
+// stage; the launcher picks the staged one only at or above kStageMinRuns
+// runs per owner chunk in the slab.
 template <int G, int P, bool COMP, bool OUT, int BITS>
+struct ReduceShape {
+    static constexpr bool STAGE_OK = !COMP && OUT && G == 128 && BITS == 4 && P == 8;
+};
+constexpr int64_t kStageMinRuns = int64_t(1) << 16;   // 2^20 elements
+
+template <int G, int P, bool COMP, bool OUT, int BITS, bool STAGE>
 __global__ void __launch_bounds__(kThreads)
 echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
                    uint32_t *__restrict__ rcodes, float *__restrict__ rscales,
@@ -203,7 +210,7 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
     const int64_t j = (int64_t)o * chunk_run + sl.v_begin / 2 + local;  // run index in a rank
     const float2 z = splat2(k.neg_zero);
     float s[16];
-    if (ReduceShape<G, COMP, OUT, BITS>::STAGE) {
+    if (STAGE) {
         const int64_t left = sl.v_count / 2 - (local - threadIdx.x);   // runs from the block's first
         const int nrun = (int)(left < kThreads ? left : kThreads);
         if (!stage_sum<G, P, BITS>(codes, scales, n_vec, j - threadIdx.x, nrun, z, s)) return;

@@ -68,8 +68,7 @@ typedef enum echo_status {
     ECHO_ERR_UNSUPPORTED = 4, /* P, G or bits outside the supported set */
     ECHO_ERR_OOM = 5,         /* device allocation failed */
     ECHO_ERR_CUDA = 6,        /* a CUDA runtime call failed */
-    ECHO_ERR_TIMEOUT = 7      /* reserved: a kernel whose bounded wait runs out reports
-                               * it in the device error word (echo_device_error_get) */
+    ECHO_ERR_TIMEOUT = 7      /* a kernel's bounded wait ran out (echo_device_error_get) */
 } echo_status;
 
 /* Where the owner's requantization error enters its EMA states (step 7).
@@ -331,12 +330,13 @@ echo_status echo_allreduce_noalloc(const echo_config *cfg, const void *const *in
 /* ------------------------------------------------------------------------
  * Device error word.  The one kernel here that waits -- the reduce that
  * stages its blocks' tiles in shared memory with bulk copies (uncompensated
- * calls at G = 128 with 4-bit codes) waits for those copies -- gives up after 1 s, sets
+ * calls at P = 8, G = 128, 4-bit codes, N >= 2^23) waits for those copies -- gives up after 1 s, sets
  * ECHO_DEVERR_WAIT_TIMEOUT in this library's device error word on its
  * device and writes none of its outputs; the call that launched it has
  * already returned ECHO_OK.  echo_device_error_get copies the word of
  * `device` into *flags (a synchronous copy: read it once the work to check
- * has finished) and clears it when clear != 0.
+ * has finished), clears it when clear != 0, and returns ECHO_ERR_TIMEOUT
+ * when the word has ECHO_DEVERR_WAIT_TIMEOUT set, ECHO_OK when it is clear.
  * Errors: INVALID_ARG (null flags, device < 0), CUDA. */
 #define ECHO_DEVERR_WAIT_TIMEOUT 1
 

@@ -1,6 +1,10 @@
 """Failure paths on the GPU that fault nothing: a plan whose workspace
 cannot be allocated returns ECHO_ERR_OOM (the CUDA error is cleared, not
-left sticky), and the context stays usable for the next plan and call."""
+left sticky), a kernel wait that runs out is reported as ECHO_ERR_TIMEOUT
+through the device error word, and the context stays usable for the next
+plan and call."""
+import ctypes
+
 import pytest
 import torch
 
@@ -68,6 +72,11 @@ def test_bounded_wait_runs_out_and_reports():
     abi.echo_selftest_wait_limit(0)
     took = time.monotonic() - t0
     assert 0.9 <= took < 30.0, took
+    flags = ctypes.c_int32()
+    # the C call reports the run-out wait as ECHO_ERR_TIMEOUT
+    assert abi.lib.echo_device_error_get(0, ctypes.byref(flags), 0) == abi.ECHO_ERR_TIMEOUT
+    assert flags.value == abi.ECHO_DEVERR_WAIT_TIMEOUT
     assert abi.echo_device_error_get(0, clear=True) == abi.ECHO_DEVERR_WAIT_TIMEOUT
+    assert abi.lib.echo_device_error_get(0, ctypes.byref(flags), 0) == abi.ECHO_OK
     assert abi.echo_device_error_get(0) == 0
     _small_call_works()

@@ -355,3 +355,19 @@ def test_message_beyond_int32_elements(comp):
         del x, out
     torch.cuda.empty_cache()
 
+
+
+def test_staged_reduce_every_element_ragged():
+    """The uncompensated reduce that stages its code tiles in shared memory
+    (P=8, G=128, owner chunks of at least 2^20 elements): owner chunks of
+    2^20 + 384 elements, so each owner's last block of 256 runs is partial
+    (24 runs); two calls, every element against the oracle."""
+    P, G = 8, 128
+    C = (1 << 20) + 3 * G
+    N = P * C
+    assert (C // 16) % 256 == 24
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    with _plan(P, N, G, False) as plan:
+        chk = SequenceChecker(plan, oracle_params(plan))
+        for t in range(2):
+            chk.step(W.generate(w, t, DEV))
