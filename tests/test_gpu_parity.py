@@ -233,6 +233,25 @@ def test_host_call_uncompensated_large_slabs():
         assert torch.equal(yd.cpu(), yh)
 
 
+def test_host_call_uncompensated_staged_slabs():
+    """512 MiB per rank, P=8, G=128: each of the host call's 32 slabs holds
+    2^17 runs of every owner chunk, so its reduce stages the code tiles in
+    shared memory; in place on pinned memory, its outputs equal the device
+    call's."""
+    N = 1 << 28
+    w = W.with_size(W.LARGE, P=8, rows=1, hidden=N, G=128)
+    with _plan(w.P, N, w.G, False) as a, _plan(w.P, N, w.G, False) as b:
+        x = W.generate(w, 0, DEV)
+        yd = a.allreduce(x).cpu()
+        xh = x.cpu().pin_memory()
+        del x
+        b.allreduce_host(xh, xh)
+        torch.cuda.synchronize()
+        assert torch.equal(yd, xh)
+        del yd, xh
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("comp", [True, False])
 def test_host_call_in_place(comp):
     """The host call with out_host == in_host (the bench's end-to-end leg)
