@@ -132,19 +132,33 @@ def exit_bytes(P: int, N: int, G: int, bits: int = 4) -> float:
 MERGE_MAX_N = 1 << 19
 
 
+def rs_kernel_bytes(P: int, N: int, G: int, comp: bool, fixup: str, bits: int = 4) -> float:
+    """Algorithmic bytes of the reduce-scatter's second kernel (echo_rs): read
+    the entry transport (P*q per element of N), write each owner's bf16
+    chunk (2); compensated, write the owner residual (4) or, with the fix-up
+    in the kernel, read and write the owner's states (16)."""
+    b = P * N * transport_bytes_per_elem(G, bits) + 2 * N
+    if comp:
+        b += N * (16 if fixup == "exit" else 4)
+    return b
+
+
 def kernel_rooflines(prof: dict, P: int, N: int, G: int, comp: bool, fixup: str, bits: int,
-                     peak: float) -> dict:
+                     peak: float, rs: bool = False) -> dict:
     """Each kernel's algorithmic bytes per launch over its average launch
     time (the plan's CUDA events on the launch stream), against the HBM peak.
     When the reduce writes the outputs (no exit launch) its bytes include
-    them."""
+    them; for a reduce-scatter call the second kernel is echo_rs."""
     calls = max(int(prof["calls"]), 1)
     merged = not comp or N <= MERGE_MAX_N
     rb = reduce_bytes(P, N, G, comp, fixup, bits) + (P * N * 2 if comp and merged else 0)
-    kernels = [("echo_entry", entry_bytes(P, N, G, comp, fixup, bits), "entry_ms"),
-               ("echo_reduce", rb, "reduce_ms")]
-    if not merged:
-        kernels.append(("echo_exit", exit_bytes(P, N, G, bits), "exit_ms"))
+    kernels = [("echo_entry", entry_bytes(P, N, G, comp, fixup, bits), "entry_ms")]
+    if rs:
+        kernels.append(("echo_rs", rs_kernel_bytes(P, N, G, comp, fixup, bits), "reduce_ms"))
+    else:
+        kernels.append(("echo_reduce", rb, "reduce_ms"))
+        if not merged:
+            kernels.append(("echo_exit", exit_bytes(P, N, G, bits), "exit_ms"))
     out = {}
     for name, b, key in kernels:
         ms = prof[key] / calls
@@ -571,8 +585,8 @@ def run_step_mode(args, ws, rank, local):
                          "algorithmic_bytes": eb, "avg_launch_ms": round(entry_ms, 4)},
             "kernels_ms": {k: round(prof[k] / max(calls, 1), 4)
                            for k in ("entry_ms", "reduce_ms", "exit_ms", "fixup_ms")},
-            "kernels_roofline": (None if rs else
-                                 kernel_rooflines(prof, P, N, G, comp, fixup, args.bits, peak)),
+            "kernels_roofline": kernel_rooflines(prof, P, N, G, comp, fixup, args.bits, peak,
+                                                 rs=rs),
             "gpu_launches": int(prof["launches"]),
             "e2e": e2e, "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_par,
             "host": host_info() if cpu else None, "parity": parity, "clocks": clk,

@@ -221,3 +221,7 @@ def test_bench_kernel_rooflines():
     assert r["echo_reduce"]["bytes"] == P * N * q + N * q + 2 * P * N
     small = bench.kernel_rooflines(off, P, 1 << 19, G, True, "exit", 4, 6543.4)
     assert small["echo_reduce"]["bytes"] == P * (1 << 19) * (q + 2) + (1 << 19) * (q + 16)
+    rs = bench.kernel_rooflines(dict(prof, exit_ms=0.0028), P, N, G, True, "deferred", 4,
+                                6543.4, rs=True)
+    assert set(rs) == {"echo_entry", "echo_rs"}
+    assert rs["echo_rs"]["bytes"] == P * N * q + 2 * N + 4 * N
