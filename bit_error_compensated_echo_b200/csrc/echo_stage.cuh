@@ -20,7 +20,11 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s
 constexpr int kDevErrWaitTimeout = 1;
 
 // The device error word of this library on each device (one per context
-// that loads the kernels).  Only kernels set bits in it; the host reads it.
+// that loads the kernels).  Only kernels set bits in it; the host reads it
+// (device_error_read).  Being a static in a header, it is one variable only
+// because a single translation unit -- echo_launch.cu, the one that
+// instantiates the kernels and holds device_error_read -- includes this
+// file; another unit that included it would set a copy the host never reads.
 static __device__ int echo_device_error;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
