@@ -135,18 +135,27 @@ void exit_b(const Bufs &b, const ChunkSrc &src, const OutPtrs &out, int n_out, i
 }
 
 // ---- reduce-scatter
-template <int G, int P, int BITS>
-void rs_t(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix, cudaStream_t st) {
+template <int G, int P, int BITS, bool STAGE>
+void rs_s(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix, cudaStream_t st) {
     dim3 grid(reduce_blocks(sl.v_count), (unsigned)owners);
     if (!b.comp)
-        echo_rs_kernel<G, P, false, false, BITS><<<grid, kThreads, 0, st>>>(
+        echo_rs_kernel<G, P, false, false, BITS, STAGE><<<grid, kThreads, 0, st>>>(
             b.codes, b.scales, out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec, sl, b.k);
     else if (fix)
-        echo_rs_kernel<G, P, true, true, BITS><<<grid, kThreads, 0, st>>>(
+        echo_rs_kernel<G, P, true, true, BITS, STAGE><<<grid, kThreads, 0, st>>>(
             b.codes, b.scales, out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec, sl, b.k);
     else
-        echo_rs_kernel<G, P, true, false, BITS><<<grid, kThreads, 0, st>>>(
+        echo_rs_kernel<G, P, true, false, BITS, STAGE><<<grid, kThreads, 0, st>>>(
             b.codes, b.scales, out, b.m_fast, b.m_slow, b.e_req, b.n_vec, b.chunk_vec, sl, b.k);
+}
+
+template <int G, int P, int BITS>
+void rs_t(const Bufs &b, const OutPtrs &out, int owners, Slab sl, bool fix, cudaStream_t st) {
+    constexpr bool stage_ok = RsShape<G, P, BITS>::STAGE_OK;
+    if (stage_ok && sl.v_count / 2 >= kStageMinRuns)
+        rs_s<G, P, BITS, stage_ok>(b, out, owners, sl, fix, st);
+    else
+        rs_s<G, P, BITS, false>(b, out, owners, sl, fix, st);
 }
 
 template <int G, int BITS>

@@ -195,6 +195,17 @@ struct ReduceShape {
 };
 constexpr int64_t kStageMinRuns = int64_t(1) << 16;   // 2^20 elements
 
+// The reduce-scatter's kernel (echo_rs) is bound by the wait for its loads
+// (ncu: long scoreboard the top stall, issue 37% busy), and staging its
+// tiles measured faster at P = 8, G = 128, 4-bit codes (1 GiB per rank,
+// compensated: 1.23 -> 0.98 ms, the call 13.02 -> 12.82 ms; 16 MiB per
+// rank: 29 -> 24 us), slower at G = 32 (1.25 -> 1.39 ms) and at P = 2
+// (0.82 -> 0.85 ms).  The same size threshold applies.
+template <int G, int P, int BITS>
+struct RsShape {
+    static constexpr bool STAGE_OK = G == 128 && BITS == 4 && P == 8;
+};
+
 template <int G, int P, bool COMP, bool OUT, int BITS, bool STAGE>
 __global__ void __launch_bounds__(kThreads)
 echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
@@ -293,7 +304,8 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
 // side-stream or deferred fix-up (COMP && !FIX).
 // Grid: x over the 16-element runs of the slab, y = owner (out is a
 // __grid_constant__ parameter, indexed by the owner without a local copy).
-template <int G, int P, bool COMP, bool FIX, int BITS>
+// STAGE: the P code tiles staged in shared memory (stage_sum, see RsShape).
+template <int G, int P, bool COMP, bool FIX, int BITS, bool STAGE>
 __global__ void __launch_bounds__(kThreads)
 echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ scales,
                const __grid_constant__ OutPtrs out,
@@ -302,12 +314,19 @@ echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ sca
     const int o = blockIdx.y;
     const int64_t chunk_run = chunk_vec / 2;
     const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (local >= sl.v_count / 2) return;    // no shuffles below: lanes may leave
     const int64_t lr = sl.v_begin / 2 + local;          // run index within chunk o
     const int64_t j = (int64_t)o * chunk_run + lr;       // run index within a rank
     const float2 z = splat2(k.neg_zero);
     float s[16];
-    sum_run<G, P, BITS>(codes, scales, n_vec, j, true, z, s);
+    if (STAGE) {   // every thread takes part in the staging's barriers
+        const int64_t left = sl.v_count / 2 - (local - threadIdx.x);   // runs from the block's first
+        const int nrun = (int)(left < kThreads ? left : kThreads);
+        if (!stage_sum<G, P, BITS>(codes, scales, n_vec, j - threadIdx.x, nrun, z, s)) return;
+        if ((int)threadIdx.x >= nrun) return;   // no shuffles below: lanes may leave
+    } else {
+        if (local >= sl.v_count / 2) return;    // no shuffles below: lanes may leave
+        sum_run<G, P, BITS>(codes, scales, n_vec, j, true, z, s);
+    }
 
     uint32_t yw[8];
 #pragma unroll

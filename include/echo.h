@@ -328,12 +328,13 @@ echo_status echo_allreduce_noalloc(const echo_config *cfg, const void *const *in
                                    float *m_slow_device, void *stream);
 
 /* ------------------------------------------------------------------------
- * Device error word.  The one kernel here that waits -- the reduce that
- * stages its blocks' tiles in shared memory with bulk copies (uncompensated
- * calls at P = 8, G = 128, 4-bit codes, N >= 2^23) waits for those copies -- gives up after 1 s, sets
- * ECHO_DEVERR_WAIT_TIMEOUT in this library's device error word on its
- * device and writes none of its outputs; the call that launched it has
- * already returned ECHO_OK.  echo_device_error_get copies the word of
+ * Device error word.  Two kernels here wait: the reduce and the
+ * reduce-scatter kernel, when they stage their blocks' tiles in shared
+ * memory with bulk copies (P = 8, G = 128, 4-bit codes, N >= 2^23; for the
+ * all-reduce only uncompensated calls), wait for those copies.  A wait
+ * gives up after 1 s, sets ECHO_DEVERR_WAIT_TIMEOUT in this library's device
+ * error word on its device, and the kernel writes none of its outputs; the
+ * call that launched it has already returned ECHO_OK.  echo_device_error_get copies the word of
  * `device` into *flags (a synchronous copy: read it once the work to check
  * has finished), clears it when clear != 0, and returns ECHO_ERR_TIMEOUT
  * when the word has ECHO_DEVERR_WAIT_TIMEOUT set, ECHO_OK when it is clear.

@@ -72,3 +72,23 @@ def test_rs_profile_counts_two_launches():
             plan.reduce_scatter(W.generate(w, t, DEV))
         p = plan.profile_read(reset=True)
         assert p["calls"] == 3 and p["launches"] == 6
+
+
+@pytest.mark.parametrize("comp,fixup", [(True, "exit"), (True, "side"), (True, "deferred"),
+                                        (False, "deferred")])
+def test_rs_staged_every_element_ragged(comp, fixup):
+    """The reduce-scatter kernel that stages its code tiles in shared memory
+    (P=8, G=128, owner chunks of at least 2^20 elements): owner chunks of
+    2^20 + 384 elements, so each owner's last block of 256 runs is partial
+    (24 runs); two calls, every element of the owners' outputs and both
+    states against the oracle."""
+    P, G = 8, 128
+    C = (1 << 20) + 3 * G
+    N = P * C
+    assert (C // 16) % 256 == 24
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    side = torch.cuda.Stream() if fixup == "side" else None
+    with EchoPlan(P, N, G, compensate=comp, fixup=fixup, device=0) as plan:
+        chk = RSChecker(plan, oracle_params(plan))
+        for t in range(2):
+            chk.step_rs(W.generate(w, t, DEV), side_stream=side)
