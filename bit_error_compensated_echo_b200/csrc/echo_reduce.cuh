@@ -176,12 +176,14 @@ __device__ __forceinline__ bool stage_sum(const uint32_t *__restrict__ codes,
 
 // Which way the reduce reads the transport.  Staging the block's tiles in
 // shared memory (stage_sum) measured faster only for the uncompensated
-// reduce that also writes the P outputs, at P = 8, G = 128, 4-bit codes and
-// owner chunks of at least 2^20 elements (16 MiB of bf16 per rank; 1 GiB
-// per rank: 1.87 -> 1.76 ms, call 0.89 -> 0.93 of its roofline in the
-// sweep; its loads then leave the load/store queues to the stores).
+// reduce that also writes the P outputs, at P = 8, G = 128 and owner
+// chunks of at least 2^20 elements (16 MiB of bf16 per rank; 1 GiB per
+// rank, 4-bit codes: 1.87 -> 1.76 ms, call 0.89 -> 0.93 of its roofline in
+// the sweep; 8-bit codes: 2.29 -> 2.10 ms; its loads then leave the
+// load/store queues to the stores).
 // Elsewhere the direct loads of sum_run are faster: compensated (1 GiB per
-// rank: 1.00 ms direct, 1.07 ms staged), uncompensated at G = 32 or 64 (1.9
+// rank: 1.00 ms direct, 1.07 ms staged; 8-bit 1.21 against 1.24 ms),
+// uncompensated at G = 32 or 64 (1.9
 // against 2.3 ms), at P = 2 and 4 (the call 1-3 points of its roofline
 // lower), and below 16 MiB per rank (4 MiB, P = 8: 29.7 against 31.7 us).
 // The block-wide wait for the tiles exposes latency that the direct form
@@ -191,19 +193,20 @@ __device__ __forceinline__ bool stage_sum(const uint32_t *__restrict__ codes,
 // runs per owner chunk in the slab.
 template <int G, int P, bool COMP, bool OUT, int BITS>
 struct ReduceShape {
-    static constexpr bool STAGE_OK = !COMP && OUT && G == 128 && BITS == 4 && P == 8;
+    static constexpr bool STAGE_OK = !COMP && OUT && G == 128 && P == 8;
 };
 constexpr int64_t kStageMinRuns = int64_t(1) << 16;   // 2^20 elements
 
 // The reduce-scatter's kernel (echo_rs) is bound by the wait for its loads
 // (ncu: long scoreboard the top stall, issue 37% busy), and staging its
-// tiles measured faster at P = 8, G = 128, 4-bit codes (1 GiB per rank,
-// compensated: 1.23 -> 0.98 ms, the call 13.02 -> 12.82 ms; 16 MiB per
-// rank: 29 -> 24 us), slower at G = 32 (1.25 -> 1.39 ms) and at P = 2
+// tiles measured faster at P = 8, G = 128 (1 GiB per rank, compensated,
+// 4-bit codes: 1.23 -> 0.98 ms, the call 13.02 -> 12.82 ms; 8-bit codes:
+// 1.38 -> 1.10 ms; uncompensated 0.77 -> 0.70 and 0.82 -> 0.78 ms; 16 MiB
+// per rank: 29 -> 24 us), slower at G = 32 (1.25 -> 1.39 ms) and at P = 2
 // (0.82 -> 0.85 ms).  The same size threshold applies.
 template <int G, int P, int BITS>
 struct RsShape {
-    static constexpr bool STAGE_OK = G == 128 && BITS == 4 && P == 8;
+    static constexpr bool STAGE_OK = G == 128 && P == 8;
 };
 
 template <int G, int P, bool COMP, bool OUT, int BITS, bool STAGE>

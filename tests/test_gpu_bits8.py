@@ -143,3 +143,26 @@ def test_set_bits_limits():
                 p8.set_bits(bad)
         p8.set_bits(4)
         assert p8.debug_view()["codes"].shape == (2, 2 * 32 * 4 // 2)
+
+
+@pytest.mark.parametrize("op,comp", [("allreduce", False), ("reduce_scatter", True),
+                                     ("reduce_scatter", False)])
+def test_staged_8bit_every_element_ragged(op, comp):
+    """The kernels that stage their code tiles in shared memory, at 8 bits
+    (P=8, G=128, owner chunks of at least 2^20 elements): the uncompensated
+    reduce that writes the outputs and the reduce-scatter kernel.  Owner
+    chunks of 2^20 + 384 elements (each owner's last block of 256 runs holds
+    24); two calls, every element against the oracle."""
+    P, G = 8, 128
+    C = (1 << 20) + 3 * G
+    N = P * C
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    with _plan(P, N, G, comp, "deferred") as plan:
+        if op == "allreduce":
+            chk = SequenceChecker(plan, oracle_params(plan))
+            for t in range(2):
+                chk.step(W.generate(w, t, DEV))
+        else:
+            chk = RSChecker(plan, oracle_params(plan))
+            for t in range(2):
+                chk.step_rs(W.generate(w, t, DEV))
