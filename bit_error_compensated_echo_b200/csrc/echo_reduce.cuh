@@ -202,11 +202,13 @@ constexpr int64_t kStageMinRuns = int64_t(1) << 16;   // 2^20 elements
 // tiles measured faster at P = 8, G = 128 (1 GiB per rank, compensated,
 // 4-bit codes: 1.23 -> 0.98 ms, the call 13.02 -> 12.82 ms; 8-bit codes:
 // 1.38 -> 1.10 ms; uncompensated 0.77 -> 0.70 and 0.82 -> 0.78 ms; 16 MiB
-// per rank: 29 -> 24 us), slower at G = 32 (1.25 -> 1.39 ms) and at P = 2
-// (0.82 -> 0.85 ms).  The same size threshold applies.
+// per rank: 29 -> 24 us) and at P = 8, G = 64 (1.18 -> 1.07 ms); slower at
+// G = 32 (1.25 -> 1.39 ms), at P = 2 (0.82 -> 0.85 ms) and at P = 4 (even at
+// G = 128, worse at G = 64: 0.88 -> 0.90 ms).  The same size threshold
+// applies.
 template <int G, int P, int BITS>
 struct RsShape {
-    static constexpr bool STAGE_OK = G == 128 && P == 8;
+    static constexpr bool STAGE_OK = P == 8 && G >= 64;
 };
 
 template <int G, int P, bool COMP, bool OUT, int BITS, bool STAGE>

@@ -330,8 +330,9 @@ echo_status echo_allreduce_noalloc(const echo_config *cfg, const void *const *in
 /* ------------------------------------------------------------------------
  * Device error word.  Two kernels here wait: the reduce and the
  * reduce-scatter kernel, when they stage their blocks' tiles in shared
- * memory with bulk copies (P = 8, G = 128, N >= 2^23; for the all-reduce
- * only uncompensated calls), wait for those copies.  A wait
+ * memory with bulk copies (P = 8, N >= 2^23; the all-reduce only for
+ * uncompensated calls at G = 128, the reduce-scatter at G = 64 and 128),
+ * wait for those copies.  A wait
  * gives up after 1 s, sets ECHO_DEVERR_WAIT_TIMEOUT in this library's device
  * error word on its device, and the kernel writes none of its outputs; the
  * call that launched it has already returned ECHO_OK.  echo_device_error_get copies the word of
