@@ -199,3 +199,35 @@ def test_rank_group_mixed_widths():
             _compare_wires(grp, plan, t)
             for a, b in zip(grp.get_state(), plan.get_state()):
                 _same("state", a, b, t)
+
+
+@pytest.mark.parametrize("transport", ["copies", "peers"])
+def test_rank_reduce_scatter_staged_size_against_oracle(transport):
+    """P=8 ranks of 2048 x 4096 (owner chunks of 2^20 elements, where the
+    reduce-scatter kernel stages the received code tiles in shared memory):
+    three reduce-scatter calls of the rank group, deferred fix-up, against
+    the oracle on 258 sampled group columns -- every rank's chunk of the
+    sum and both states."""
+    from rank_emulation import EmulatedPeerGroup
+    wl = W.LLAMA
+    P, N, G = wl.P, wl.N, wl.G
+    cols = W.column_sample(wl, 256, seed=5)
+    idx = torch.from_numpy(W.column_elements(cols, G)).to(DEV)
+    prm = oracle.Params(P=P, N=N, G=G, compensate=True)
+    mf = np.zeros((P, idx.numel()), np.float32)
+    ms = np.zeros_like(mf)
+    C = N // P
+    group = EmulatedGroup if transport == "copies" else EmulatedPeerGroup
+    with group(P, N, G, fixup="deferred") as grp:
+        for t in range(3):
+            x = W.generate(wl, t, DEV)
+            y = grp.reduce_scatter(x)           # [P, C]: row r = rank r's chunk
+            torch.cuda.synchronize()
+            ref = oracle.reduce_scatter(prm, _bits_u16(x.index_select(1, idx)), mf, ms, cols)
+            got = y.reshape(-1).index_select(0, idx)   # element i of the sum at [i // C][i % C]
+            assert_same("owner outputs", _bits_u16(got), ref.y, "bf16", t)
+            gmf, gms = grp.get_state()
+            assert_same("m_fast", _f32(gmf.index_select(1, idx)), mf, "f32", t)
+            assert_same("m_slow", _f32(gms.index_select(1, idx)), ms, "f32", t)
+            del gmf, gms
+    assert C >= 1 << 20
