@@ -657,6 +657,7 @@ def run_sweep_mode(args, ws, rank, local):
     flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     rows = []
+    copy_rate = {}   # (P, N) -> bytes/s of a plain device copy of the same tensors
     points = W.sweep()
     if args.sweep_max_mib:
         points = [w for w in points if w.N * 2 <= args.sweep_max_mib << 20]
@@ -675,6 +676,13 @@ def run_sweep_mode(args, ws, rank, local):
         torch.cuda.synchronize()
         t_graph = _time_calls(g.replay, args.steps, flush, stream)
         del g
+        if (w.P, w.N) not in copy_rate:
+            # calibration only (not the path): the rate a plain copy of the
+            # inputs into the outputs reaches at this size, timed the same way
+            for _ in range(3):
+                out.copy_(x)
+            t_copy = _time_calls(lambda: out.copy_(x), args.steps, flush, stream)
+            copy_rate[(w.P, w.N)] = 4 * w.P * w.N / (t_copy / 1e3)
         bmin = call_min_bytes(w.P, w.N, w.G, w.compensate)
         q = transport_bytes_per_elem(w.G)
         row = {"mode": "sweep", "point": w.name, "MiB_per_rank": w.N * 2 // (1 << 20), "P": w.P,
@@ -682,7 +690,9 @@ def run_sweep_mode(args, ws, rank, local):
                "ms_graph": round(t_graph, 4),
                "input_gbs": round(2 * w.P * w.N / (min(t_eager, t_graph) / 1e3) / 1e9, 2),
                "roofline_frac": round(bmin / peak / (min(t_eager, t_graph) / 1e3) / 1e9, 4),
-               "min_bytes": bmin, "packed_ratio": q / 2}
+               "min_bytes": bmin, "packed_ratio": q / 2,
+               "copy_gbs": round(copy_rate[(w.P, w.N)] / 1e9, 1),
+               "frac_of_copy": round(bmin / (min(t_eager, t_graph) / 1e3) / copy_rate[(w.P, w.N)], 4)}
         dv = plan.debug_view()
         row["packed_ratio_allocated"] = (dv["codes"].numel() + 4 * dv["scales"].numel()) / (2.0 * w.P * w.N)
         rows.append(row)
@@ -692,13 +702,14 @@ def run_sweep_mode(args, ws, rank, local):
         torch.cuda.empty_cache()
     if args.sweep_table:
         with open(args.sweep_table, "w") as f:
-            f.write("| MiB/rank | P | G | mode | ms eager | ms graph | input GB/s | % of call roofline | packed/bf16 |\n")
-            f.write("|---|---|---|---|---|---|---|---|---|\n")
+            f.write("| MiB/rank | P | G | mode | ms eager | ms graph | input GB/s | % of call roofline "
+                    "| same-size copy GB/s | % of same-size copy | packed/bf16 |\n")
+            f.write("|---|---|---|---|---|---|---|---|---|---|---|\n")
             for r in rows:
-                f.write("| %d | %d | %d | %s | %.4f | %.4f | %.1f | %.1f | %.6f |\n" % (
+                f.write("| %d | %d | %d | %s | %.4f | %.4f | %.1f | %.1f | %.1f | %.1f | %.6f |\n" % (
                     r["MiB_per_rank"], r["P"], r["G"], "comp" if r["compensate"] else "off",
                     r["ms_eager"], r["ms_graph"], r["input_gbs"], 100 * r["roofline_frac"],
-                    r["packed_ratio"]))
+                    r["copy_gbs"], 100 * r["frac_of_copy"], r["packed_ratio"]))
 
 
 def run_overlap_mode(args, ws, rank, local):
