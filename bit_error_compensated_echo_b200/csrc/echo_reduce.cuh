@@ -22,7 +22,8 @@ namespace echo {
 // codes per rank (16 bytes at 8 bits), all P loads issued before any
 // arithmetic (sum_run), or, for the configuration where that measured
 // faster, the block's 256 runs of every rank staged in shared memory by bulk
-// copies (stage_sum; STAGE, see ReduceShape).
+// copies (stage_sum; STAGE, see ReduceShape).  Its 32 bytes of each output
+// and 64 bytes of e_req leave as 32-byte stores where the buffer allows.
 // Grid: x over the slab's runs in blocks of 256, y = owner.
 constexpr int kRedVec = 16;
 
@@ -261,8 +262,12 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
         for (int r = 0; r < kMaxRanks; ++r) {
             if (r < n_out) {
                 uint4 *dst = out.p[r] + j * 2;
-                __stcs(dst, make_uint4(yw[0], yw[1], yw[2], yw[3]));
-                __stcs(dst + 1, make_uint4(yw[4], yw[5], yw[6], yw[7]));
+                if (aligned32(out.p[r])) {
+                    st32_words_cs(dst, yw);
+                } else {
+                    __stcs(dst, make_uint4(yw[0], yw[1], yw[2], yw[3]));
+                    __stcs(dst + 1, make_uint4(yw[4], yw[5], yw[6], yw[7]));
+                }
             }
         }
     }
@@ -294,8 +299,7 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
                 st8(m_slow + e0 + 8 * h, ms);
             }
         } else {
-            st8(e_req + j * kRedVec, e);
-            st8(e_req + j * kRedVec + 8, e + 8);
+            store_run16(e_req, j, e);
         }
     }
 }
@@ -337,8 +341,12 @@ echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ sca
 #pragma unroll
     for (int i = 0; i < 8; ++i) yw[i] = bf16x2_bits_rn(make_float2(s[2 * i], s[2 * i + 1]));
     uint4 *dst = out.p[o] + lr * 2;
-    dst[0] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
-    dst[1] = make_uint4(yw[4], yw[5], yw[6], yw[7]);
+    if (aligned32(out.p[o])) {
+        st32_words(dst, yw);
+    } else {
+        dst[0] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+        dst[1] = make_uint4(yw[4], yw[5], yw[6], yw[7]);
+    }
     if (COMP) {
         float e[16];
 #pragma unroll
@@ -367,8 +375,7 @@ echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ sca
                 st8(m_slow + e0 + 8 * h, ms);
             }
         } else {
-            st8(e_req + j * kRedVec, e);
-            st8(e_req + j * kRedVec + 8, e + 8);
+            store_run16(e_req, j, e);
         }
     }
 }

@@ -132,6 +132,39 @@ def test_in_place():
             assert torch.equal(ref, y)
 
 
+@pytest.mark.parametrize("P,G,k,comp", [(8, 128, 1 << 13, False), (4, 32, 37, False),
+                                         (4, 32, 37, True), (8, 128, 64, True)],
+                         ids=["off-staged", "off", "comp-merged", "comp-merged-p8"])
+def test_outputs_aligned_to_16_bytes_only(P, G, k, comp):
+    """Outputs that start 16 bytes past a 32-byte boundary (the ABI asks for
+    16-byte alignment; the kernels' 32-byte stores must then fall back):
+    the same bits as outputs on aligned buffers, for all-reduce calls whose
+    reduce writes the outputs (staged and direct) and for reduce-scatter."""
+    N = P * G * k
+    C = N // P
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    stride = N + 16                               # elements: a 32-byte multiple
+    buf = torch.empty(8 + P * stride, dtype=torch.bfloat16, device=DEV)
+    ys = [buf[8 + r * stride:8 + r * stride + N] for r in range(P)]
+    zs = [buf[8 + r * stride:8 + r * stride + C] for r in range(P)]
+    assert all(t.data_ptr() % 32 == 16 for t in ys + zs)
+    with _plan(P, N, G, comp, "deferred") as a, _plan(P, N, G, comp, "deferred") as b:
+        for t in range(3):
+            x = W.generate(w, t, DEV)
+            a.allreduce(x, out=ys)
+            want = b.allreduce(x)
+            assert torch.equal(torch.stack(ys).view(torch.int16), want.view(torch.int16)), t
+        x = W.generate(w, 7, DEV)
+        a.reduce_scatter(x, out=zs)
+        want = b.reduce_scatter(x)
+        assert torch.equal(torch.stack(zs).view(torch.int16), want.view(torch.int16))
+        if comp:
+            fa, sa = a.get_state()
+            fb, sb = b.get_state()
+            assert torch.equal(fa.view(torch.int32), fb.view(torch.int32))
+            assert torch.equal(sa.view(torch.int32), sb.view(torch.int32))
+
+
 def test_p1_identity_of_codes():
     """P=1: the requantization reproduces the entry codes."""
     w = W.with_size(W.TINY, P=1, rows=1, hidden=128 * 40, G=128)
