@@ -412,6 +412,42 @@ __device__ __forceinline__ void st32_words_cs(void *p, const uint32_t w[8]) {
                  : "memory");
 }
 
+__device__ __forceinline__ void ld32(const float *p, float v[8]) {
+    asm volatile("ld.global.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]),
+                   "=f"(v[6]), "=f"(v[7])
+                 : "l"(p));
+}
+
+// 8 floats at p (32 bytes): one 32-byte access when wide (p 32-byte aligned),
+// else two 16-byte ones
+__device__ __forceinline__ void ld8w(const float *p, float v[8], bool wide) {
+    if (wide) ld32(p, v);
+    else ld8(p, v);
+}
+__device__ __forceinline__ void st8w(float *p, const float v[8], bool wide) {
+    if (wide) st32(p, v);
+    else st8(p, v);
+}
+
+// 16 bf16 values (8 words) to the same 32 bytes of each of the n_out
+// outputs, streamed: out.p[r] + run * 2 in 16-byte units
+__device__ __forceinline__ void store_run_outputs(const OutPtrs &out, int n_out, int64_t run,
+                                                  const uint32_t yw[8]) {
+#pragma unroll
+    for (int r = 0; r < kMaxRanks; ++r) {
+        if (r < n_out) {
+            uint4 *dst = out.p[r] + run * 2;
+            if (aligned32(out.p[r])) {
+                st32_words_cs(dst, yw);
+            } else {
+                __stcs(dst, make_uint4(yw[0], yw[1], yw[2], yw[3]));
+                __stcs(dst + 1, make_uint4(yw[4], yw[5], yw[6], yw[7]));
+            }
+        }
+    }
+}
+
 // the 16 floats of run `run` of a buffer of 16-float runs
 __device__ __forceinline__ void store_run16(float *base, int64_t run, const float v[16]) {
     float *p = base + run * 16;

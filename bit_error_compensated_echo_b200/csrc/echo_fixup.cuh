@@ -20,25 +20,28 @@ echo_fixup_kernel(const float *__restrict__ src_fast, const float *__restrict__ 
     const int64_t local = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     if (local >= sl.v_count) return;
     const int o = blockIdx.y;
+    // 32-byte accesses where every buffer allows (offsets are multiples of 32 bytes)
+    const bool wide = aligned32(src_fast) && aligned32(src_slow) && aligned32(dst_fast) &&
+                      aligned32(dst_slow) && aligned32(e_req);
     for (int r = 0; r < P; ++r) {
         const bool own = (r == o);
         if (only_owner && !own) continue;
         const int64_t j = (int64_t)o * chunk_vec + sl.v_begin + local;
         const int64_t e0 = ((int64_t)r * n_vec + j) * kVec;
         float mf[8], ms[8];
-        ld8(src_fast + e0, mf);
-        ld8(src_slow + e0, ms);
+        ld8w(src_fast + e0, mf, wide);
+        ld8w(src_slow + e0, ms, wide);
         if (own && apply) {
             float er[8];
-            ld8(e_req + j * kVec, er);
+            ld8w(e_req + j * kVec, er, wide);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 mf[i] = __fadd_rn(mf[i], __fmul_rn(k.one_m_beta_fast, er[i]));
                 ms[i] = __fadd_rn(ms[i], __fmul_rn(k.one_m_beta_slow, er[i]));
             }
         }
-        st8(dst_fast + e0, mf);
-        st8(dst_slow + e0, ms);
+        st8w(dst_fast + e0, mf, wide);
+        st8w(dst_slow + e0, ms, wide);
     }
 }
 

@@ -120,6 +120,11 @@ void reduce_b(const Bufs &b, int owners, Slab sl, cudaStream_t st, const ReduceO
 template <int G, int BITS>
 void exit_g(const ChunkSrc &src, int64_t chunk_vec, const OutPtrs &out, int n_out, int owners,
             Slab sl, cudaStream_t st) {
+    if (sl.v_count / 2 >= kExitRunMinRuns) {   // a thread per 16-element run
+        dim3 grid((unsigned)((sl.v_count / 2 + kThreads - 1) / kThreads), (unsigned)owners);
+        echo_exit_run_kernel<G, BITS><<<grid, kThreads, 0, st>>>(src, out, n_out, chunk_vec, sl);
+        return;
+    }
     dim3 grid((unsigned)((sl.v_count + kThreads - 1) / kThreads), (unsigned)owners);
     echo_exit_kernel<G, BITS><<<grid, kThreads, 0, st>>>(src, out, n_out, chunk_vec, sl);
 }

@@ -257,20 +257,7 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
 #pragma unroll
     for (int i = 0; i < 8; ++i)
         yw[i] = bf16x2_bits_rn(mul2(make_float2(k2[2 * i], k2[2 * i + 1]), sc2));
-    if (OUT) {
-#pragma unroll
-        for (int r = 0; r < kMaxRanks; ++r) {
-            if (r < n_out) {
-                uint4 *dst = out.p[r] + j * 2;
-                if (aligned32(out.p[r])) {
-                    st32_words_cs(dst, yw);
-                } else {
-                    __stcs(dst, make_uint4(yw[0], yw[1], yw[2], yw[3]));
-                    __stcs(dst + 1, make_uint4(yw[4], yw[5], yw[6], yw[7]));
-                }
-            }
-        }
-    }
+    if (OUT) store_run_outputs(out, n_out, j, yw);
     if (COMP) {
         float e[16];
 #pragma unroll
@@ -282,11 +269,12 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
         if (fix) {   // the owner's own states, this run's 16 elements
             const int64_t e0 = ((int64_t)o * n_vec + j * 2) * kVec;
             const float2 obf = splat2(k.one_m_beta_fast), obs = splat2(k.one_m_beta_slow);
+            const bool wide = aligned32(m_fast) && aligned32(m_slow);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float mf[8], ms[8];
-                ld8(m_fast + e0 + 8 * h, mf);
-                ld8(m_slow + e0 + 8 * h, ms);
+                ld8w(m_fast + e0 + 8 * h, mf, wide);
+                ld8w(m_slow + e0 + 8 * h, ms, wide);
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {
                     const float2 e2 = make_float2(e[8 * h + i], e[8 * h + i + 1]);
@@ -295,8 +283,8 @@ echo_reduce_kernel(const uint32_t *__restrict__ codes, const float *__restrict__
                     mf[i] = f.x; mf[i + 1] = f.y;
                     ms[i] = g.x; ms[i + 1] = g.y;
                 }
-                st8(m_fast + e0 + 8 * h, mf);
-                st8(m_slow + e0 + 8 * h, ms);
+                st8w(m_fast + e0 + 8 * h, mf, wide);
+                st8w(m_slow + e0 + 8 * h, ms, wide);
             }
         } else {
             store_run16(e_req, j, e);
@@ -358,11 +346,12 @@ echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ sca
         if (FIX) {
             const int64_t e0 = ((int64_t)o * n_vec + j * 2) * kVec;   // rank o's own state
             const float2 obf = splat2(k.one_m_beta_fast), obs = splat2(k.one_m_beta_slow);
+            const bool wide = aligned32(m_fast) && aligned32(m_slow);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float mf[8], ms[8];
-                ld8(m_fast + e0 + 8 * h, mf);
-                ld8(m_slow + e0 + 8 * h, ms);
+                ld8w(m_fast + e0 + 8 * h, mf, wide);
+                ld8w(m_slow + e0 + 8 * h, ms, wide);
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {
                     const float2 e2 = make_float2(e[8 * h + i], e[8 * h + i + 1]);
@@ -371,8 +360,8 @@ echo_rs_kernel(const uint32_t *__restrict__ codes, const float *__restrict__ sca
                     mf[i] = f.x; mf[i + 1] = f.y;
                     ms[i] = g.x; ms[i + 1] = g.y;
                 }
-                st8(m_fast + e0 + 8 * h, mf);
-                st8(m_slow + e0 + 8 * h, ms);
+                st8w(m_fast + e0 + 8 * h, mf, wide);
+                st8w(m_slow + e0 + 8 * h, ms, wide);
             }
         } else {
             store_run16(e_req, j, e);

@@ -423,3 +423,22 @@ def test_staged_reduce_every_element_ragged():
         chk = SequenceChecker(plan, oracle_params(plan))
         for t in range(2):
             chk.step(W.generate(w, t, DEV))
+
+
+@pytest.mark.parametrize("fixup", ["exit", "deferred"])
+def test_run_exit_every_element_ragged(fixup):
+    """The exit pass with a thread per 16-element run (owner chunks of at
+    least 2^22 elements): P=2, G=128, owner chunks of 2^22 + 128 elements,
+    so each owner's last block of 256 runs is partial (8 runs); the fix-up
+    in the reduce (32-byte state accesses) or deferred; two calls, every
+    element against the oracle."""
+    P, G = 2, 128
+    C = (1 << 22) + G
+    N = P * C
+    assert (C // 16) % 256 == 8
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    with _plan(P, N, G, True, fixup) as plan:
+        assert plan.launches_per_call() == 3
+        chk = SequenceChecker(plan, oracle_params(plan))
+        for t in range(2):
+            chk.step(W.generate(w, t, DEV))

@@ -90,6 +90,41 @@ def test_noalloc_matches_plan_two_calls(P, G, k, comp):
                             "m_slow, call %d" % t)
 
 
+@pytest.mark.parametrize("P,G,k", [(8, 128, 600), (3, 32, 41)])
+def test_noalloc_state_and_outputs_aligned_to_16_bytes_only(P, G, k):
+    """The caller's states and outputs 16 bytes past a 32-byte boundary
+    (the ABI asks for 16-byte alignment): the owner fix-up in the reduce
+    and the output stores take their 16-byte form and give the same bits
+    as the plan, two calls; with the exit pass and without."""
+    N = P * G * k
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    cfg = _cfg(P, G, N, True)
+    stream = torch.cuda.current_stream().cuda_stream
+    s2 = (4 + P * N + 7) // 8 * 8 + 4             # floats: 16 bytes past a 32-byte boundary
+    sbuf = torch.zeros(s2 + P * N, dtype=torch.float32, device=DEV)
+    mf = sbuf[4:4 + P * N].view(P, N)
+    ms = sbuf[s2:s2 + P * N].view(P, N)
+    obuf = torch.empty(P * (N + 16) + 8, dtype=torch.bfloat16, device=DEV)
+    outs = [obuf[8 + r * (N + 16):8 + r * (N + 16) + N] for r in range(P)]
+    assert mf.data_ptr() % 32 == 16 and ms.data_ptr() % 32 == 16
+    assert all(t.data_ptr() % 32 == 16 for t in outs)
+    with EchoPlan(P, N, G, compensate=True, fixup="exit", device=0) as plan:
+        for t in range(2):
+            x = W.generate(w, t, DEV)
+            want = plan.allreduce(x)
+            abi.echo_allreduce_noalloc(cfg, [x[r].data_ptr() for r in range(P)],
+                                       [o.data_ptr() for o in outs], mf.data_ptr(),
+                                       ms.data_ptr(), stream)
+            torch.cuda.synchronize()
+            _check_same(_bits(torch.stack(outs)), _bits(want), "outputs, call %d" % t)
+            pmf, pms = plan.get_state()
+            torch.cuda.synchronize()
+            _check_same(mf.cpu().numpy().view(np.uint32), pmf.cpu().numpy().view(np.uint32),
+                        "m_fast, call %d" % t)
+            _check_same(ms.cpu().numpy().view(np.uint32), pms.cpu().numpy().view(np.uint32),
+                        "m_slow, call %d" % t)
+
+
 def test_noalloc_largest_supported_and_rejected_sizes():
     """8 ranks of 2048 x 4096 with the compensator fit the fixed scratch at
     every group size; 1 GiB per rank does not and is refused before anything
