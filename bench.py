@@ -121,17 +121,6 @@ def reduce_bytes(P: int, N: int, G: int, comp: bool, fixup: str, bits: int = 4) 
     return b
 
 
-def exit_bytes(P: int, N: int, G: int, bits: int = 4) -> float:
-    """echo_exit (compensated calls): read the reduced transport, write the
-    P bf16 outputs."""
-    return N * transport_bytes_per_elem(G, bits) + P * N * 2
-
-
-# compensated calls of at most this many elements per rank have no exit
-# launch: their reduce writes the outputs (as every uncompensated call's does)
-MERGE_MAX_N = 1 << 19
-
-
 def rs_kernel_bytes(P: int, N: int, G: int, comp: bool, fixup: str, bits: int = 4) -> float:
     """Algorithmic bytes of the reduce-scatter's second kernel (echo_rs): read
     the entry transport (P*q per element of N), write each owner's bf16
@@ -147,18 +136,16 @@ def kernel_rooflines(prof: dict, P: int, N: int, G: int, comp: bool, fixup: str,
                      peak: float, rs: bool = False) -> dict:
     """Each kernel's algorithmic bytes per launch over its average launch
     time (the plan's CUDA events on the launch stream), against the HBM peak.
-    When the reduce writes the outputs (no exit launch) its bytes include
-    them; for a reduce-scatter call the second kernel is echo_rs."""
+    On one GPU the reduce writes the P outputs (there is no exit launch), so
+    its bytes include them; for a reduce-scatter call the second kernel is
+    echo_rs."""
     calls = max(int(prof["calls"]), 1)
-    merged = not comp or N <= MERGE_MAX_N
-    rb = reduce_bytes(P, N, G, comp, fixup, bits) + (P * N * 2 if comp and merged else 0)
+    rb = reduce_bytes(P, N, G, comp, fixup, bits) + (P * N * 2 if comp else 0)
     kernels = [("echo_entry", entry_bytes(P, N, G, comp, fixup, bits), "entry_ms")]
     if rs:
         kernels.append(("echo_rs", rs_kernel_bytes(P, N, G, comp, fixup, bits), "reduce_ms"))
     else:
         kernels.append(("echo_reduce", rb, "reduce_ms"))
-        if not merged:
-            kernels.append(("echo_exit", exit_bytes(P, N, G, bits), "exit_ms"))
     out = {}
     for name, b, key in kernels:
         ms = prof[key] / calls

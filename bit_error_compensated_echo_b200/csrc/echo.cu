@@ -128,23 +128,19 @@ void plan_entry(echo_plan *p, const InPtrs &x, Slab sl, cudaStream_t st, bool de
     launch_entry(p->b, x, p->cfg.P, 0, p->chunk_vec, sl, defer, st);
 }
 
-// Whether the reduce also writes every rank's output (no exit pass):
-// always uncompensated (no state traffic, the merged pass measured 6% faster
-// per call at 1 GiB per rank), and for small compensated calls.
-bool outputs_in_reduce(const echo_plan *p) {
-    return !p->cfg.compensate || p->cfg.N <= kMergeMaxN;
-}
-
-bool exit_pass(const echo_plan *p) { return !outputs_in_reduce(p); }
-
-// The reduce; fix applies the owner fix-up in it.
+// The reduce; fix applies the owner fix-up in it.  On one GPU the reduce
+// also writes every rank's output: the owner that requantizes a value
+// computes y = bf16(k2*scale2) from the requantized codes anyway, and
+// writing it to the P outputs there replaces the exit pass (re-reading the
+// reduced codes and a launch).  A/B at P = 8, G = 128, bit-identical:
+// uncompensated call at 1 GiB per rank 5.10 -> 4.80 ms when this was
+// introduced; compensated calls, once the reduce stored 32 bytes at a time,
+// 14.03 -> 13.77 ms at 1 GiB per rank, 0.883 -> 0.863 ms at 64 MiB,
+// 67.7 -> 63.5 us at 4 MiB (with 16-byte stores the separate exit pass had
+// been faster from 2 MiB per rank up).  The exit kernel remains the rank
+// path's all-gather.
 void plan_reduce(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
-    const int n_out = outputs_in_reduce(p) ? p->cfg.P : 0;
-    launch_reduce(p->b, p->cfg.P, sl, st, &out, n_out, fix);
-}
-
-void plan_exit(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st) {
-    launch_exit(p->b, out, p->cfg.P, p->cfg.P, sl, st);
+    launch_reduce(p->b, p->cfg.P, sl, st, &out, p->cfg.P, fix);
 }
 
 void plan_rs(echo_plan *p, const OutPtrs &out, Slab sl, cudaStream_t st, bool fix) {
@@ -279,7 +275,7 @@ echo_status echo_plan_destroy(echo_plan *p) {
 int32_t echo_launches_per_call(const echo_plan *p) {
     if (!p) return 0;
     const int side = (p->cfg.compensate && p->cfg.fixup == ECHO_FIXUP_SIDE) ? 1 : 0;
-    return (exit_pass(p) ? 3 : 2) + side;
+    return 2 + side;
 }
 
 echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out, void *stream,
@@ -316,7 +312,7 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
         return ECHO_ERR_UNSUPPORTED;
 
     ProfRecord rec{};
-    rec.kernels = exit_pass(p) ? 3 : 2;
+    rec.kernels = 2;
     if (p->profiling) {
         for (int i = 0; i < 6; ++i) rec.ev[i] = nullptr;
         for (int i = 0; i < 4; ++i) {
@@ -338,11 +334,7 @@ echo_status echo_allreduce(echo_plan *p, const void *const *in, void *const *out
     ECHO_TRY(cudaGetLastError());
     if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[2], st));
     if (fix_on_side && side) ECHO_TRY(cudaEventRecord(p->ev_reduced, st));
-    if (exit_pass(p)) {
-        plan_exit(p, yo, whole(p), st);
-        ECHO_TRY(cudaGetLastError());
-    }
-    if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[3], st));
+    if (p->profiling) ECHO_TRY(cudaEventRecord(rec.ev[3], st));   // no exit pass on one GPU
 
     if (fix_on_side) {
         cudaStream_t fs = side ? side : st;
@@ -512,7 +504,6 @@ echo_status echo_allreduce_host(echo_plan *p, const void *const *in_host, void *
         ECHO_TRY(cudaStreamWaitEvent(s_comp, p->hev[2 * k], 0));
         plan_entry(p, xi, sl, s_comp, defer);
         plan_reduce(p, yo, sl, s_comp, comp && !deferred);
-        if (exit_pass(p)) plan_exit(p, yo, sl, s_comp);
         ECHO_TRY(cudaGetLastError());
         ECHO_TRY(cudaEventRecord(p->hev[2 * k + 1], s_comp));
         ECHO_TRY(cudaStreamWaitEvent(s_out, p->hev[2 * k + 1], 0));

@@ -144,9 +144,9 @@ echo_status echo_plan_destroy(echo_plan *plan);
  *   in_device[r]  : bf16, N contiguous elements of rank r (read)
  *   out_device[r] : bf16, N contiguous elements (written with y); may equal
  *                   in_device[r] (in-place)
- *   stream        : stream the entry, reduce and exit kernels run on
- *                   (uncompensated, or compensated with N <= 2^19, the
- *                   reduce writes the outputs and there is no exit pass)
+ *   stream        : stream the entry and reduce kernels run on (on one
+ *                   GPU the reduce writes the outputs: there is no exit
+ *                   pass; the rank path's exit kernel is the all-gather)
  *   side_stream   : used with ECHO_FIXUP_SIDE only (the owner fix-up runs
  *                   there after an event on stream); NULL runs the fix-up
  *                   on stream.  Ignored by the other modes.
@@ -255,9 +255,9 @@ typedef struct echo_profile {
     int64_t calls;          /* calls recorded */
     double entry_ms;        /* total time of echo_entry launches */
     double reduce_ms;       /* total time of echo_reduce launches */
-    double exit_ms;         /* total time of echo_exit launches (0 when the
-                             * reduce writes the outputs: uncompensated
-                             * calls, compensated calls with N <= 2^19) */
+    double exit_ms;         /* total time of echo_exit launches: 0, since
+                             * a plan's reduce writes the outputs (kept for
+                             * the layout of this struct) */
     double fixup_ms;        /* total time of side-stream fix-up launches */
     int64_t launches;       /* kernels launched by the recorded calls */
 } echo_profile;

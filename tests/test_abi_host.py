@@ -202,16 +202,16 @@ def test_cross_rank_aggregation_gloo():
 
 def test_bench_kernel_rooflines():
     """Per-kernel roofline fractions of the bench line: the algorithmic bytes
-    of each kernel over its average launch time; a reduce that writes the
-    outputs (no exit launch) counts them."""
+    of each kernel over its average launch time; the reduce writes the
+    outputs (there is no exit launch on one GPU) and counts them."""
     import bench
     P, N, G = 8, 1 << 29, 128
-    prof = {"calls": 10, "entry_ms": 117.0, "reduce_ms": 10.0, "exit_ms": 13.8, "fixup_ms": 0.0}
+    prof = {"calls": 10, "entry_ms": 117.0, "reduce_ms": 20.0, "exit_ms": 0.0028, "fixup_ms": 0.0}
     r = bench.kernel_rooflines(prof, P, N, G, True, "deferred", 4, 6543.4)
     q = 0.5 + 4 / 128
+    assert set(r) == {"echo_entry", "echo_reduce"}
     assert r["echo_entry"]["bytes"] == P * N * (18 + q) + 4 * N
-    assert r["echo_reduce"]["bytes"] == P * N * q + N * q + 4 * N
-    assert r["echo_exit"]["bytes"] == N * q + 2 * P * N
+    assert r["echo_reduce"]["bytes"] == P * N * q + N * q + 4 * N + 2 * P * N
     for k in r.values():
         assert abs(k["achieved"] - k["bytes"] / (k["avg_launch_ms"] / 1e3) / 1e9) < 0.1
         assert abs(k["frac"] - k["achieved"] / 6543.4) < 1e-3

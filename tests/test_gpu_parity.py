@@ -311,8 +311,7 @@ def test_profile_counts_launches(N):
     w = W.with_size(W.TINY, P=2, rows=1, hidden=N, G=32)
     side = torch.cuda.Stream()
     for comp, mode in ((True, "exit"), (True, "side"), (True, "deferred"), (False, "exit")):
-        exit_pass = comp and N > (1 << 19)
-        per = 2 + int(exit_pass) + int(comp and mode == "side")
+        per = 2 + int(comp and mode == "side")   # on one GPU the reduce writes the outputs
         with _plan(w.P, w.N, w.G, comp, mode) as plan:
             assert plan.launches_per_call() == per
             plan.profile_enable(True)
@@ -321,8 +320,6 @@ def test_profile_counts_launches(N):
             p = plan.profile_read(reset=True)
             assert p["calls"] == 3 and p["launches"] == 3 * per
             assert p["entry_ms"] > 0 and p["reduce_ms"] > 0
-            if exit_pass:
-                assert p["exit_ms"] > 0
 
 
 def test_argument_errors_on_device():
@@ -424,21 +421,3 @@ def test_staged_reduce_every_element_ragged():
         for t in range(2):
             chk.step(W.generate(w, t, DEV))
 
-
-@pytest.mark.parametrize("fixup", ["exit", "deferred"])
-def test_run_exit_every_element_ragged(fixup):
-    """The exit pass with a thread per 16-element run (owner chunks of at
-    least 2^22 elements): P=2, G=128, owner chunks of 2^22 + 128 elements,
-    so each owner's last block of 256 runs is partial (8 runs); the fix-up
-    in the reduce (32-byte state accesses) or deferred; two calls, every
-    element against the oracle."""
-    P, G = 2, 128
-    C = (1 << 22) + G
-    N = P * C
-    assert (C // 16) % 256 == 8
-    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
-    with _plan(P, N, G, True, fixup) as plan:
-        assert plan.launches_per_call() == 3
-        chk = SequenceChecker(plan, oracle_params(plan))
-        for t in range(2):
-            chk.step(W.generate(w, t, DEV))

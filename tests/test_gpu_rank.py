@@ -231,3 +231,36 @@ def test_rank_reduce_scatter_staged_size_against_oracle(transport):
             assert_same("m_slow", _f32(gms.index_select(1, idx)), ms, "f32", t)
             del gmf, gms
     assert C >= 1 << 20
+
+
+@pytest.mark.parametrize("transport", ["copies", "peers"])
+@pytest.mark.parametrize("fixup", ["exit", "deferred"])
+def test_rank_run_exit_every_element_ragged(transport, fixup):
+    """The all-gather kernel with a thread per 16-element run (owner chunks of
+    at least 2^22 elements): P=2 ranks, owner chunks of 2^22 + 128
+    elements, so each owner's last block of 256 runs is partial (8 runs);
+    the fix-up in the reduce (32-byte state accesses) or deferred; two
+    all-reduce calls of the rank group, every element of every rank's
+    output and both states against the oracle."""
+    from rank_emulation import EmulatedPeerGroup
+    P, G = 2, 128
+    C = (1 << 22) + G
+    N = P * C
+    assert (C // 16) % 256 == 8
+    w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
+    prm = oracle.Params(P=P, N=N, G=G, compensate=True)
+    mf = np.zeros((P, N), np.float32)
+    ms = np.zeros_like(mf)
+    group = EmulatedGroup if transport == "copies" else EmulatedPeerGroup
+    with group(P, N, G, fixup=fixup) as grp:
+        for t in range(2):
+            x = W.generate(w, t, DEV)
+            y = grp.allreduce(x)
+            torch.cuda.synchronize()
+            ref = oracle.allreduce(prm, _bits_u16(x), mf, ms)
+            yb = _bits_u16(y)
+            assert_same("outputs", yb, np.broadcast_to(ref.y, yb.shape), "bf16", t)
+            gmf, gms = grp.get_state()
+            assert_same("m_fast", _f32(gmf), mf, "f32", t)
+            assert_same("m_slow", _f32(gms), ms, "f32", t)
+            del gmf, gms
