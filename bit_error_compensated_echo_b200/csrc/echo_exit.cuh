@@ -1,4 +1,4 @@
-// echo_exit.cuh -- the all-gather half: dequantize to bf16, owner fix-up
+// echo_exit.cuh -- the all-gather half: dequantize the reduced chunks to bf16
 // (operation: include/echo.h; conventions: echo_common.cuh)
 #pragma once
 
@@ -12,8 +12,10 @@ namespace echo {
 // to n_out outputs (all P ranks' on one GPU, this process's one across
 // GPUs).  Owner o's reduced chunk is read from src.codes[o] / src.scales[o]
 // (ChunkSrc): one local buffer, or, on the rank path, owner o's own buffer
-// on its GPU, so that the all-gather is these loads.  Uncompensated calls
-// on one GPU skip the kernel: their reduce writes the outputs itself.
+// on its GPU, so that the all-gather is these loads.  Calls on one GPU
+// skip the kernel: their reduce writes the outputs itself (plan_reduce);
+// the rank path and the allocation-free call above 2^19 elements per rank
+// launch it.
 // Grid: x over the vectors of the slab, y = owner.
 template <int G, int BITS>
 __global__ void __launch_bounds__(kThreads)
@@ -42,10 +44,11 @@ echo_exit_kernel(const __grid_constant__ ChunkSrc src, const __grid_constant__ O
 
 // The same pass with a thread per 16-element run: 8 (16) bytes of codes, 16
 // bf16 values, and one 32-byte store per output (store_run_outputs).  Half
-// as many threads as the kernel above, so it pays only on large slabs: at
-// 1 GiB per rank (P = 8, G = 128) 1.377 -> 1.330 ms, at 64 MiB per rank the
-// call within 0.2 %, at 16 MiB 1 % slower and at the Llama shape (1 Mi
-// elements per owner) 7 % slower.  The launcher takes it from
+// as many threads as the kernel above, so it pays only on large slabs
+// (measured with P outputs, while one GPU's compensated calls still ran this
+// pass: at 1 GiB per rank, P = 8, G = 128, 1.377 -> 1.330 ms; at 64 MiB per
+// rank the call within 0.2 %, at 16 MiB 1 % slower and at the Llama shape,
+// 1 Mi elements per owner, 7 % slower).  The launcher takes it from
 // kExitRunMinRuns runs per owner chunk in the slab.
 // Grid: x over the 16-element runs of the slab, y = owner.
 constexpr int64_t kExitRunMinRuns = int64_t(1) << 18;   // 2^22 elements per owner

@@ -12,9 +12,10 @@ namespace echo {
 // Reduce-scatter half: for every element, dequantize the P ranks' codes,
 // sum them in fp32 in ascending rank order from +0, requantize the sum and
 // pack it (the reduced transport).  The dequantized sum y = bf16(k2*scale2)
-// is what every rank receives, so on one GPU the kernel can also write it to
+// is what every rank receives, so on one GPU the kernel also writes it to
 // the n_out outputs itself (OUT), with no second pass over the reduced
-// codes; without OUT that is the exit kernel's job.  Compensating, the
+// codes; without OUT (the rank path) that is the exit kernel's job.
+// Compensating, the
 // output residual e_req = s - float(y) is either
 // written out (for a side-stream or deferred fix-up) or, with fix, folded
 // into the owner's states here (state row o, the owner's own chunk).
