@@ -44,12 +44,15 @@ echo_exit_kernel(const __grid_constant__ ChunkSrc src, const __grid_constant__ O
 
 // The same pass with a thread per 16-element run: 8 (16) bytes of codes, 16
 // bf16 values, and one 32-byte store per output (store_run_outputs).  Half
-// as many threads as the kernel above, so it pays only on large slabs
-// (measured with P outputs, while one GPU's compensated calls still ran this
-// pass: at 1 GiB per rank, P = 8, G = 128, 1.377 -> 1.330 ms; at 64 MiB per
-// rank the call within 0.2 %, at 16 MiB 1 % slower and at the Llama shape,
-// 1 Mi elements per owner, 7 % slower).  The launcher takes it from
-// kExitRunMinRuns runs per owner chunk in the slab.
+// as many threads as the kernel above, so it pays only on large slabs.
+// With P = 8 outputs per thread (measured while one GPU's compensated calls
+// still ran this pass, G = 128): 1.377 -> 1.330 ms at 1 GiB per rank; the
+// call within 0.2 % at 64 MiB per rank, 1 % slower at 16 MiB, 7 % slower at
+// the Llama shape (1 Mi elements per owner).  With one output (a rank of
+// the rank path, P = 8): 0.283 -> 0.209 ms at 2^29 elements per rank, 0.074
+// -> 0.056 ms at 2^27, 16.8 -> 14.7 us at 2^25; at 2^23 and below both take
+// 4-6 us, bound by the launch.  The launcher takes it from kExitRunMinRuns
+// runs per owner chunk in the slab.
 // Grid: x over the 16-element runs of the slab, y = owner.
 constexpr int64_t kExitRunMinRuns = int64_t(1) << 18;   // 2^22 elements per owner
 
