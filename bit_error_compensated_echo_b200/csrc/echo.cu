@@ -3,10 +3,10 @@
 // A plan owns one device allocation carved into the EMA states, the entry
 // transport (packed codes + scales of all P ranks: the 4-bit "wire" of the
 // reduce-scatter), the reduced transport (the wire of the all-gather) and
-// e_req.  A call launches entry, reduce and exit on the caller's stream --
-// uncompensated, or compensated with N <= 2^19, the reduce writes every
-// rank's output itself and there is no exit pass -- plus, in side-stream
-// mode, the owner fix-up on the side stream.  Host code here only validates, carves memory, orders streams and
+// e_req.  A call launches the entry and the reduce on the caller's stream
+// (the reduce writes every rank's output itself: there is no exit pass on
+// one GPU), plus, in side-stream mode, the owner fix-up on the side stream.
+// Host code here only validates, carves memory, orders streams and
 // launches: every step of the arithmetic runs in the kernels of echo_*.cuh.
 #include <cuda_runtime.h>
 

@@ -13,9 +13,8 @@ namespace echo {
 // GPUs).  Owner o's reduced chunk is read from src.codes[o] / src.scales[o]
 // (ChunkSrc): one local buffer, or, on the rank path, owner o's own buffer
 // on its GPU, so that the all-gather is these loads.  Calls on one GPU
-// skip the kernel: their reduce writes the outputs itself (plan_reduce);
-// the rank path and the allocation-free call above 2^19 elements per rank
-// launch it.
+// skip the kernel: their reduce writes the outputs itself; the rank path
+// launches it.
 // Grid: x over the vectors of the slab, y = owner.
 template <int G, int BITS>
 __global__ void __launch_bounds__(kThreads)

@@ -66,14 +66,6 @@ void launch_entry(const Bufs &b, const InPtrs &x, int rows, int rank0, int64_t e
 ChunkDst chunks_of(const Bufs &b);
 ChunkSrc reduced_chunks_of(const Bufs &b);
 
-// The allocation-free call (echo_allreduce_noalloc) lets its reduce write
-// the outputs for compensated calls of at most this many elements per rank
-// (1 MiB of bf16) and runs an exit pass above it, the rule measured best
-// when its reduce still wrote 16 bytes at a time.  A plan's calls on one GPU
-// always write the outputs in the reduce (plan_reduce); both give the same
-// bits.
-constexpr int64_t kMergeMaxN = int64_t(1) << 19;
-
 // Reduce of `owners` chunks (grid y): sum the P rows, requantize; with
 // n_out > 0 also write the dequantized sum to the n_out outputs (else that
 // is launch_exit's job); compensating, either write e_req or, with fix,

@@ -141,12 +141,9 @@ void launch_all(const InPtrs &x, const OutPtrs &y, float *mf, float *ms, unsigne
     b.k = make_consts(c);
     const Slab sl{0, b.chunk_vec};
     launch_entry(b, x, c.P, 0, b.chunk_vec, sl, false, st);
-    if (b.comp && c.N > kMergeMaxN) {   // owner fix-up in the reduce, outputs in the exit
-        launch_reduce(b, c.P, sl, st, nullptr, 0, true);
-        launch_exit(b, y, c.P, c.P, sl, st);
-    } else {                            // the reduce writes the outputs
-        launch_reduce(b, c.P, sl, st, &y, c.P, b.comp);
-    }
+    // the reduce writes the outputs and, compensating, applies the owner
+    // fix-up (as a plan's calls on one GPU do)
+    launch_reduce(b, c.P, sl, st, &y, c.P, b.comp);
 }
 
 }  // namespace

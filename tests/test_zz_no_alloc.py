@@ -57,8 +57,9 @@ def scratch_bytes(P, N, G, comp):
     return need + (r(N * 4) if comp else 0)
 
 
-# N above and below 2^19 per rank: the call with and without the exit pass;
-# the last case (8 ranks of 2048 x 4096, G = 32) needs 77 MiB of the 80 MiB
+# small and large N per rank, all four code paths of the reduce (with and
+# without the compensator and the fix-up); the last case (8 ranks of
+# 2048 x 4096, G = 32) needs 77 MiB of the 80 MiB
 @pytest.mark.parametrize("P,G,k,comp", [(8, 128, 70, True), (3, 32, 41, True),
                                         (4, 64, 33, False), (8, 128, 600, True),
                                         (8, 32, 32768, True)])
@@ -95,7 +96,7 @@ def test_noalloc_state_and_outputs_aligned_to_16_bytes_only(P, G, k):
     """The caller's states and outputs 16 bytes past a 32-byte boundary
     (the ABI asks for 16-byte alignment): the owner fix-up in the reduce
     and the output stores take their 16-byte form and give the same bits
-    as the plan, two calls; with the exit pass and without."""
+    as the plan, two calls; a large and a small N."""
     N = P * G * k
     w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
     cfg = _cfg(P, G, N, True)
