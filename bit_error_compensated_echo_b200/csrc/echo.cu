@@ -65,7 +65,8 @@ Layout layout_of(const echo_config &c) {
 constexpr int kHostSlabs = 32;
 
 struct ProfRecord {
-    cudaEvent_t ev[6];   // entry start, entry end, reduce end, exit end, fixup start, fixup end
+    cudaEvent_t ev[6];   // entry start, entry end, reduce end, call end (no exit pass on one
+                         // GPU: exit_ms stays ~0), fixup start, fixup end
     bool side;
     int kernels;         // kernels on the main stream
 };
