@@ -233,26 +233,29 @@ def test_rank_reduce_scatter_staged_size_against_oracle(transport):
     assert C >= 1 << 20
 
 
-@pytest.mark.parametrize("transport", ["copies", "peers"])
-@pytest.mark.parametrize("fixup", ["exit", "deferred"])
-def test_rank_run_exit_every_element_ragged(transport, fixup):
+@pytest.mark.parametrize("transport,fixup,bits", [("copies", "exit", 4), ("peers", "exit", 4),
+                                                  ("copies", "deferred", 4),
+                                                  ("peers", "deferred", 4),
+                                                  ("copies", "deferred", 8),
+                                                  ("peers", "exit", 8)])
+def test_rank_run_exit_every_element_ragged(transport, fixup, bits):
     """The all-gather kernel with a thread per 16-element run (owner chunks of
     at least 2^22 elements): P=2 ranks, owner chunks of 2^22 + 128
     elements, so each owner's last block of 256 runs is partial (8 runs);
-    the fix-up in the reduce (32-byte state accesses) or deferred; two
-    all-reduce calls of the rank group, every element of every rank's
-    output and both states against the oracle."""
+    the fix-up in the reduce (32-byte state accesses) or deferred; 4- and
+    8-bit codes; two all-reduce calls of the rank group, every element of
+    every rank's output and both states against the oracle."""
     from rank_emulation import EmulatedPeerGroup
     P, G = 2, 128
     C = (1 << 22) + G
     N = P * C
     assert (C // 16) % 256 == 8
     w = W.with_size(W.TINY, P=P, rows=1, hidden=N, G=G)
-    prm = oracle.Params(P=P, N=N, G=G, compensate=True)
+    prm = oracle.Params(P=P, N=N, G=G, compensate=True, bits=bits)
     mf = np.zeros((P, N), np.float32)
     ms = np.zeros_like(mf)
     group = EmulatedGroup if transport == "copies" else EmulatedPeerGroup
-    with group(P, N, G, fixup=fixup) as grp:
+    with group(P, N, G, fixup=fixup, bits=bits) as grp:
         for t in range(2):
             x = W.generate(w, t, DEV)
             y = grp.allreduce(x)
