@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload large|llama|depth|tiny] [--fixup exit|side|deferred]
-                    [--uncompensated] [--mode step|sweep|overlap|depth-chain|group]
+                    [--uncompensated] [--mode step|sweep|overlap|depth-chain|group|rank-stages]
 
 Default (mode "step"): one step = one echo_allreduce call (entry kernel, then
 the reduce kernel that also writes every rank's output) of P=8 virtual ranks
@@ -25,6 +25,9 @@ form ONE Echo group (P = N real ranks, one GPU each, the workload's N
 elements per rank), the two exchanges go over NCCL, and the line compares
 the call with NCCL's bf16 all-reduce of the same tensors (max over ranks of
 CUDA-event times).  With one GPU it runs a one-rank group.
+
+--mode rank-stages times the rank path's three stage kernels for P ranks
+emulated on one GPU (the fused transport inside one process, no NVLink).
 
 --impl reference times the CPU oracle on bounded samples of the same
 workload (rank 0 only) and prints the same JSON line with "impl":
@@ -699,6 +702,78 @@ def run_sweep_mode(args, ws, rank, local):
                     r["copy_gbs"], 100 * r["frac_of_copy"], r["packed_ratio"]))
 
 
+def run_rank_stages_mode(args, ws, rank, local):
+    """The rank path's stage kernels for the workload's P ranks on this one
+    GPU: P rank plans in one process whose entries store into each other's
+    windows and whose exits load from them (PeerWindows.in_process, the
+    fused transport without NVLink), stage by stage, so no kernel waits on
+    another.  Per step: echo_rank_entry_peers of every rank, echo_rank_reduce
+    of every owner, echo_rank_exit_peers of every rank, CUDA events between
+    the stages.  Prints the stages' times (all ranks' work per call) and
+    their algorithmic bytes over time against the measured copy rate."""
+    from bit_error_compensated_echo_b200.rank import EchoRankPlan, PeerWindows
+    if rank != 0:
+        return
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    P, N, G, bits = w.P, w.N, w.G, args.bits
+    comp = not args.uncompensated
+    peak, peak_kind = load_peaks()
+    x = W.generate(w, 0, dev)
+    out = torch.empty_like(x)
+    plans = [EchoRankPlan(P, r, N, G, compensate=comp, fixup=args.fixup, device=local, bits=bits)
+             for r in range(P)]
+    try:
+        wins = PeerWindows.in_process(plans)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+        def step():
+            ev[0].record()
+            for r, (p, win) in enumerate(zip(plans, wins)):
+                p.entry_peers(x[r], win)
+            ev[1].record()
+            for p, win in zip(plans, wins):
+                p.reduce_window(win)
+            ev[2].record()
+            for r, (p, win) in enumerate(zip(plans, wins)):
+                p.exit_peers(win, out[r])
+            ev[3].record()
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize()
+        tot = [0.0, 0.0, 0.0]
+        for _ in range(args.steps):
+            step()
+            torch.cuda.synchronize()
+            for i in range(3):
+                tot[i] += ev[i].elapsed_time(ev[i + 1])
+        t = [v / args.steps for v in tot]
+        q = transport_bytes_per_elem(G, bits)
+        stage_bytes = {
+            "entry_peers": entry_bytes(P, N, G, comp, args.fixup, bits),
+            # the owner reads P received chunks and writes its reduced chunk, no outputs
+            "reduce": N * (P * q + q) + (N * (16 if args.fixup == "exit" else 4) if comp else 0),
+            # every rank reads every owner's reduced chunk and writes its own output
+            "exit_peers": P * N * (q + 2),
+        }
+        stages = {}
+        for (name, b), ms in zip(stage_bytes.items(), t):
+            gbs = b / (ms / 1e3) / 1e9
+            stages[name] = {"ms": round(ms, 4), "bytes": b, "achieved_gbs": round(gbs, 1),
+                            "frac": round(gbs / peak, 4)}
+        print(json.dumps({"mode": "rank-stages", "workload": w.name, "P": P, "N_per_rank": N,
+                          "G": G, "bits": bits, "compensate": comp, "fixup": args.fixup,
+                          "steps": args.steps, "stages_all_ranks": stages,
+                          "call_ms_all_ranks": round(sum(t), 4), "peak_gbs": peak,
+                          "peak_kind": peak_kind,
+                          "note": "P ranks' plans on one GPU, fused transport in one process "
+                                  "(no NVLink); each stage timed over all ranks"}), flush=True)
+    finally:
+        for p in plans:
+            p.close()
+
+
 def run_overlap_mode(args, ws, rank, local):
     """1 GiB per rank, P=8: the stand-in next matmul (bf16 8192^3) after each
     call, with the owner fix-up in the reduce kernel, on a side stream beside
@@ -935,7 +1010,8 @@ def main(argv=None):
     ap.add_argument("--uncompensated", action="store_true")
     ap.add_argument("--op", choices=("all-reduce", "reduce-scatter"), default="all-reduce")
     ap.add_argument("--bits", type=int, choices=(4, 8), default=4)
-    ap.add_argument("--mode", choices=("step", "depth-chain", "sweep", "overlap", "group", "cpu"),
+    ap.add_argument("--mode", choices=("step", "depth-chain", "sweep", "overlap", "group",
+                                       "rank-stages", "cpu"),
                     default="step")
     ap.add_argument("--sweep-max-mib", type=int, default=0,
                     help="sweep only points up to this many MiB per rank (0: all)")
@@ -968,6 +1044,8 @@ def main(argv=None):
             run_overlap_mode(args, ws, rank, local)
         elif args.mode == "group":
             run_group_mode(args, ws, rank, local)
+        elif args.mode == "rank-stages":
+            run_rank_stages_mode(args, ws, rank, local)
         elif args.mode == "cpu":
             run_cpu_mode(args, ws, rank, local)
         else:
